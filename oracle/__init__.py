@@ -1,0 +1,130 @@
+"""fp64 CPU oracle for the Gated DeltaNet-2 recurrence (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library in
+``gated_delta_rule_92_b200`` and its binding) never imports it, and this
+package never imports the product path.
+
+The arithmetic lives in ``gdn2_oracle.c``: the per-token recurrence of the
+burn-gdn2 README, section "Architecture",
+``S_t = (I - k_t (b_t . k_t)^T) diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T``,
+``o_t = S_t^T q_t``, evaluated in double precision.  This module only
+compiles it (gcc, OpenMP) and marshals numpy arrays into it.
+
+Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
+an explicit d_k x d_k matrix brute force, the linear-attention and
+gated-linear-attention closed forms, separately written KDA and Gated DeltaNet
+recurrences, a hand-derived worked example, and invariants (delta-write,
+state split, linearity, w/v symmetry).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn2_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``gdn2_oracle.c`` into ``liboracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+    return _LIB
+
+
+def open_library(path: str):
+    """Open a compiled oracle library and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.gdn2_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, P,
+                                        I, I, I, I, I, P, I, I]
+    lib.gdn2_oracle_forward.restype = I
+    lib.gdn2_oracle_max_threads.restype = I
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = open_library(_LIB)
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().gdn2_oracle_max_threads())
+
+
+def _f32(x) -> np.ndarray:
+    if hasattr(x, "detach"):            # a torch tensor (bf16 has no numpy dtype)
+        x = x.detach().float().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
+            want_state: bool = True, want_smax: bool = False, lib=None):
+    """Run the recurrence in fp64.
+
+    q, k, log_alpha, b : [B, T, H, d_k];  v, w : [B, T, H, d_v] (any float
+    dtype; values are taken as float32, which holds bf16 values exactly).
+    S0 : [B, H, d_k, d_v] or None (zeros).  heads : iterable of flat b*H+h
+    indices, or None for all.  Returns (o, S_T[, smax]) with
+    o : [n_heads, T, d_v] and S_T : [n_heads, d_k, d_v] (float64), heads in
+    the order requested.
+    """
+    q, k, v, la, b, w = (_f32(x) for x in (q, k, v, log_alpha, b, w))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for x in (k, la, b):
+        assert x.shape == (B, T, H, dk), x.shape
+    for x in (v, w):
+        assert x.shape == (B, T, H, dv), x.shape
+    s0 = None
+    if S0 is not None:
+        if hasattr(S0, "detach"):
+            S0 = S0.detach().double().cpu().numpy()
+        s0 = np.ascontiguousarray(np.asarray(S0, dtype=np.float64))
+        assert s0.shape == (B, H, dk, dv), s0.shape
+    if heads is None:
+        hl = None
+        nh = B * H
+    else:
+        hl = np.ascontiguousarray(np.asarray(list(heads), dtype=np.int32))
+        nh = int(hl.size)
+    o = np.empty((nh, T, dv), dtype=np.float64)
+    st = np.empty((nh, dk, dv), dtype=np.float64) if want_state else None
+    sm = np.empty((nh,), dtype=np.float64) if want_smax else None
+    rc = (lib or _load()).gdn2_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w),
+                                     _ptr(s0), _ptr(o), _ptr(st), _ptr(sm),
+                                     B, T, H, dk, dv, _ptr(hl), nh, int(n_threads))
+    if rc != 0:
+        raise ValueError("gdn2 oracle rejected its arguments")
+    if want_smax:
+        return o, st, sm
+    return o, st
+
+
+def decode_steps(q, k, v, log_alpha, b, w, S0, heads=None, n_threads: int = 0):
+    """Token-by-token decode over a step axis.
+
+    Inputs are [steps, B, H, d] (one token per step and sequence), S0 is
+    [B, H, d_k, d_v].  Returns (o [n_heads, steps, d_v], S [n_heads, d_k, d_v]).
+    Decode is the same recurrence run one token at a time, so this is the
+    forward pass with the step axis taken as time.
+    """
+    def tb(x):
+        return np.ascontiguousarray(np.swapaxes(_f32(x), 0, 1))
+    return forward(tb(q), tb(k), tb(v), tb(log_alpha), tb(b), tb(w), S0=S0,
+                   heads=heads, n_threads=n_threads)

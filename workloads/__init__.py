@@ -1,0 +1,158 @@
+"""Seeded synthetic inputs for the Gated DeltaNet-2 mixer.
+
+This module only draws random numbers and casts them; it holds none of the
+recurrence's arithmetic, so both the CUDA path's tests and the fp64 oracle can
+take their inputs from here without sharing method code.
+
+Workloads (sizes follow the burn-gdn2 README "Configuration" table: 16 heads,
+head_dim 128, hidden 2048 by default, chunk 64):
+
+  chunk_f32_small   B1 T256  H4  d_k=d_v=64   fp32 I/O, S0 = 0
+  chunk_bf16_small  B1 T1024 H4  d_k=d_v=64   bf16 I/O, S0 ~ N(0, 0.02)
+  chunk_bf16_h2048  B8 T4096 H16 d_k=d_v=128  bf16 I/O, S0 = 0
+  chunk_bf16_negeig B4 T8192 H16 d_k=128 d_v=256, bf16, b in (0,2),
+                    alpha in [0.8, 0.9999], S0 ~ N(0, 0.02)
+  decode_bf16       256 sequences x H16 x d128, one token per step,
+                    1024 steps, S0 ~ N(0, 0.02)
+
+Recipe (every workload): a CPU ``torch.Generator`` seeded with
+``1000 + index``; draw order q, k, v, alpha, b, w, S0.  q and k are N(0,1)
+then L2-normalised over d_k per (b, t, h) in fp32 before the cast (the README
+puts an L2-norm in front of the mixer); v ~ N(0,1); alpha ~ U[lo, hi] i.i.d.
+per (b, t, h, key channel) and log_alpha = ln(alpha); b = scale * sigmoid(N(0,1))
+per key channel (scale 2 when negative eigenvalues are allowed, "b x 2" in the
+README table); w = sigmoid(N(0,1)) per value channel; S0 ~ N(0, std) in fp32.
+Token tensors are then cast to the I/O dtype; the oracle reads the cast values.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    index: int
+    name: str
+    B: int
+    T: int
+    H: int
+    d_k: int
+    d_v: int
+    io: str                    # "f32" or "bf16"
+    chunk: int = 64
+    alpha_lo: float = 0.9
+    alpha_hi: float = 0.999
+    b_scale: float = 1.0
+    s0_std: Optional[float] = None
+    decode_steps: int = 0      # > 0: decode workload (T is 1 per step)
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def seed(self) -> int:
+        return 1000 + self.index
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.io == "f32" else torch.bfloat16
+
+    def describe(self) -> str:
+        if self.decode_steps:
+            return (f"decode B{self.B} H{self.H} d_k{self.d_k} d_v{self.d_v} "
+                    f"{self.io} steps{self.decode_steps}")
+        return (f"chunk_fwd B{self.B} T{self.T} H{self.H} d_k{self.d_k} d_v{self.d_v} "
+                f"chunk{self.chunk} {self.io}")
+
+
+WORKLOADS = [
+    Workload(0, "chunk_f32_small", B=1, T=256, H=4, d_k=64, d_v=64, io="f32"),
+    Workload(1, "chunk_bf16_small", B=1, T=1024, H=4, d_k=64, d_v=64, io="bf16", s0_std=0.02),
+    Workload(2, "chunk_bf16_h2048", B=8, T=4096, H=16, d_k=128, d_v=128, io="bf16"),
+    Workload(3, "chunk_bf16_negeig", B=4, T=8192, H=16, d_k=128, d_v=256, io="bf16",
+             alpha_lo=0.8, alpha_hi=0.9999, b_scale=2.0, s0_std=0.02),
+    Workload(4, "decode_bf16", B=256, T=1, H=16, d_k=128, d_v=128, io="bf16",
+             s0_std=0.02, decode_steps=1024),
+]
+BY_NAME = {w.name: w for w in WORKLOADS}
+
+
+def _l2n(x: torch.Tensor) -> torch.Tensor:
+    return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-30)
+
+
+def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
+         dtype=torch.bfloat16, alpha_lo: float = 0.9, alpha_hi: float = 0.999,
+         b_scale: float = 1.0, s0_std: Optional[float] = None,
+         generator: Optional[torch.Generator] = None) -> dict:
+    """Draw one batch of token inputs [B, T, H, d] (CPU tensors).
+
+    Returns a dict with q, k, v, log_alpha, b, w in ``dtype`` and S0 (fp32
+    [B, H, d_k, d_v] or None).
+    """
+    g = generator if generator is not None else torch.Generator().manual_seed(seed)
+    f32 = torch.float32
+    q = _l2n(torch.randn(B, T, H, d_k, generator=g, dtype=f32))
+    k = _l2n(torch.randn(B, T, H, d_k, generator=g, dtype=f32))
+    v = torch.randn(B, T, H, d_v, generator=g, dtype=f32)
+    alpha = torch.empty(B, T, H, d_k, dtype=f32).uniform_(alpha_lo, alpha_hi, generator=g)
+    b = b_scale * torch.sigmoid(torch.randn(B, T, H, d_k, generator=g, dtype=f32))
+    w = torch.sigmoid(torch.randn(B, T, H, d_v, generator=g, dtype=f32))
+    S0 = None
+    if s0_std is not None:
+        S0 = s0_std * torch.randn(B, H, d_k, d_v, generator=g, dtype=f32)
+    out = dict(q=q, k=k, v=v, log_alpha=torch.log(alpha), b=b, w=w)
+    out = {n: t.to(dtype).contiguous() for n, t in out.items()}
+    out["S0"] = S0
+    return out
+
+
+def make_chunk_inputs(wl: Workload, *, B: Optional[int] = None, T: Optional[int] = None,
+                      H: Optional[int] = None, seed: Optional[int] = None) -> dict:
+    """Inputs of a chunk workload (optionally resized, same recipe)."""
+    return draw(B or wl.B, T or wl.T, H or wl.H, wl.d_k, wl.d_v,
+                seed=wl.seed if seed is None else seed, dtype=wl.torch_dtype,
+                alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, b_scale=wl.b_scale,
+                s0_std=wl.s0_std)
+
+
+def make_decode_inputs(wl: Workload, steps: int, *, B: Optional[int] = None,
+                       seed: Optional[int] = None) -> dict:
+    """Decode inputs: token tensors [steps, B, H, d] and S0 [B, H, d_k, d_v].
+
+    Drawn as a [B, steps, H, d] batch with the same recipe, then laid out with
+    the step axis first so that step s is one contiguous [B, H, d] slab.
+    """
+    Bn = B or wl.B
+    d = draw(Bn, steps, wl.H, wl.d_k, wl.d_v, seed=wl.seed if seed is None else seed,
+             dtype=wl.torch_dtype, alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi,
+             b_scale=wl.b_scale, s0_std=wl.s0_std)
+    for n in ("q", "k", "v", "log_alpha", "b", "w"):
+        d[n] = d[n].transpose(0, 1).contiguous()
+    return d
+
+
+def kda_collapse(inp: dict, seed: int, b_scale: float = 1.0) -> dict:
+    """Same inputs with b and w replaced by one scalar beta per (b, t, h).
+
+    beta is drawn with the workload's b recipe (b_scale * sigmoid(N(0,1))) and
+    broadcast over d_k (for b) and over d_v (for w).
+    """
+    g = torch.Generator().manual_seed(seed)
+    q = inp["q"]
+    B, T, H, dk = q.shape
+    dv = inp["v"].shape[-1]
+    beta = b_scale * torch.sigmoid(torch.randn(B, T, H, 1, generator=g, dtype=torch.float32))
+    out = dict(inp)
+    out["b"] = beta.expand(B, T, H, dk).to(q.dtype).contiguous()
+    out["w"] = beta.expand(B, T, H, dv).to(q.dtype).contiguous()
+    return out
+
+
+def gdn_collapse(inp: dict, seed: int, b_scale: float = 1.0) -> dict:
+    """KDA collapse plus a scalar decay per (b, t, h): channel 0 broadcast."""
+    out = kda_collapse(inp, seed, b_scale)
+    la = inp["log_alpha"]
+    out["log_alpha"] = la[..., :1].expand_as(la).contiguous()
+    return out
