@@ -1,0 +1,170 @@
+"""Python binding of the sm_100a Gated DeltaNet-2 library (``libgdn2.so``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/gdn2.h``.  torch supplies device
+memory and the stream; there is no CPU path and no fallback.  If the
+library has not been built this module raises on first use.
+
+    chunk_fwd(q, k, v, log_alpha, b, w, S0=None) -> (o, S_T)
+    decode_step(q, k, v, log_alpha, b, w, S)     -> o      (S updated in place)
+
+Token tensors are [B, T, H, d] (decode: [B, H, d]) in bfloat16 or float32,
+contiguous, on one CUDA device; states are float32 [B, H, d_k, d_v].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn2.so")
+
+IO_F32 = 0
+IO_BF16 = 1
+STATUS_NAMES = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
+                3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT"}
+EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_decode_step",
+            "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_status_string",
+            "gdn2_version")
+
+_lib = None
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        super().__init__(f"{what}: {STATUS_NAMES.get(self.status, self.status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Open libgdn2.so and declare the C signatures (raises if missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m gated_delta_rule_92_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        chunk_args = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        for name in ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core"):
+            getattr(L, name).argtypes = chunk_args
+            getattr(L, name).restype = I
+        L.gdn2_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P]
+        L.gdn2_decode_step.restype = I
+        L.gdn2_device_status.argtypes = [P]
+        L.gdn2_device_status.restype = I
+        L.gdn2_selftest_wait_timeout.argtypes = [I, P]
+        L.gdn2_selftest_wait_timeout.restype = I
+        L.gdn2_status_string.argtypes = [I]
+        L.gdn2_status_string.restype = ctypes.c_char_p
+        L.gdn2_version.argtypes = []
+        L.gdn2_version.restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().gdn2_status_string(int(code)).decode()
+
+
+def _io(dtype) -> int:
+    if dtype == torch.bfloat16:
+        return IO_BF16
+    if dtype == torch.float32:
+        return IO_F32
+    raise TypeError(f"unsupported I/O dtype {dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_tokens(ts, dtype, device):
+    for t in ts:
+        if not t.is_cuda or t.device != device:
+            raise ValueError("all tensors must be on the same CUDA device")
+        if t.dtype != dtype:
+            raise TypeError("token tensors must share one dtype")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _check_state(S, shape, device):
+    if S is None:
+        return
+    if S.dtype != torch.float32 or tuple(S.shape) != tuple(shape) or not S.is_contiguous() \
+            or S.device != device:
+        raise ValueError(f"state must be contiguous float32 {tuple(shape)} on {device}")
+
+
+def _chunk(fn_name, q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check_tokens((q, k, v, log_alpha, b, w), q.dtype, dev)
+    for t in (k, log_alpha, b):
+        if tuple(t.shape) != (B, T, H, dk):
+            raise ValueError("q, k, log_alpha, b must be [B, T, H, d_k]")
+    if tuple(w.shape) != (B, T, H, dv):
+        raise ValueError("v, w must be [B, T, H, d_v]")
+    _check_state(S0, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check_tokens((o,), q.dtype, dev)
+    _check_state(S_T, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        st = getattr(lib(), fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                     _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk),
+                                     _io(q.dtype), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, fn_name)
+    return o, S_T
+
+
+def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int = 64,
+              stream=None, want_state: bool = True):
+    """Chunk-parallel forward; returns (o [B,T,H,d_v], S_T [B,H,d_k,d_v] or None)."""
+    return _chunk("gdn2_chunk_fwd", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state)
+
+
+def chunk_fwd_cuda_core(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int = 64,
+                        stream=None, want_state: bool = True):
+    """The same forward on the CUDA-core (fp32 FFMA) chunk kernel."""
+    return _chunk("gdn2_chunk_fwd_cuda_core", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream,
+                  want_state)
+
+
+def decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
+    """One token per sequence: S [B,H,d_k,d_v] fp32 is updated in place; returns o [B,H,d_v]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check_tokens((q, k, v, log_alpha, b, w), q.dtype, dev)
+    _check_state(S, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                    _ptr(S), _ptr(o), B, H, dk, dv, _io(q.dtype), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_decode_step")
+    return o
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and read/clear the device status word."""
+    return int(lib().gdn2_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
+    return int(lib().gdn2_selftest_wait_timeout(int(limit_us), _stream(stream)))

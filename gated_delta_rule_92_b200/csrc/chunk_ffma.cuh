@@ -1,0 +1,188 @@
+// chunk_ffma.cuh -- chunk-parallel GDN-2 forward on CUDA cores (fp32 products).
+//
+// The recurrence (burn-gdn2 README, "Architecture") regrouped over chunks of
+// C = 64 tokens ("Chunk WY (train)" mode of the README).  For one chunk with
+// chunk-start state S (d_k x d_v), per key channel c and local row r:
+//     g_r   = sum_{s<=r} log_alpha_s           gamma_r = exp(g_r)
+//     Q~_r  = q_r . gamma_r     K~_i = k_i / gamma_i     E_r = b_r . k_r . gamma_r
+//     A_ri  = E_r . K~_i  (i < r)      P_ri = Q~_r . K~_i  (i <= r)
+//     T     = (I + A)^{-1}             (unit lower triangular)
+//     U     = T (W.V) - T (E S)        (the corrected writes u_r)
+//     O     = Q~ S + P U
+//     S'    = diag(gamma_C) (S + K~^T U)
+// which unrolls u_r = w_r.v_r - (diag(alpha_r) S_{r-1})^T (b_r.k_r) over the
+// chunk: (I + A) U = W.V - E S.  Every product here is an fp32 FMA, so this
+// kernel meets fp32-I/O tolerances; it also cross-checks the tensor-core
+// kernel, which evaluates the same products on tcgen05 in a different order.
+//
+// One block of 256 threads per (b, h, 64-column slice of d_v); everything
+// for one chunk lives in shared memory (about 215 KB at d_k = 128).
+#pragma once
+#include "decode.cuh"
+#include "gdn2_device.cuh"
+
+namespace gdn2 {
+
+template <int DK>
+struct FfmaCfg {
+    static constexpr int C = 64;
+    static constexpr int NV = 64;
+    static constexpr int LK = DK + 1;   // padded row stride for [64][DK] tiles
+    static constexpr int LC = C + 1;    // padded row stride for [.][64] tiles
+    // float offsets
+    static constexpr int O_Q = 0;
+    static constexpr int O_K = O_Q + C * LK;
+    static constexpr int O_E = O_K + C * LK;
+    static constexpr int O_G = O_E + C * LK;            // log-decay, then A and P
+    static constexpr int G_SIZE = (C * LK > 2 * C * LC) ? C * LK : 2 * C * LC;
+    static constexpr int O_T = O_G + G_SIZE;
+    static constexpr int O_WV = O_T + C * LC;           // W.V, then E S
+    static constexpr int O_U = O_WV + C * LC;           // T (W.V), then U
+    static constexpr int O_S = O_U + C * LC;            // state slice [DK][NV]
+    static constexpr int O_GC = O_S + DK * LC;
+    static constexpr int FLOATS = O_GC + DK;
+    static constexpr size_t BYTES = sizeof(float) * FLOATS;
+};
+
+template <typename IO, int DK>
+__global__ void __launch_bounds__(256, 1)
+chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
+                      const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ wg,
+                      const float *__restrict__ S0, IO *__restrict__ o, float *__restrict__ S_T,
+                      int T, int H, int d_v) {
+    using Cfg = FfmaCfg<DK>;
+    constexpr int C = Cfg::C, NV = Cfg::NV, LK = Cfg::LK, LC = Cfg::LC;
+    extern __shared__ float sm[];
+    float *sQ = sm + Cfg::O_Q, *sK = sm + Cfg::O_K, *sE = sm + Cfg::O_E, *sG = sm + Cfg::O_G;
+    float *sA = sG, *sP = sG + C * LC;
+    float *sT = sm + Cfg::O_T, *sWV = sm + Cfg::O_WV, *sU = sm + Cfg::O_U, *sS = sm + Cfg::O_S;
+    float *sGC = sm + Cfg::O_GC;
+
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * NV, h = blockIdx.y, bb = blockIdx.z;
+    const long head = (long)bb * H + h;
+    const int NC = T / C;
+
+    // initial state slice
+    for (int idx = tid; idx < DK * NV; idx += 256) {
+        const int c = idx / NV, j = idx % NV;
+        sS[c * LC + j] = S0 ? S0[(head * DK + c) * d_v + j0 + j] : 0.f;
+    }
+
+    for (int n = 0; n < NC; ++n) {
+        const long tok0 = (long)bb * T + (long)n * C;   // token row of local r = 0
+        __syncthreads();
+        // ---- load the chunk (fp32 in shared memory)
+        for (int idx = tid; idx < C * DK; idx += 256) {
+            const int r = idx / DK, c = idx % DK;
+            const long g = ((tok0 + r) * H + h) * DK + c;
+            sQ[r * LK + c] = ld_io(q + g);
+            sK[r * LK + c] = ld_io(k + g);
+            sE[r * LK + c] = ld_io(bg + g);
+            sG[r * LK + c] = ld_io(la + g);
+        }
+        for (int idx = tid; idx < C * NV; idx += 256) {
+            const int r = idx / NV, j = idx % NV;
+            const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
+            sWV[r * LC + j] = ld_io(wg + g) * ld_io(v + g);
+        }
+        __syncthreads();
+        // ---- cumulative log-decay per key channel and the scaled operands
+        if (tid < DK) {
+            const int c = tid;
+            float g = 0.f;
+            for (int r = 0; r < C; ++r) {
+                g += sG[r * LK + c];
+                const float gam = expf(g), inv = expf(-g);
+                const float kv = sK[r * LK + c];
+                sQ[r * LK + c] *= gam;
+                sE[r * LK + c] = sE[r * LK + c] * kv * gam;
+                sK[r * LK + c] = kv * inv;
+            }
+            sGC[c] = expf(g);
+        }
+        __syncthreads();
+        // ---- A (strictly lower) and P (lower, inclusive); overwrite the log-decay
+        for (int idx = tid; idx < C * C; idx += 256) {
+            const int r = idx / C, i = idx % C;
+            float a = 0.f, p = 0.f;
+            if (i <= r) {
+                for (int c = 0; c < DK; ++c) {
+                    const float kt = sK[i * LK + c];
+                    a = fmaf(sE[r * LK + c], kt, a);
+                    p = fmaf(sQ[r * LK + c], kt, p);
+                }
+            }
+            sA[r * LC + i] = (i < r) ? a : 0.f;
+            sP[r * LC + i] = p;
+        }
+        __syncthreads();
+        // ---- T = (I + A)^{-1}, one column per thread by forward substitution
+        if (tid < C) {
+            const int j = tid;
+            for (int r = 0; r < C; ++r) {
+                float x = (r == j) ? 1.f : 0.f;
+                for (int i = j; i < r; ++i) x = fmaf(-sA[r * LC + i], sT[i * LC + j], x);
+                sT[r * LC + j] = (r < j) ? 0.f : x;
+            }
+        }
+        __syncthreads();
+        // ---- T (W.V) -> sU ;  E S -> sWV (W.V is dead afterwards)
+        float acc[C * NV / 256];
+        for (int m = 0; m < C * NV / 256; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            float x = 0.f;
+            for (int i = 0; i <= r; ++i) x = fmaf(sT[r * LC + i], sWV[i * LC + j], x);
+            acc[m] = x;
+        }
+        __syncthreads();
+        for (int m = 0; m < C * NV / 256; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            sU[r * LC + j] = acc[m];
+            float x = 0.f;
+            for (int c = 0; c < DK; ++c) x = fmaf(sE[r * LK + c], sS[c * LC + j], x);
+            sWV[r * LC + j] = x;
+        }
+        __syncthreads();
+        // ---- U = T (W.V) - T (E S)
+        for (int m = 0; m < C * NV / 256; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            float x = sU[r * LC + j];
+            for (int i = 0; i <= r; ++i) x = fmaf(-sT[r * LC + i], sWV[i * LC + j], x);
+            acc[m] = x;
+        }
+        __syncthreads();
+        for (int m = 0; m < C * NV / 256; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            sU[r * LC + j] = acc[m];
+        }
+        __syncthreads();
+        // ---- O = Q~ S + P U
+        for (int m = 0; m < C * NV / 256; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            float x = 0.f;
+            for (int c = 0; c < DK; ++c) x = fmaf(sQ[r * LK + c], sS[c * LC + j], x);
+            for (int i = 0; i <= r; ++i) x = fmaf(sP[r * LC + i], sU[i * LC + j], x);
+            const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
+            if constexpr (sizeof(IO) == 4) o[g] = x;
+            else o[g] = __float2bfloat16_rn(x);
+        }
+        __syncthreads();
+        // ---- S <- diag(gamma_C) (S + K~^T U)
+        for (int idx = tid; idx < DK * NV; idx += 256) {
+            const int c = idx / NV, j = idx % NV;
+            float x = sS[c * LC + j];
+            for (int i = 0; i < C; ++i) x = fmaf(sK[i * LK + c], sU[i * LC + j], x);
+            sS[c * LC + j] = sGC[c] * x;
+        }
+    }
+    __syncthreads();
+    if (S_T) {
+        for (int idx = tid; idx < DK * NV; idx += 256) {
+            const int c = idx / NV, j = idx % NV;
+            S_T[(head * DK + c) * d_v + j0 + j] = sS[c * LC + j];
+        }
+    }
+}
+
+}  // namespace gdn2

@@ -1,0 +1,248 @@
+// gdn2_lib.cu -- the C ABI declared in include/gdn2.h.
+//
+// One translation unit: it includes every kernel header, validates
+// arguments on the host, encodes the TMA tensor maps and launches on the
+// caller's stream.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <climits>
+#include <mutex>
+
+#include "../../include/gdn2.h"
+#include "chunk_ffma.cuh"
+#include "chunk_tc.cuh"
+#include "decode.cuh"
+#include "gdn2_device.cuh"
+
+namespace gdn2 {
+
+// Default bound on any single device-side wait (2 s): far above any wait a
+// correct launch performs, short enough that a stuck kernel returns.
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        // Nothing arrives on this barrier, so phase 0 never completes.
+        if (!mbar_wait(&bar, 0u, limit_ns)) record_timeout();
+    }
+}
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn2_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Token tensor [B, T, H, d] bf16 viewed as 3-D (d, H, B*T); box = 64 columns
+// x 1 head x 64 tokens, 128-byte swizzle.
+bool make_token_map(CUtensorMap *m, const void *base, long BT, int H, int d) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)BT};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2u, (cuuint64_t)H * (cuuint64_t)d * 2u};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DK, int NV>
+gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void *la, const void *b, const void *w,
+                        const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st) {
+    using Cfg = TcCfg<DK, NV>;
+    CUtensorMap tq, tk, tla, tb, tv, tw;
+    const long BT = (long)B * T;
+    if (!make_token_map(&tq, q, BT, H, DK) || !make_token_map(&tk, k, BT, H, DK) ||
+        !make_token_map(&tla, la, BT, H, DK) || !make_token_map(&tb, b, BT, H, DK) ||
+        !make_token_map(&tv, v, BT, H, d_v) || !make_token_map(&tw, w, BT, H, d_v))
+        return GDN2_ERR_CUDA;
+    auto kern = chunk_fwd_tc_kernel<DK, NV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    dim3 grid(d_v / NV, H, B);
+    kern<<<grid, 128, Cfg::SMEM_ALLOC, st>>>(tq, tk, tla, tb, tv, tw, S0, static_cast<__nv_bfloat16 *>(o), S_T, T,
+                                             H, d_v, kWaitNs);
+    return from_cuda(cudaGetLastError());
+}
+
+template <typename IO, int DK>
+gdn2_status_t launch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
+                          const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_v,
+                          cudaStream_t st) {
+    using Cfg = FfmaCfg<DK>;
+    auto kern = chunk_fwd_ffma_kernel<IO, DK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    dim3 grid(d_v / Cfg::NV, H, B);
+    kern<<<grid, 256, Cfg::BYTES, st>>>(static_cast<const IO *>(q), static_cast<const IO *>(k),
+                                        static_cast<const IO *>(v), static_cast<const IO *>(la),
+                                        static_cast<const IO *>(b), static_cast<const IO *>(w), S0,
+                                        static_cast<IO *>(o), S_T, T, H, d_v);
+    return from_cuda(cudaGetLastError());
+}
+
+template <typename IO, int DK, int NVD>
+gdn2_status_t launch_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
+                            const void *w, float *S, void *o, int B, int H, int d_v, cudaStream_t st) {
+    dim3 grid((unsigned)((long)B * H), d_v / NVD);
+    decode_step_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
+        static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
+        static_cast<const IO *>(la), static_cast<const IO *>(b), static_cast<const IO *>(w), S,
+        static_cast<IO *>(o), d_v);
+    return from_cuda(cudaGetLastError());
+}
+
+// Shared validation of the chunk entry points.
+gdn2_status_t check_chunk(const void *q, const void *k, const void *v, const void *la, const void *b,
+                          const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
+                          int d_v, int chunk, gdn2_io_t io) {
+    // With T = 0 the token tensors are empty and may be null.
+    if (T > 0 && (!q || !k || !v || !la || !b || !w || !o)) return GDN2_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || T < 0 || d_k <= 0 || d_v <= 0 || chunk <= 0) return GDN2_ERR_INVALID_ARG;
+    if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    const void *ptrs[9] = {q, k, v, la, b, w, S0, o, S_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN2_ERR_MISALIGNED;
+    if (chunk != 64) return GDN2_ERR_UNSUPPORTED;
+    if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
+    if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
+    if (T % chunk != 0) return GDN2_ERR_UNSUPPORTED;
+    if ((long)B * T > INT_MAX || B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;
+    return GDN2_OK;
+}
+
+// T = 0: no tokens; the final state is the initial state.
+gdn2_status_t empty_sequence(const float *S0, float *S_T, int B, int H, int d_k, int d_v, cudaStream_t st) {
+    if (!S_T) return GDN2_OK;
+    const size_t bytes = sizeof(float) * (size_t)B * H * d_k * d_v;
+    if (!S0) return from_cuda(cudaMemsetAsync(S_T, 0, bytes, st));
+    if (S0 == S_T) return GDN2_OK;
+    return from_cuda(cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st));
+}
+
+gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
+                            const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
+                            int d_v, gdn2_io_t io, cudaStream_t st) {
+    if (io == GDN2_IO_F32) {
+        if (d_k == 64) return launch_ffma<float, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
+        return launch_ffma<float, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
+    }
+    if (d_k == 64) return launch_ffma<__nv_bfloat16, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
+    return launch_ffma<__nv_bfloat16, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
+}
+
+}  // namespace
+}  // namespace gdn2
+
+using namespace gdn2;
+
+extern "C" gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
+                                        const void *b, const void *w, const float *S0, void *o, float *S_T, int B,
+                                        int T, int H, int d_k, int d_v, int chunk, gdn2_io_t io, void *stream) {
+    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, io);
+    if (s != GDN2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
+    if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st);
+    const bool wide = (d_v % 128 == 0);
+    if (d_k == 64)
+        return wide ? launch_tc<64, 128>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st)
+                    : launch_tc<64, 64>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st);
+    return wide ? launch_tc<128, 128>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st)
+                : launch_tc<128, 64>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st);
+}
+
+extern "C" gdn2_status_t gdn2_chunk_fwd_cuda_core(const void *q, const void *k, const void *v,
+                                                  const void *log_alpha, const void *b, const void *w,
+                                                  const float *S0, void *o, float *S_T, int B, int T, int H,
+                                                  int d_k, int d_v, int chunk, gdn2_io_t io, void *stream) {
+    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, io);
+    if (s != GDN2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
+    return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st);
+}
+
+extern "C" gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
+                                          const void *b, const void *w, float *S, void *o, int B, int H, int d_k,
+                                          int d_v, gdn2_io_t io, void *stream) {
+    if (!q || !k || !v || !log_alpha || !b || !w || !S || !o) return GDN2_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || d_k <= 0 || d_v <= 0) return GDN2_ERR_INVALID_ARG;
+    if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    const void *ptrs[8] = {q, k, v, log_alpha, b, w, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDN2_ERR_MISALIGNED;
+    if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
+    if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
+    if ((long)B * H > INT_MAX) return GDN2_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool wide = (d_v % 128 == 0);
+#define GDN2_DECODE(IO, DK)                                                                            \
+    return wide ? launch_decode<IO, DK, 128>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st)             \
+                : launch_decode<IO, DK, 64>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st)
+    if (io == GDN2_IO_F32) {
+        if (d_k == 64) GDN2_DECODE(float, 64);
+        GDN2_DECODE(float, 128);
+    }
+    if (d_k == 64) GDN2_DECODE(__nv_bfloat16, 64);
+    GDN2_DECODE(__nv_bfloat16, 128);
+#undef GDN2_DECODE
+}
+
+extern "C" gdn2_status_t gdn2_device_status(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GDN2_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return GDN2_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return GDN2_ERR_CUDA;
+        return static_cast<gdn2_status_t>(v);
+    }
+    return GDN2_OK;
+}
+
+extern "C" gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream) {
+    if (limit_us < 1 || limit_us > 1000000) return GDN2_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    selftest_wait_kernel<<<1, 32, 0, st>>>(1000ull * (unsigned long long)limit_us);
+    if (cudaGetLastError() != cudaSuccess) return GDN2_ERR_CUDA;
+    return gdn2_device_status(stream);
+}
+
+extern "C" const char *gdn2_status_string(int status) {
+    switch (status) {
+        case GDN2_OK: return "GDN2_OK";
+        case GDN2_ERR_INVALID_ARG: return "GDN2_ERR_INVALID_ARG";
+        case GDN2_ERR_UNSUPPORTED: return "GDN2_ERR_UNSUPPORTED";
+        case GDN2_ERR_MISALIGNED: return "GDN2_ERR_MISALIGNED";
+        case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA";
+        case GDN2_ERR_DEVICE_TIMEOUT: return "GDN2_ERR_DEVICE_TIMEOUT";
+        default: return "GDN2_ERR_UNKNOWN";
+    }
+}
+
+extern "C" int gdn2_version(void) { return 100; }

@@ -1,0 +1,156 @@
+/*
+ * gdn2.h -- C ABI of the B200 (sm_100a) Gated DeltaNet-2 token mixer.
+ *
+ * The operation (burn-gdn2 README, docs.rs burn-gdn2 0.1.9, section
+ * "Architecture"): for every batch row b and head h, a matrix state
+ * S in R^{d_k x d_v} evolves token by token as
+ *
+ *     S_t = (I - k_t (b_t . k_t)^T) diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T
+ *     o_t = S_t^T q_t
+ *
+ * alpha_t = exp(log_alpha_t) is a per-key-channel decay (KDA-style, as the
+ * asapai.co.kr Gated DeltaNet-2 article describes), b_t the per-key-channel
+ * erase gate and w_t the per-value-channel write gate (README, text under
+ * the equation).  o_t reads the state after the update.  No scaling is
+ * applied to q; callers pass q and k already L2-normalised (the README's
+ * layer diagram applies an L2-norm before the mixer).
+ *
+ * Two entry points follow the README's two forward modes ("Chunk WY (train)"
+ * and "Fused Recurrent (infer)"):
+ *   gdn2_chunk_fwd   -- a whole sequence, chunk-parallel (chunked WY form);
+ *   gdn2_decode_step -- one token per sequence against a caller-held state.
+ *
+ * Common conventions
+ * ------------------
+ * Pointers are DEVICE pointers (cudaMalloc'd or torch CUDA tensors) on the
+ * current device, unless a function says otherwise.  All tensors are dense,
+ * contiguous, row-major:
+ *     q, k, log_alpha, b : [B, T, H, d_k]
+ *     v, w, o            : [B, T, H, d_v]
+ *     S0, S_T, S         : [B, H, d_k, d_v]   always float32
+ * Token tensors (q, k, v, log_alpha, b, w, o) share one I/O dtype `io`:
+ * GDN2_IO_F32 (float32) or GDN2_IO_BF16 (bfloat16).  log_alpha holds natural
+ * logarithms.  Every pointer must be 16-byte aligned.
+ *
+ * The caller owns every buffer; the library allocates no device memory.
+ * Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = the
+ * legacy default stream) and the call returns without synchronising.
+ *
+ * Errors are returned as gdn2_status_t; nothing aborts, throws or traps.
+ * Argument errors are detected on the host before any launch.  Device-side
+ * waits inside the kernels are bounded: a wait that runs out records
+ * GDN2_ERR_DEVICE_TIMEOUT in a per-device status word, the kernel releases
+ * its tensor memory and returns; gdn2_device_status() reads and clears it.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN2_IO_F32 = 0,
+    GDN2_IO_BF16 = 1
+} gdn2_io_t;
+
+typedef enum {
+    GDN2_OK = 0,
+    GDN2_ERR_INVALID_ARG = 1,     /* null pointer, negative size, bad enum   */
+    GDN2_ERR_UNSUPPORTED = 2,     /* valid but outside the built shapes      */
+    GDN2_ERR_MISALIGNED = 3,      /* a pointer is not 16-byte aligned        */
+    GDN2_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed       */
+    GDN2_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait ran out      */
+} gdn2_status_t;
+
+/*
+ * gdn2_chunk_fwd -- chunk-parallel forward over whole sequences.
+ *
+ * Computes o_t for t = 0..T-1 and the final state S_T of every (b, h) from
+ * the initial state S0 (README "Architecture" equation; "Chunk WY (train)"
+ * mode).  The result equals the token-by-token recurrence up to rounding:
+ * the chunk form is an exact regrouping, not an approximation.
+ *
+ *   q, k, log_alpha, b : in,  [B, T, H, d_k], dtype io
+ *   v, w               : in,  [B, T, H, d_v], dtype io
+ *   S0                 : in,  [B, H, d_k, d_v] float32, or NULL for zeros
+ *   o                  : out, [B, T, H, d_v], dtype io
+ *   S_T                : out, [B, H, d_k, d_v] float32, or NULL (not written).
+ *                        May alias S0 (each block reads its slice of S0
+ *                        before it writes that slice of S_T).
+ *   chunk              : chunk length; must be 64 (the README default).
+ *
+ * Built shapes: d_k in {64, 128}; d_v a multiple of 64 with d_v <= 512;
+ * T a multiple of `chunk` (T = 0 is allowed: o is empty, token pointers may
+ * be NULL, and S_T = S0).
+ * Other shapes return GDN2_ERR_UNSUPPORTED.
+ *
+ * Precision: bf16 I/O runs the tensor-core kernel (bf16 operands, fp32
+ * accumulation, fp32 state carried between chunks); fp32 I/O runs the
+ * CUDA-core kernel with fp32 products throughout.  o is rounded to the I/O
+ * dtype (round to nearest even); S_T is fp32.
+ */
+gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v,
+                             const void *log_alpha, const void *b, const void *w,
+                             const float *S0, void *o, float *S_T,
+                             int B, int T, int H, int d_k, int d_v, int chunk,
+                             gdn2_io_t io, void *stream);
+
+/*
+ * gdn2_chunk_fwd_cuda_core -- the same operation and arguments as
+ * gdn2_chunk_fwd, always on the CUDA-core (FFMA, fp32 products) chunk
+ * kernel, for either I/O dtype.  It is the fp32-I/O path of gdn2_chunk_fwd
+ * and serves as an independent second GPU implementation of the chunk form.
+ */
+gdn2_status_t gdn2_chunk_fwd_cuda_core(const void *q, const void *k, const void *v,
+                                       const void *log_alpha, const void *b, const void *w,
+                                       const float *S0, void *o, float *S_T,
+                                       int B, int T, int H, int d_k, int d_v, int chunk,
+                                       gdn2_io_t io, void *stream);
+
+/*
+ * gdn2_decode_step -- one recurrent step for B independent sequences
+ * (README "Fused Recurrent (infer)" mode; the README's inference example
+ * carries the state between calls in a caller-held variable).
+ *
+ *   q, k, log_alpha, b : in,  [B, H, d_k], dtype io   (T = 1)
+ *   v, w               : in,  [B, H, d_v], dtype io
+ *   S                  : in/out, [B, H, d_k, d_v] float32, updated in place
+ *                        from S_{t-1} to S_t
+ *   o                  : out, [B, H, d_v], dtype io, o_t = S_t^T q_t
+ *
+ * Built shapes: d_k in {64, 128}; d_v a multiple of 64 with d_v <= 512.
+ * The step reads and writes S exactly once.
+ */
+gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v,
+                               const void *log_alpha, const void *b, const void *w,
+                               float *S, void *o, int B, int H, int d_k, int d_v,
+                               gdn2_io_t io, void *stream);
+
+/*
+ * gdn2_device_status -- synchronise `stream`, then read and clear the
+ * current device's status word.  Returns GDN2_OK, GDN2_ERR_DEVICE_TIMEOUT if
+ * a kernel gave up on a bounded wait since the last call, or GDN2_ERR_CUDA.
+ */
+gdn2_status_t gdn2_device_status(void *stream);
+
+/*
+ * gdn2_selftest_wait_timeout -- exercise the bounded-wait path without any
+ * fault: launches one block that waits on a shared-memory barrier which
+ * nothing ever completes, with a limit of `limit_us` microseconds (1..10^6).
+ * The kernel records GDN2_ERR_DEVICE_TIMEOUT and returns; the call then
+ * returns gdn2_device_status(stream), i.e. GDN2_ERR_DEVICE_TIMEOUT when the
+ * mechanism works.
+ */
+gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *gdn2_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int gdn2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN2_H */

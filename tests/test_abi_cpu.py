@@ -1,0 +1,91 @@
+"""CPU-side checks of the C ABI: the library builds, loads and exports every
+symbol include/gdn2.h declares; status strings; host-side argument checks
+that return before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_92_b200 as g
+from gated_delta_rule_92_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return g.lib()
+
+
+def declared_functions():
+    with open(os.path.join(ROOT, "include", "gdn2.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn2_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert names == sorted(g.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {g.LIB_PATH}").read()
+    exported = set(re.findall(r" T (gdn2_[a-z0-9_]+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings(L):
+    for code, name in g.STATUS_NAMES.items():
+        assert g.status_string(code) == name
+    assert g.status_string(99) == "GDN2_ERR_UNKNOWN"
+    assert L.gdn2_version() >= 100
+
+
+def _chunk_call(L, ptr=16, B=1, T=64, H=1, dk=64, dv=64, chunk=64, io=1, o=16, s0=None, st=None):
+    P = ctypes.c_void_p
+    p = P(ptr) if ptr is not None else None
+    return L.gdn2_chunk_fwd(p, p, p, p, p, p, P(s0) if s0 else None, P(o) if o else None,
+                            P(st) if st else None, B, T, H, dk, dv, chunk, io, None)
+
+
+def test_chunk_argument_validation_on_host(L):
+    # these return before touching the device
+    assert _chunk_call(L, ptr=None) == 1                 # null input
+    assert _chunk_call(L, ptr=None, T=0, o=None) == 0    # empty sequence, no state: no-op
+    assert _chunk_call(L, B=0) == 1
+    assert _chunk_call(L, T=-1) == 1
+    assert _chunk_call(L, io=7) == 1
+    assert _chunk_call(L, ptr=24) == 3                   # misaligned
+    assert _chunk_call(L, o=40) == 3
+    assert _chunk_call(L, chunk=32) == 2                 # only chunk 64 is built
+    assert _chunk_call(L, dk=96) == 2
+    assert _chunk_call(L, dv=96) == 2
+    assert _chunk_call(L, dv=1024) == 2
+    assert _chunk_call(L, T=100) == 2                    # T % chunk
+    assert _chunk_call(L, B=70000) == 2
+
+
+def test_decode_argument_validation_on_host(L):
+    P = ctypes.c_void_p
+    p = P(16)
+    assert L.gdn2_decode_step(p, p, p, p, p, p, None, p, 1, 1, 64, 64, 1, None) == 1
+    assert L.gdn2_decode_step(p, p, p, p, p, p, p, p, 0, 1, 64, 64, 1, None) == 1
+    assert L.gdn2_decode_step(p, p, p, p, p, p, P(8), p, 1, 1, 64, 64, 1, None) == 3
+    assert L.gdn2_decode_step(p, p, p, p, p, p, p, p, 1, 1, 32, 64, 1, None) == 2
+    assert L.gdn2_decode_step(p, p, p, p, p, p, p, p, 1, 1, 64, 80, 1, None) == 2
+    assert L.gdn2_selftest_wait_timeout(0, None) == 1
+
+
+def test_product_path_does_not_touch_oracle():
+    """The binding and the CUDA sources never reference the oracle."""
+    pkg = os.path.join(ROOT, "gated_delta_rule_92_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    assert "oracle" not in f.read().lower(), fn
