@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 Gated DeltaNet-2 mixer (chunk forward + decode).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one chunk-forward call over the headline workload
+(B8 T4096 H16 d_k=d_v=128, chunk 64, bf16 I/O, fp32 state: the burn-gdn2
+default configuration of 16 heads x head_dim 128, hidden 2048), inputs
+resident in HBM (948 MB, larger than the 126 MB L2, so no flush is needed).
+`value` is tokens/s over all ranks (a token = one (b, t) position through all
+16 heads), timed on the device with CUDA events, max over ranks.  The same
+JSON line carries:
+  e2e          the same metric through the public API with pinned host
+               buffers: H2D inputs + call + D2H of o and S_T every step;
+  roofline     the chunk kernel's algorithmic HBM bytes / launch time vs the
+               measured copy bandwidth;
+  decode       tokens/s of the decode workload (256 sequences x 16 heads x
+               d128, 1024 consecutive steps) with its own HBM roofline;
+  expanded_v   the d_v=256, b in (0,2) chunk workload;
+  cpu_baseline the fp64 oracle on the host cores over a bounded sample.
+With torchrun (N > 1) every rank runs its own batch (weak scaling, no
+collective on the data path); only the barrier and the max-over-ranks time
+reduction use NCCL.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+HEADLINE = "chunk_bf16_h2048"
+METRIC = "GDN-2 chunk-fwd tokens/s and decode tokens/s at 1 B200; % of roofline"
+
+
+# ------------------------------------------------------------ accounting
+def chunk_bytes(wl, with_s0: bool, with_st: bool = True) -> int:
+    """Algorithmic HBM bytes of one chunk-forward launch: every input read
+    once, o written once, the fp32 state read (S0) / written (S_T) once."""
+    io = 4 if wl.io == "f32" else 2
+    tok = wl.B * wl.T * wl.H * (4 * wl.d_k + 3 * wl.d_v) * io
+    st = wl.B * wl.H * wl.d_k * wl.d_v * 4
+    return tok + st * (int(with_s0) + int(with_st))
+
+
+def chunk_flops(wl) -> float:
+    """Useful FLOPs of the chunk form per launch (triangles counted half):
+    per token-head C(3 d_k + 2 d_v) + C^2/3 + 6 d_k d_v."""
+    C = wl.chunk
+    per = C * (3 * wl.d_k + 2 * wl.d_v) + C * C / 3 + 6 * wl.d_k * wl.d_v
+    return per * wl.B * wl.T * wl.H
+
+
+def decode_bytes(wl) -> int:
+    io = 4 if wl.io == "f32" else 2
+    return wl.B * wl.H * ((4 * wl.d_k + 3 * wl.d_v) * io + 2 * wl.d_k * wl.d_v * 4)
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------- clocks
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read only)."""
+
+    def __init__(self, period_s: float = 0.005):
+        self.period = period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            props = torch.cuda.get_device_properties(torch.cuda.current_device())
+            try:
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _reasons(self):
+        nv = self._nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return int(getattr(nv, fn)(self._h))
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                self.reasons |= self._reasons()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self) -> dict:
+        names = sorted(n for bit, n in REASONS.items() if self.reasons & bit and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- timing
+def device_time_ms(fn, steps: int, stream) -> float:
+    """Time `steps` calls of fn on `stream` with CUDA events (ms total)."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------- our measurements
+def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None):
+    d = W.make_chunk_inputs(wl, seed=wl.seed + 100 * rank, device="cuda")
+    o = torch.empty_like(d["v"])
+    S_T = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
+
+    def step():
+        g.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], o=o, S_T=S_T,
+                    stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        with sampler:
+            ms = device_time_ms(step, steps, stream)
+    else:
+        ms = device_time_ms(step, steps, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    if g.device_status() != 0:
+        raise RuntimeError("chunk kernel reported a device timeout")
+    return ms, d, o, S_T
+
+
+def bench_chunk_e2e(g, wl, d, steps, stream):
+    """Same call through the public API, with pinned host inputs copied in
+    and o, S_T copied out inside the timed region, every step."""
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    host = {n: d[n].cpu().pin_memory() for n in names}
+    s0_host = d["S0"].cpu().pin_memory() if d["S0"] is not None else None
+    dev = {n: torch.empty_like(d[n]) for n in names}
+    s0_dev = torch.empty_like(d["S0"]) if d["S0"] is not None else None
+    o_dev = torch.empty_like(d["v"])
+    st_dev = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
+    o_host = torch.empty(o_dev.shape, dtype=o_dev.dtype).pin_memory()
+    st_host = torch.empty(st_dev.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + \
+        (s0_host.numel() * 4 if s0_host is not None else 0)
+    d2h = o_host.numel() * o_host.element_size() + st_host.numel() * 4
+
+    def step():
+        with torch.cuda.stream(stream):
+            for n in names:
+                dev[n].copy_(host[n], non_blocking=True)
+            if s0_dev is not None:
+                s0_dev.copy_(s0_host, non_blocking=True)
+            g.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["b"], dev["w"], s0_dev,
+                        o=o_dev, S_T=st_dev, stream=stream)
+            o_host.copy_(o_dev, non_blocking=True)
+            st_host.copy_(st_dev, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    ms = device_time_ms(step, steps, stream)
+    return ms, h2d, d2h
+
+
+def bench_decode(g, wl, steps, rank, stream):
+    d = W.make_decode_inputs(wl, steps, seed=wl.seed + 100 * rank, device="cuda")
+    S = d["S0"].clone()
+    o = torch.empty(wl.B, wl.H, wl.d_v, dtype=wl.torch_dtype, device="cuda")
+    it = {"s": 0}
+
+    def step():
+        s = it["s"] % steps
+        it["s"] += 1
+        g.decode_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["b"][s], d["w"][s], S,
+                      o=o, stream=stream)
+
+    for _ in range(8):
+        step()
+    torch.cuda.synchronize()
+    S.copy_(d["S0"])
+    it["s"] = 0
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("decode kernel reported a device timeout")
+    return ms
+
+
+# --------------------------------------------------------- oracle (CPU)
+def oracle_sample(wl, d_cpu_fn, budget_s: float = 10.0):
+    """Time the fp64 oracle, as it stands, on whole heads of the workload
+    until about `budget_s` of wall time has passed.  Returns (tokens/s,
+    cores, description); a token is one (b, t) through all H heads."""
+    import oracle
+    cores = oracle.max_threads()
+    heads_done, t_used, rounds = 0, 0.0, 0
+    while t_used < budget_s and rounds < 64:
+        inp = d_cpu_fn(cores, rounds)
+        t0 = time.perf_counter()
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"],
+                       S0=inp["S0"], n_threads=cores, want_state=True)
+        t_used += time.perf_counter() - t0
+        heads_done += inp["q"].shape[2]
+        rounds += 1
+    tok = heads_done * wl.T / wl.H
+    return tok / t_used, cores, f"{heads_done} whole heads (T={wl.T}) of {wl.describe()}, {t_used:.1f} s"
+
+
+def head_sample_fn(wl):
+    """Sample n heads of the workload as a [1, T, n, d] CPU batch."""
+    def fn(n, r):
+        return W.draw(1, wl.T, n, wl.d_k, wl.d_v, seed=wl.seed + 7919 * (r + 1), dtype=wl.torch_dtype,
+                      alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, b_scale=wl.b_scale, s0_std=wl.s0_std)
+    return fn
+
+
+def profile_case(g, args, stream):
+    """A reduced launch of one kernel for profiler captures."""
+    import dataclasses
+    if args.profile_case == "decode":
+        wl = dataclasses.replace(W.BY_NAME["decode_bf16"], decode_steps=args.warmup + args.steps)
+        ms = bench_decode(g, wl, wl.decode_steps, 0, stream)
+        print(json.dumps({"profile_case": "decode", "workload": wl.describe(),
+                          "us_per_step": 1e3 * ms / wl.decode_steps}))
+        return
+    base = W.BY_NAME[HEADLINE if args.profile_case == "chunk" else "chunk_bf16_negeig"]
+    wl = dataclasses.replace(base, B=2 if base.d_v == 128 else 1)
+    ms, d, _, _ = bench_chunk(g, wl, args.steps, args.warmup, 0, 1, stream)
+    print(json.dumps({"profile_case": args.profile_case, "workload": wl.describe(),
+                      "ms_per_call": ms / args.steps,
+                      "bytes_per_call": chunk_bytes(wl, with_s0=d["S0"] is not None)}))
+
+
+# ------------------------------------------------------------------ main
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world
+
+
+def run_reference(args, world):
+    """The reference arm: the fp64 oracle on the host cores (no GPU)."""
+    wl = W.BY_NAME[HEADLINE]
+    fn = head_sample_fn(wl)
+    import oracle
+    cores = oracle.max_threads()
+    for r in range(args.warmup):
+        inp = fn(cores, 1000 + r)
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"],
+                       S0=inp["S0"], n_threads=cores)
+    t_total, heads = 0.0, 0
+    for r in range(args.steps):
+        inp = fn(cores, r)
+        t0 = time.perf_counter()
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"],
+                       S0=inp["S0"], n_threads=cores)
+        t_total += time.perf_counter() - t0
+        heads += inp["q"].shape[2]
+    tok_s = heads * wl.T / wl.H / t_total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.describe(), "parallelism": "host cores (OpenMP over heads)"},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {cores} whole heads (T={wl.T}) of {wl.describe()}"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-extras", action="store_true", help="skip decode/expanded-value/CPU legs")
+    ap.add_argument("--profile-case", choices=["chunk", "chunk_v256", "decode"], default=None,
+                    help="only launch one kernel on a reduced batch (inputs still larger than L2), "
+                         "for ncu captures; prints a short line")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, world)
+        return
+
+    rank, world = dist_setup()
+    import gated_delta_rule_92_b200 as g
+    g.lib()
+    peaks = load_peaks()
+    stream = torch.cuda.Stream()
+    wl = W.BY_NAME[HEADLINE]
+    if args.profile_case is not None:
+        profile_case(g, args, stream)
+        return
+
+    sampler = ClockSampler()
+    ms, d, o, S_T = bench_chunk(g, wl, args.steps, args.warmup, rank, world, stream, sampler)
+    ms_max = max_over_ranks(ms, world)
+    tokens = wl.B * wl.T * world * args.steps
+    value = tokens / (ms_max / 1e3)
+    launch_ms = ms / args.steps
+    abytes = chunk_bytes(wl, with_s0=d["S0"] is not None)
+    achieved = abytes / (launch_ms / 1e3) / 1e9
+    flops = chunk_flops(wl)
+
+    e2e_ms, h2d, d2h = bench_chunk_e2e(g, wl, d, args.e2e_steps, stream)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e_val = wl.B * wl.T * world * args.e2e_steps / (e2e_ms / 1e3)
+    del d, o, S_T
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if not args.no_extras:
+        wl3 = W.BY_NAME["chunk_bf16_negeig"]
+        ms3, d3, _, _ = bench_chunk(g, wl3, max(5, args.steps // 4), 3, rank, world, stream)
+        l3 = ms3 / max(5, args.steps // 4)
+        b3 = chunk_bytes(wl3, with_s0=True)
+        extras["expanded_v"] = {
+            "workload": wl3.describe(), "value": wl3.B * wl3.T / (l3 / 1e3), "unit": "tokens/s",
+            "ms_per_call": l3,
+            "roofline": {"bound": "hbm", "achieved": b3 / (l3 / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": b3 / (l3 / 1e3) / 1e9 / peaks["hbm_gbs"]}}
+        del d3
+        torch.cuda.empty_cache()
+        wl4 = W.BY_NAME["decode_bf16"]
+        with ClockSampler() as s4:
+            ms4 = bench_decode(g, wl4, wl4.decode_steps, rank, stream)
+        ms4 = max_over_ranks(ms4, world)
+        per = ms4 / wl4.decode_steps
+        b4 = decode_bytes(wl4)
+        extras["decode"] = {
+            "workload": wl4.describe(), "value": wl4.B * world * wl4.decode_steps / (ms4 / 1e3),
+            "unit": "tokens/s", "us_per_step": 1e3 * per, "steps": wl4.decode_steps,
+            "roofline": {"bound": "hbm", "achieved": b4 / (per / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": b4 / (per / 1e3) / 1e9 / peaks["hbm_gbs"],
+                         "bytes_per_step": b4},
+            "clocks": s4.summary()}
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        tok_s, cores, desc = oracle_sample(wl, head_sample_fn(wl))
+        cpu = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.describe(), "global_batch": wl.B * world, "seq_len": wl.T,
+                       "heads": wl.H, "d_k": wl.d_k, "d_v": wl.d_v, "chunk": wl.chunk,
+                       "state": "fp32", "parallelism": f"dp{world} (independent batches)",
+                       "l2": f"inputs larger than L2 ({abytes / 1e6:.0f} MB per step); no flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peaks["source"], "bytes_per_launch": abytes,
+                         "tensor_tflops": flops / (launch_ms / 1e3) / 1e12,
+                         "tensor_frac": flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+            "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": sampler.summary(),
+            "cpu_baseline": cpu,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

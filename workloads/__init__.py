@@ -85,23 +85,27 @@ def _l2n(x: torch.Tensor) -> torch.Tensor:
 def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
          dtype=torch.bfloat16, alpha_lo: float = 0.9, alpha_hi: float = 0.999,
          b_scale: float = 1.0, s0_std: Optional[float] = None,
-         generator: Optional[torch.Generator] = None) -> dict:
-    """Draw one batch of token inputs [B, T, H, d] (CPU tensors).
+         generator: Optional[torch.Generator] = None, device="cpu") -> dict:
+    """Draw one batch of token inputs [B, T, H, d].
 
     Returns a dict with q, k, v, log_alpha, b, w in ``dtype`` and S0 (fp32
-    [B, H, d_k, d_v] or None).
+    [B, H, d_k, d_v] or None).  With ``device="cuda"`` the draws are made by
+    a CUDA generator with the same seed and recipe (a different stream of
+    numbers than the CPU generator; used where only the distribution matters,
+    e.g. timing).
     """
-    g = generator if generator is not None else torch.Generator().manual_seed(seed)
+    g = generator if generator is not None else torch.Generator(device=device).manual_seed(seed)
     f32 = torch.float32
-    q = _l2n(torch.randn(B, T, H, d_k, generator=g, dtype=f32))
-    k = _l2n(torch.randn(B, T, H, d_k, generator=g, dtype=f32))
-    v = torch.randn(B, T, H, d_v, generator=g, dtype=f32)
-    alpha = torch.empty(B, T, H, d_k, dtype=f32).uniform_(alpha_lo, alpha_hi, generator=g)
-    b = b_scale * torch.sigmoid(torch.randn(B, T, H, d_k, generator=g, dtype=f32))
-    w = torch.sigmoid(torch.randn(B, T, H, d_v, generator=g, dtype=f32))
+    kw = dict(generator=g, dtype=f32, device=device)
+    q = _l2n(torch.randn(B, T, H, d_k, **kw))
+    k = _l2n(torch.randn(B, T, H, d_k, **kw))
+    v = torch.randn(B, T, H, d_v, **kw)
+    alpha = torch.empty(B, T, H, d_k, dtype=f32, device=device).uniform_(alpha_lo, alpha_hi, generator=g)
+    b = b_scale * torch.sigmoid(torch.randn(B, T, H, d_k, **kw))
+    w = torch.sigmoid(torch.randn(B, T, H, d_v, **kw))
     S0 = None
     if s0_std is not None:
-        S0 = s0_std * torch.randn(B, H, d_k, d_v, generator=g, dtype=f32)
+        S0 = s0_std * torch.randn(B, H, d_k, d_v, **kw)
     out = dict(q=q, k=k, v=v, log_alpha=torch.log(alpha), b=b, w=w)
     out = {n: t.to(dtype).contiguous() for n, t in out.items()}
     out["S0"] = S0
@@ -109,16 +113,16 @@ def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
 
 
 def make_chunk_inputs(wl: Workload, *, B: Optional[int] = None, T: Optional[int] = None,
-                      H: Optional[int] = None, seed: Optional[int] = None) -> dict:
+                      H: Optional[int] = None, seed: Optional[int] = None, device="cpu") -> dict:
     """Inputs of a chunk workload (optionally resized, same recipe)."""
     return draw(B or wl.B, T or wl.T, H or wl.H, wl.d_k, wl.d_v,
                 seed=wl.seed if seed is None else seed, dtype=wl.torch_dtype,
                 alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, b_scale=wl.b_scale,
-                s0_std=wl.s0_std)
+                s0_std=wl.s0_std, device=device)
 
 
 def make_decode_inputs(wl: Workload, steps: int, *, B: Optional[int] = None,
-                       seed: Optional[int] = None) -> dict:
+                       seed: Optional[int] = None, device="cpu") -> dict:
     """Decode inputs: token tensors [steps, B, H, d] and S0 [B, H, d_k, d_v].
 
     Drawn as a [B, steps, H, d] batch with the same recipe, then laid out with
@@ -127,7 +131,7 @@ def make_decode_inputs(wl: Workload, steps: int, *, B: Optional[int] = None,
     Bn = B or wl.B
     d = draw(Bn, steps, wl.H, wl.d_k, wl.d_v, seed=wl.seed if seed is None else seed,
              dtype=wl.torch_dtype, alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi,
-             b_scale=wl.b_scale, s0_std=wl.s0_std)
+             b_scale=wl.b_scale, s0_std=wl.s0_std, device=device)
     for n in ("q", "k", "v", "log_alpha", "b", "w"):
         d[n] = d[n].transpose(0, 1).contiguous()
     return d
