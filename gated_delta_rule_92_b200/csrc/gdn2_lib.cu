@@ -83,12 +83,8 @@ gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
     dim3 grid(d_v / NV, H, B);
-    using bf = __nv_bfloat16;
-    kern<<<grid, 256, Cfg::SMEM_ALLOC, st>>>(tq, tk, tla, tb, tv, tw, static_cast<const bf *>(q),
-                                             static_cast<const bf *>(k), static_cast<const bf *>(v),
-                                             static_cast<const bf *>(la), static_cast<const bf *>(b),
-                                             static_cast<const bf *>(w), S0, static_cast<bf *>(o), S_T, T, H, d_v,
-                                             kWaitNs);
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tla, tb, tv, tw, S0, static_cast<__nv_bfloat16 *>(o), S_T, T,
+                                             H, d_v, kWaitNs);
     return from_cuda(cudaGetLastError());
 }
 

@@ -47,18 +47,28 @@ def test_chunk_form_matches_recurrence(oracle_mod, C, bs):
         assert rel_err(Sm, ST[hi]) < 1e-10
 
 
-def test_blocked_unit_lower_inverse():
-    """The 16x16-blocked forward substitution of the tensor-core kernel:
-    diagonal blocks by substitution, then T_ib = -D_ib sum_k A_ib,k T_k."""
+def test_doubling_unit_lower_inverse():
+    """The in-place inverse of the tensor-core kernel, step by step:
+    16x16 diagonal blocks by right-looking substitution, then
+    T_{2p+1,2p} = -D_{2p+1} A_{2p+1,2p} D_{2p}, then T_ba = -T_b A_ba T_a."""
     rng = np.random.default_rng(3)
     A = np.tril(rng.standard_normal((64, 64)) * 0.3, -1)
-    Tb = A.copy()
+    M = A.copy()
     for blk in range(4):
         R = 16 * blk
-        D = np.linalg.inv(np.eye(16) + A[R:R + 16, R:R + 16])
-        Tb[R:R + 16, R:R + 16] = D
-    for ib in range(1, 4):
-        n = 16 * ib
-        Wm = A[n:n + 16, :n] @ Tb[:n, :n]
-        Tb[n:n + 16, :n] = -Tb[n:n + 16, n:n + 16] @ Wm
-    np.testing.assert_allclose(Tb, np.linalg.inv(np.eye(64) + A), rtol=1e-10, atol=1e-10)
+        X = np.zeros((16, 16))
+        for j in range(16):
+            s = np.eye(16)[:, j].copy()
+            x = np.zeros(16)
+            for i in range(16):
+                x[i] = s[i]
+                s[i + 1:] -= A[R + i + 1:R + 16, R + i] * x[i]
+            X[:, j] = x
+        M[R:R + 16, R:R + 16] = X
+    for p in range(2):
+        R = 32 * p
+        Y = M[R + 16:R + 32, R:R + 16] @ M[R:R + 16, R:R + 16]
+        M[R + 16:R + 32, R:R + 16] = -M[R + 16:R + 32, R + 16:R + 32] @ Y
+    Y = M[32:, :32] @ M[:32, :32]
+    M[32:, :32] = -M[32:, 32:] @ Y
+    np.testing.assert_allclose(M, np.linalg.inv(np.eye(64) + A), rtol=1e-10, atol=1e-10)
