@@ -67,6 +67,27 @@ def decode_bytes(wl) -> int:
     return wl.B * wl.H * ((4 * wl.d_k + 3 * wl.d_v) * io + 2 * wl.d_k * wl.d_v * 4)
 
 
+def measured_traffic(kernel: str, batch: int):
+    """DRAM bytes per launch from the committed ncu capture in
+    profiles/traffic.json, scaled to `batch`; None if the kernel sources have
+    changed since that capture (digest mismatch) or no capture exists."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != rec["digest"]:
+        return None
+    return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * batch / rec["case_batch"]
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -158,18 +179,31 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Max of a per-rank scalar over all ranks (NCCL on cuda, gloo on cpu)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
+def rank_seed(wl, rank: int) -> int:
+    """Each rank draws its own batch of the workload (weak scaling)."""
+    return wl.seed + 100 * rank
+
+
+def aggregate_throughput(ms_local: float, steps: int, tokens_per_rank_step: int, world: int,
+                         device: str = "cuda"):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    ms_max = max_over_ranks(ms_local, world, device)
+    return tokens_per_rank_step * world * steps / (ms_max / 1e3), ms_max
+
+
 # ------------------------------------------------------- our measurements
 def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None):
-    d = W.make_chunk_inputs(wl, seed=wl.seed + 100 * rank, device="cuda")
+    d = W.make_chunk_inputs(wl, seed=rank_seed(wl, rank), device="cuda")
     o = torch.empty_like(d["v"])
     S_T = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
 
@@ -229,7 +263,7 @@ def bench_chunk_e2e(g, wl, d, steps, stream):
 
 
 def bench_decode(g, wl, steps, rank, stream):
-    d = W.make_decode_inputs(wl, steps, seed=wl.seed + 100 * rank, device="cuda")
+    d = W.make_decode_inputs(wl, steps, seed=rank_seed(wl, rank), device="cuda")
     S = d["S0"].clone()
     o = torch.empty(wl.B, wl.H, wl.d_v, dtype=wl.torch_dtype, device="cuda")
     it = {"s": 0}
@@ -378,17 +412,14 @@ def main():
 
     sampler = ClockSampler()
     ms, d, o, S_T = bench_chunk(g, wl, args.steps, args.warmup, rank, world, stream, sampler)
-    ms_max = max_over_ranks(ms, world)
-    tokens = wl.B * wl.T * world * args.steps
-    value = tokens / (ms_max / 1e3)
+    value, ms_max = aggregate_throughput(ms, args.steps, wl.B * wl.T, world)
     launch_ms = ms / args.steps
     abytes = chunk_bytes(wl, with_s0=d["S0"] is not None)
     achieved = abytes / (launch_ms / 1e3) / 1e9
     flops = chunk_flops(wl)
 
     e2e_ms, h2d, d2h = bench_chunk_e2e(g, wl, d, args.e2e_steps, stream)
-    e2e_ms = max_over_ranks(e2e_ms, world)
-    e2e_val = wl.B * wl.T * world * args.e2e_steps / (e2e_ms / 1e3)
+    e2e_val, e2e_ms = aggregate_throughput(e2e_ms, args.e2e_steps, wl.B * wl.T, world)
     del d, o, S_T
     torch.cuda.empty_cache()
 
@@ -416,7 +447,7 @@ def main():
             "unit": "tokens/s", "us_per_step": 1e3 * per, "steps": wl4.decode_steps,
             "roofline": {"bound": "hbm", "achieved": b4 / (per / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": b4 / (per / 1e3) / 1e9 / peaks["hbm_gbs"],
-                         "bytes_per_step": b4},
+                         "bytes_per_step": b4, "traffic": measured_traffic("decode_step", wl4.B)},
             "clocks": s4.summary()}
         torch.cuda.empty_cache()
 
@@ -436,7 +467,8 @@ def main():
                        "state": "fp32", "parallelism": f"dp{world} (independent batches)",
                        "l2": f"inputs larger than L2 ({abytes / 1e6:.0f} MB per step); no flush"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": measured_traffic("chunk_fwd_tc", wl.B),
                          "peak_source": peaks["source"], "bytes_per_launch": abytes,
                          "tensor_tflops": flops / (launch_ms / 1e3) / 1e12,
                          "tensor_frac": flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
