@@ -105,9 +105,12 @@ constexpr int kTcThreads = kKeyThreads + kChainThreads + 32;   // + producer war
 //   1. each 16x16 diagonal block D_k = (I + A_kk)^{-1} by right-looking
 //      forward substitution, one column per thread (threads 0-63);
 //   2. 16 -> 32: T_{2p+1,2p} = -D_{2p+1} (A_{2p+1,2p} D_{2p}), p = 0, 1
-//      (threads 0-127, one float4 of one row each);
+//      (threads 0-63);
 //   3. 32 -> 64: T_ba = -T_b (A_ba T_a) with a = rows/cols 0-31, b = 32-63
-//      (all 256 threads, one float4 of one row each).
+//      (threads 0-127).
+// Block products keep two rows of the left factor in registers per thread
+// and stream one float4 of the right factor per step, so each 128-bit
+// shared-memory load feeds eight FMAs.
 // The intermediate products go to the upper-right 32x32 block, which T
 // leaves zero; readers of T must mask columns above the diagonal.
 // Barriers are named barrier 1 (256 threads).
@@ -135,64 +138,105 @@ __device__ __forceinline__ void unit_lower_inverse64(float *sA, int t) {
         }
         named_bar(1, kKeyThreads);
     }
-    {   // 2. 16 -> 32; products in the upper-right block (rows 16p + r, cols 32 + 4c4)
-        const int p = (t >> 6) & 1, r = (t >> 2) & 15, c4 = t & 3;
+    {   // 2. 16 -> 32 (threads 0-63: two rows x one float4 each); products in the
+        //    upper-right block, rows 16p + r, cols 32 + 4c4
+        const int p = (t >> 5) & 1, r = 2 * ((t >> 2) & 7), c4 = t & 3;
         const int R = 32 * p;   // block (2p+1, 2p) lives at rows R+16.., cols R..
-        if (t < 128) {
-            const float *arow = sA + (R + 16 + r) * LDA + R;
+        if (t < 64) {
+            float a0[16], a1[16];   // rows r, r+1 of A_{2p+1,2p}
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (R + 16 + r) * LDA + R + 4 * q);
+                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (R + 17 + r) * LDA + R + 4 * q);
+                a0[4 * q] = v0.x; a0[4 * q + 1] = v0.y; a0[4 * q + 2] = v0.z; a0[4 * q + 3] = v0.w;
+                a1[4 * q] = v1.x; a1[4 * q + 1] = v1.y; a1[4 * q + 2] = v1.z; a1[4 * q + 3] = v1.w;
+            }
             const float *dcol = sA + R * LDA + R + 4 * c4;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const float a = arow[k];
                 const float4 d = *reinterpret_cast<const float4 *>(dcol + k * LDA);
-                acc.x = fmaf(a, d.x, acc.x); acc.y = fmaf(a, d.y, acc.y);
-                acc.z = fmaf(a, d.z, acc.z); acc.w = fmaf(a, d.w, acc.w);
+                y0.x = fmaf(a0[k], d.x, y0.x); y0.y = fmaf(a0[k], d.y, y0.y);
+                y0.z = fmaf(a0[k], d.z, y0.z); y0.w = fmaf(a0[k], d.w, y0.w);
+                y1.x = fmaf(a1[k], d.x, y1.x); y1.y = fmaf(a1[k], d.y, y1.y);
+                y1.z = fmaf(a1[k], d.z, y1.z); y1.w = fmaf(a1[k], d.w, y1.w);
             }
-            *reinterpret_cast<float4 *>(sA + (16 * p + r) * LDA + 32 + 4 * c4) = acc;
+            *reinterpret_cast<float4 *>(sA + (16 * p + r) * LDA + 32 + 4 * c4) = y0;
+            *reinterpret_cast<float4 *>(sA + (16 * p + r + 1) * LDA + 32 + 4 * c4) = y1;
         }
         named_bar(1, kKeyThreads);
-        if (t < 128) {
-            const float *drow = sA + (R + 16 + r) * LDA + R + 16;
+        if (t < 64) {
+            float d0[16], d1[16];   // rows r, r+1 of D_{2p+1}
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (R + 16 + r) * LDA + R + 16 + 4 * q);
+                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (R + 17 + r) * LDA + R + 16 + 4 * q);
+                d0[4 * q] = v0.x; d0[4 * q + 1] = v0.y; d0[4 * q + 2] = v0.z; d0[4 * q + 3] = v0.w;
+                d1[4 * q] = v1.x; d1[4 * q + 1] = v1.y; d1[4 * q + 2] = v1.z; d1[4 * q + 3] = v1.w;
+            }
             const float *ycol = sA + (16 * p) * LDA + 32 + 4 * c4;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 z0 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = z0;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const float d = drow[k];
                 const float4 y = *reinterpret_cast<const float4 *>(ycol + k * LDA);
-                acc.x = fmaf(d, y.x, acc.x); acc.y = fmaf(d, y.y, acc.y);
-                acc.z = fmaf(d, y.z, acc.z); acc.w = fmaf(d, y.w, acc.w);
+                z0.x = fmaf(d0[k], y.x, z0.x); z0.y = fmaf(d0[k], y.y, z0.y);
+                z0.z = fmaf(d0[k], y.z, z0.z); z0.w = fmaf(d0[k], y.w, z0.w);
+                z1.x = fmaf(d1[k], y.x, z1.x); z1.y = fmaf(d1[k], y.y, z1.y);
+                z1.z = fmaf(d1[k], y.z, z1.z); z1.w = fmaf(d1[k], y.w, z1.w);
             }
-            *reinterpret_cast<float4 *>(sA + (R + 16 + r) * LDA + R + 4 * c4) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            *reinterpret_cast<float4 *>(sA + (R + 16 + r) * LDA + R + 4 * c4) = make_float4(-z0.x, -z0.y, -z0.z, -z0.w);
+            *reinterpret_cast<float4 *>(sA + (R + 17 + r) * LDA + R + 4 * c4) = make_float4(-z1.x, -z1.y, -z1.z, -z1.w);
         }
         named_bar(1, kKeyThreads);
     }
-    {   // 3. 32 -> 64; Y in the upper-right block (rows r, cols 32 + 4c4)
-        const int r = t >> 3, c4 = t & 7;
-        const float *arow = sA + (32 + r) * LDA;
-        const float *tcol = sA + 4 * c4;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    {   // 3. 32 -> 64 (threads 0-127: two rows x one float4 each); Y in the
+        //    upper-right block, rows r, cols 32 + 4c4
+        const int r = 2 * (t >> 3), c4 = t & 7;
+        if (t < 128) {
+            float a0[32], a1[32];   // rows r, r+1 of A_ba
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {   // Y = A_ba T_a
-            const float a = arow[k];
-            const float4 tv = *reinterpret_cast<const float4 *>(tcol + k * LDA);
-            acc.x = fmaf(a, tv.x, acc.x); acc.y = fmaf(a, tv.y, acc.y);
-            acc.z = fmaf(a, tv.z, acc.z); acc.w = fmaf(a, tv.w, acc.w);
+            for (int q = 0; q < 8; ++q) {
+                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (32 + r) * LDA + 4 * q);
+                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (33 + r) * LDA + 4 * q);
+                a0[4 * q] = v0.x; a0[4 * q + 1] = v0.y; a0[4 * q + 2] = v0.z; a0[4 * q + 3] = v0.w;
+                a1[4 * q] = v1.x; a1[4 * q + 1] = v1.y; a1[4 * q + 2] = v1.z; a1[4 * q + 3] = v1.w;
+            }
+            const float *tcol = sA + 4 * c4;
+            float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {   // Y = A_ba T_a
+                const float4 tv = *reinterpret_cast<const float4 *>(tcol + k * LDA);
+                y0.x = fmaf(a0[k], tv.x, y0.x); y0.y = fmaf(a0[k], tv.y, y0.y);
+                y0.z = fmaf(a0[k], tv.z, y0.z); y0.w = fmaf(a0[k], tv.w, y0.w);
+                y1.x = fmaf(a1[k], tv.x, y1.x); y1.y = fmaf(a1[k], tv.y, y1.y);
+                y1.z = fmaf(a1[k], tv.z, y1.z); y1.w = fmaf(a1[k], tv.w, y1.w);
+            }
+            *reinterpret_cast<float4 *>(sA + r * LDA + 32 + 4 * c4) = y0;
+            *reinterpret_cast<float4 *>(sA + (r + 1) * LDA + 32 + 4 * c4) = y1;
         }
-        *reinterpret_cast<float4 *>(sA + r * LDA + 32 + 4 * c4) = acc;
         named_bar(1, kKeyThreads);
-        const float *drow = sA + (32 + r) * LDA + 32;
-        const float *ycol = sA + 32 + 4 * c4;
-        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < 128) {
+            float d0[32], d1[32];   // rows r, r+1 of T_b (zero above the diagonal)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {   // T_ba = -T_b Y  (T_b lower: zero for k > r)
-            const float d = drow[k];
-            const float4 y = *reinterpret_cast<const float4 *>(ycol + k * LDA);
-            acc.x = fmaf(d, y.x, acc.x); acc.y = fmaf(d, y.y, acc.y);
-            acc.z = fmaf(d, y.z, acc.z); acc.w = fmaf(d, y.w, acc.w);
+            for (int q = 0; q < 8; ++q) {
+                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (32 + r) * LDA + 32 + 4 * q);
+                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (33 + r) * LDA + 32 + 4 * q);
+                d0[4 * q] = v0.x; d0[4 * q + 1] = v0.y; d0[4 * q + 2] = v0.z; d0[4 * q + 3] = v0.w;
+                d1[4 * q] = v1.x; d1[4 * q + 1] = v1.y; d1[4 * q + 2] = v1.z; d1[4 * q + 3] = v1.w;
+            }
+            const float *ycol = sA + 32 + 4 * c4;
+            float4 z0 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = z0;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {   // T_ba = -T_b Y
+                const float4 y = *reinterpret_cast<const float4 *>(ycol + k * LDA);
+                z0.x = fmaf(d0[k], y.x, z0.x); z0.y = fmaf(d0[k], y.y, z0.y);
+                z0.z = fmaf(d0[k], y.z, z0.z); z0.w = fmaf(d0[k], y.w, z0.w);
+                z1.x = fmaf(d1[k], y.x, z1.x); z1.y = fmaf(d1[k], y.y, z1.y);
+                z1.z = fmaf(d1[k], y.z, z1.z); z1.w = fmaf(d1[k], y.w, z1.w);
+            }
+            *reinterpret_cast<float4 *>(sA + (32 + r) * LDA + 4 * c4) = make_float4(-z0.x, -z0.y, -z0.z, -z0.w);
+            *reinterpret_cast<float4 *>(sA + (33 + r) * LDA + 4 * c4) = make_float4(-z1.x, -z1.y, -z1.z, -z1.w);
         }
-        *reinterpret_cast<float4 *>(sA + (32 + r) * LDA + 4 * c4) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         named_bar(1, kKeyThreads);
     }
 }
