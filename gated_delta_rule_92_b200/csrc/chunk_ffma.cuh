@@ -61,7 +61,7 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     const int tid = threadIdx.x;
     const int j0 = blockIdx.x * NV, h = blockIdx.y, bb = blockIdx.z;
     const long head = (long)bb * H + h;
-    const int NC = T / C;
+    const int NC = (T + C - 1) / C;   // the last chunk may be partial (padded rows are zeros)
 
     // initial state slice
     for (int idx = tid; idx < DK * NV; idx += 256) {
@@ -71,20 +71,23 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
 
     for (int n = 0; n < NC; ++n) {
         const long tok0 = (long)bb * T + (long)n * C;   // token row of local r = 0
+        const int rows = min(C, T - n * C);              // valid rows of this chunk
         __syncthreads();
-        // ---- load the chunk (fp32 in shared memory)
+        // ---- load the chunk (fp32 in shared memory); rows past T are zeros,
+        // which leaves the recurrence unchanged (k = q = b = w = 0, no decay)
         for (int idx = tid; idx < C * DK; idx += 256) {
             const int r = idx / DK, c = idx % DK;
             const long g = ((tok0 + r) * H + h) * DK + c;
-            sQ[r * LK + c] = ld_io(q + g);
-            sK[r * LK + c] = ld_io(k + g);
-            sE[r * LK + c] = ld_io(bg + g);
-            sG[r * LK + c] = ld_io(la + g);
+            const bool in = r < rows;
+            sQ[r * LK + c] = in ? ld_io(q + g) : 0.f;
+            sK[r * LK + c] = in ? ld_io(k + g) : 0.f;
+            sE[r * LK + c] = in ? ld_io(bg + g) : 0.f;
+            sG[r * LK + c] = in ? ld_io(la + g) : 0.f;
         }
         for (int idx = tid; idx < C * NV; idx += 256) {
             const int r = idx / NV, j = idx % NV;
             const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
-            sWV[r * LC + j] = ld_io(wg + g) * ld_io(v + g);
+            sWV[r * LC + j] = (r < rows) ? ld_io(wg + g) * ld_io(v + g) : 0.f;
         }
         __syncthreads();
         // ---- cumulative log-decay per key channel and the scaled operands
@@ -164,8 +167,10 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
             for (int c = 0; c < DK; ++c) x = fmaf(sQ[r * LK + c], sS[c * LC + j], x);
             for (int i = 0; i <= r; ++i) x = fmaf(sP[r * LC + i], sU[i * LC + j], x);
             const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
-            if constexpr (sizeof(IO) == 4) o[g] = x;
-            else o[g] = __float2bfloat16_rn(x);
+            if (r < rows) {
+                if constexpr (sizeof(IO) == 4) o[g] = x;
+                else o[g] = __float2bfloat16_rn(x);
+            }
         }
         __syncthreads();
         // ---- S <- diag(gamma_C) (S + K~^T U)

@@ -264,9 +264,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int j0 = blockIdx.x * NV, h = blockIdx.y, bb = blockIdx.z;
-    const int NC = T / Cfg::C;
+    const int NC = (T + Cfg::C - 1) / Cfg::C;   // the last chunk may be partial
     const long head = (long)bb * H + h;
-    const int row0 = bb * T;   // TMA token coordinate of t = 0 for this batch row
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *qkb_full = bars + 0;    // [2] TMA q, k, b of a chunk landed (stage)
@@ -317,17 +316,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (warp == 12) {
         // ============================================================ producer
         if ((tid & 31) == 0 && NC > 0) {
+            // Token tiles are addressed (channel, head, token, batch); rows past T
+            // are outside the tensor and TMA fills them with zeros, which makes
+            // padded tokens exact no-ops of the recurrence (k = q = b = w = 0 and
+            // log_alpha = 0).
             auto prefetch = [&](int n) {
-                const int r = row0 + n * 64;
+                const int r = n * 64;
                 for (int kb = 0; kb < DK / 64; ++kb) {
-                    tma_prefetch_l2_3d(&tm_la, kb * 64, h, r);
-                    tma_prefetch_l2_3d(&tm_q, kb * 64, h, r);
-                    tma_prefetch_l2_3d(&tm_k, kb * 64, h, r);
-                    tma_prefetch_l2_3d(&tm_b, kb * 64, h, r);
+                    tma_prefetch_l2_4d(&tm_la, kb * 64, h, r, bb);
+                    tma_prefetch_l2_4d(&tm_q, kb * 64, h, r, bb);
+                    tma_prefetch_l2_4d(&tm_k, kb * 64, h, r, bb);
+                    tma_prefetch_l2_4d(&tm_b, kb * 64, h, r, bb);
                 }
                 for (int vb = 0; vb < Cfg::VB; ++vb) {
-                    tma_prefetch_l2_3d(&tm_v, j0 + vb * 64, h, r);
-                    tma_prefetch_l2_3d(&tm_w, j0 + vb * 64, h, r);
+                    tma_prefetch_l2_4d(&tm_v, j0 + vb * 64, h, r, bb);
+                    tma_prefetch_l2_4d(&tm_w, j0 + vb * 64, h, r, bb);
                 }
             };
             for (int p = 0; p < Cfg::PREFETCH && p < NC; ++p) prefetch(p);
@@ -336,33 +339,33 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             while (nq < NC || nl < NC || nv < NC) {
                 bool progress = false;
                 if (nq < NC && (nq < 2 || mbar_try_wait(&empty[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
-                    const int s = nq & 1, r = row0 + nq * 64;
+                    const int s = nq & 1, r = nq * 64;
                     const uint32_t oqe = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, ok = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
                     mbar_arrive_expect_tx(&qkb_full[s], 3u * Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb) {
-                        tma_load_3d(smem + oqe + kb * 16384, &tm_q, &qkb_full[s], kb * 64, h, r);
-                        tma_load_3d(smem + oqe + kb * 16384 + 8192, &tm_b, &qkb_full[s], kb * 64, h, r);
-                        tma_load_3d(smem + ok + kb * 8192, &tm_k, &qkb_full[s], kb * 64, h, r);
+                        tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qkb_full[s], kb * 64, h, r, bb);
+                        tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qkb_full[s], kb * 64, h, r, bb);
+                        tma_load_4d(smem + ok + kb * 8192, &tm_k, &qkb_full[s], kb * 64, h, r, bb);
                     }
                     if (nq + Cfg::PREFETCH < NC) prefetch(nq + Cfg::PREFETCH);
                     ++nq;
                     progress = true;
                 }
                 if (nl < NC && nl < nq && (nl < 1 || mbar_try_wait(lw_free, static_cast<uint32_t>((nl - 1) & 1)))) {
-                    const int r = row0 + nl * 64;
+                    const int r = nl * 64;
                     mbar_arrive_expect_tx(lw_full, Cfg::KEY_TILE + Cfg::VAL_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_3d(smem + Cfg::OFF_LA + kb * 8192, &tm_la, lw_full, kb * 64, h, r);
+                        tma_load_4d(smem + Cfg::OFF_LA + kb * 8192, &tm_la, lw_full, kb * 64, h, r, bb);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_load_3d(smem + Cfg::OFF_W + vb * 8192, &tm_w, lw_full, j0 + vb * 64, h, r);
+                        tma_load_4d(smem + Cfg::OFF_W + vb * 8192, &tm_w, lw_full, j0 + vb * 64, h, r, bb);
                     ++nl;
                     progress = true;
                 }
                 if (nv < NC && nv < nq && (nv < 1 || mbar_try_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
-                    const int r = row0 + nv * 64;
+                    const int r = nv * 64;
                     mbar_arrive_expect_tx(v_full, Cfg::VAL_TILE);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_load_3d(smem + Cfg::OFF_V + vb * 8192, &tm_v, v_full, j0 + vb * 64, h, r);
+                        tma_load_4d(smem + Cfg::OFF_V + vb * 8192, &tm_v, v_full, j0 + vb * 64, h, r, bb);
                     ++nv;
                     progress = true;
                 }
@@ -455,6 +458,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                               ks > 0 ? 1u : 0u);
                 umma_commit(bk1);
             }
+            // W.V in place in the v tile while MMA1 runs (the solve scratch does not
+            // touch the w tile)
+            {
+                const bool ok = mbar_wait(v_full, static_cast<uint32_t>(m & 1), wait_ns);
+                if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
+#pragma unroll
+                for (int it = 0; it < Cfg::VAL_TILE / 16 / kKeyThreads; ++it) {
+                    const uint32_t off = (t + it * kKeyThreads) * 16u;
+                    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+                    ld_shared_v4(sb + Cfg::OFF_V + off, a0, a1, a2, a3);
+                    ld_shared_v4(sb + Cfg::OFF_W + off, b0, b1, b2, b3);
+                    const uint4 r4 = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));
+                    st_shared_v4(sb + Cfg::OFF_V + off, r4.x, r4.y, r4.z, r4.w);
+                }
+            }
             {
                 const bool ok = mbar_wait(bk1, ph1, wait_ns);
                 ph1 ^= 1u;
@@ -493,20 +511,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             named_bar(1, kKeyThreads);
             // ------------------------------------------ T = (I + A)^{-1}
             unit_lower_inverse64<Cfg::LDA>(sA, t);
-            // W.V in place in the v tile (after the solve: the v load has landed)
-            {
-                const bool ok = mbar_wait(v_full, static_cast<uint32_t>(m & 1), wait_ns);
-                if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
-#pragma unroll
-                for (int it = 0; it < Cfg::VAL_TILE / 16 / kKeyThreads; ++it) {
-                    const uint32_t off = (t + it * kKeyThreads) * 16u;
-                    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-                    ld_shared_v4(sb + Cfg::OFF_V + off, a0, a1, a2, a3);
-                    ld_shared_v4(sb + Cfg::OFF_W + off, b0, b1, b2, b3);
-                    const uint4 r4 = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));
-                    st_shared_v4(sb + Cfg::OFF_V + off, r4.x, r4.y, r4.z, r4.w);
-                }
-            }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
                 // the scratch's last rows overlap the T tile
                 uint32_t tp[2][4];
@@ -720,18 +724,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc_fence_after();
             if ((warp & 3) < 2) {
-                const int r = t;   // output row r (TMEM lanes 0-63)
-                __nv_bfloat16 *orow = o + (((long)row0 + (long)n * 64 + r) * H + h) * (long)d_v + j0;
+                const int r = t;   // output row r (TMEM lanes 0-63); rows past T are padding
+                const bool valid = n * 64 + r < T;
+                __nv_bfloat16 *orow = o + (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0;
 #pragma unroll 1
                 for (int jc = 0; jc < NV / 32; ++jc) {
                     float x[32];
                     tmem_ld32(t_X + lane_q + jc * 32, x);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + jc * 32);
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + jc * 32);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int e = 8 * q4;
-                        dst[q4] = make_uint4(pack_bf16x2(x[e], x[e + 1]), pack_bf16x2(x[e + 2], x[e + 3]),
-                                             pack_bf16x2(x[e + 4], x[e + 5]), pack_bf16x2(x[e + 6], x[e + 7]));
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int e = 8 * q4;
+                            dst[q4] = make_uint4(pack_bf16x2(x[e], x[e + 1]), pack_bf16x2(x[e + 2], x[e + 3]),
+                                                 pack_bf16x2(x[e + 4], x[e + 5]), pack_bf16x2(x[e + 6], x[e + 7]));
+                        }
                     }
                 }
             }

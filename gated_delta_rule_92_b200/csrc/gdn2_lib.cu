@@ -55,16 +55,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Token tensor [B, T, H, d] bf16 viewed as 3-D (d, H, B*T); box = 64 columns
-// x 1 head x 64 tokens, 128-byte swizzle.
-bool make_token_map(CUtensorMap *m, const void *base, long BT, int H, int d) {
+// Token tensor [B, T, H, d] bf16 viewed as 4-D (d, H, T, B); box = 64 channels
+// x 1 head x 64 tokens x 1 sequence, 128-byte swizzle.  Boxes that run past T
+// are zero-filled by the TMA unit (a partial last chunk).
+bool make_token_map(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)BT};
-    cuuint64_t strides[2] = {(cuuint64_t)d * 2u, (cuuint64_t)H * (cuuint64_t)d * 2u};
-    cuuint32_t box[3] = {64, 1, 64};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2u, (cuuint64_t)H * (cuuint64_t)d * 2u,
+                             (cuuint64_t)T * (cuuint64_t)H * (cuuint64_t)d * 2u};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -74,10 +76,9 @@ gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void 
                         const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st) {
     using Cfg = TcCfg<DK, NV>;
     CUtensorMap tq, tk, tla, tb, tv, tw;
-    const long BT = (long)B * T;
-    if (!make_token_map(&tq, q, BT, H, DK) || !make_token_map(&tk, k, BT, H, DK) ||
-        !make_token_map(&tla, la, BT, H, DK) || !make_token_map(&tb, b, BT, H, DK) ||
-        !make_token_map(&tv, v, BT, H, d_v) || !make_token_map(&tw, w, BT, H, d_v))
+    if (!make_token_map(&tq, q, B, T, H, DK) || !make_token_map(&tk, k, B, T, H, DK) ||
+        !make_token_map(&tla, la, B, T, H, DK) || !make_token_map(&tb, b, B, T, H, DK) ||
+        !make_token_map(&tv, v, B, T, H, d_v) || !make_token_map(&tw, w, B, T, H, d_v))
         return GDN2_ERR_CUDA;
     auto kern = chunk_fwd_tc_kernel<DK, NV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
@@ -129,7 +130,6 @@ gdn2_status_t check_chunk(const void *q, const void *k, const void *v, const voi
     if (chunk != 64) return GDN2_ERR_UNSUPPORTED;
     if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
     if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
-    if (T % chunk != 0) return GDN2_ERR_UNSUPPORTED;
     if ((long)B * T > INT_MAX || B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;
     return GDN2_OK;
 }

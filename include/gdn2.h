@@ -81,8 +81,10 @@ typedef enum {
  *   chunk              : chunk length; must be 64 (the README default).
  *
  * Built shapes: d_k in {64, 128}; d_v a multiple of 64 with d_v <= 512;
- * T a multiple of `chunk` (T = 0 is allowed: o is empty, token pointers may
- * be NULL, and S_T = S0).
+ * any T >= 0.  A last chunk shorter than `chunk` is processed as if padded
+ * with zero tokens (q = k = v = b = w = 0, log_alpha = 0), which leaves the
+ * state and the valid outputs unchanged; nothing is written past T.  T = 0 is
+ * allowed: o is empty, token pointers may be NULL, and S_T = S0.
  * Other shapes return GDN2_ERR_UNSUPPORTED.
  *
  * Precision: bf16 I/O runs the tensor-core kernel (bf16 operands, fp32

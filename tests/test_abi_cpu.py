@@ -66,7 +66,6 @@ def test_chunk_argument_validation_on_host(L):
     assert _chunk_call(L, dk=96) == 2
     assert _chunk_call(L, dv=96) == 2
     assert _chunk_call(L, dv=1024) == 2
-    assert _chunk_call(L, T=100) == 2                    # T % chunk
     assert _chunk_call(L, B=70000) == 2
 
 

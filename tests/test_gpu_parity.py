@@ -74,6 +74,40 @@ def test_chunk_cuda_core_small_all_heads(g, case):
     _check_chunk(g, g.chunk_fwd_cuda_core, inp)
 
 
+# ------------------------------------------- partial last chunk (T % 64 != 0)
+TAILS = [  # B, T, H, d_k, d_v, dtype
+    (2, 100, 2, 128, 128, torch.bfloat16),
+    (1, 1, 2, 128, 256, torch.bfloat16),
+    (3, 65, 1, 64, 64, torch.bfloat16),
+    (1, 191, 2, 128, 64, torch.bfloat16),
+    (2, 37, 2, 64, 128, torch.float32),
+    (1, 130, 1, 128, 128, torch.float32),
+]
+
+
+@cuda
+@pytest.mark.parametrize("case", TAILS, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}k{c[3]}v{c[4]}{str(c[5])[6:]}")
+@pytest.mark.parametrize("impl", ["chunk_fwd", "chunk_fwd_cuda_core"])
+def test_chunk_partial_last_chunk(g, case, impl):
+    B, T, H, dk, dv, dt = case
+    inp = W.draw(B, T, H, dk, dv, seed=40 + T, dtype=dt, b_scale=2.0, s0_std=0.1)
+    _check_chunk(g, getattr(g, impl), inp)
+
+
+@cuda
+def test_partial_chunk_writes_nothing_past_T(g):
+    """Batch rows are contiguous: the padded rows of row b's last chunk are
+    row b+1's first tokens, which must be neither read as padding nor written."""
+    B, T, H, dk, dv = 3, 70, 2, 128, 128
+    inp = W.draw(B, T, H, dk, dv, seed=8, dtype=torch.bfloat16)
+    d = to_dev(inp)
+    o = torch.full((B, T, H, dv), 3.0, dtype=torch.bfloat16, device="cuda")
+    g.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], None, o=o)
+    torch.cuda.synchronize()
+    ro, _ = oracle_chunk(inp)
+    assert rel_inf(heads_of(o, range(B * H), H), ro) <= TOL[torch.bfloat16]
+
+
 # ------------------------------------------------------- named workloads
 @cuda
 def test_workload_chunk_f32_small(g):
@@ -245,7 +279,11 @@ def test_bounded_wait_reports_timeout(g):
 
 @cuda
 def test_unsupported_shapes_rejected_on_device_pointers(g):
-    inp = to_dev(W.draw(1, 96, 1, 64, 64, seed=4, dtype=torch.bfloat16))
+    inp = to_dev(W.draw(1, 96, 1, 96, 64, seed=4, dtype=torch.bfloat16))
     with pytest.raises(g.Gdn2Error) as e:
         g.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"], None)
+    assert e.value.status == 2
+    inp = to_dev(W.draw(1, 64, 1, 64, 64, seed=4, dtype=torch.bfloat16))
+    with pytest.raises(g.Gdn2Error) as e:
+        g.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"], None, chunk=32)
     assert e.value.status == 2
