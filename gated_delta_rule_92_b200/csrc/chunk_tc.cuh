@@ -2,29 +2,28 @@
 //
 // Chunk algebra (the burn-gdn2 README recurrence, "Architecture" section,
 // regrouped over chunks of C = 64 tokens as in its "Chunk WY (train)" mode):
-//     G = L log_alpha            (L = lower-triangular ones: per-channel cumsum)
+//     G = cumsum_rows(log_alpha)  (per key channel)
 //     Q~ = Q.exp(G), K~ = K.exp(-G), E = B.K.exp(G)
 //     A = strict_lower(E K~^T),  P = lower(Q~ K~^T),  T = (I + A)^{-1}
 //     U = T (W.V) - (T E) S,     O = Q~ S + P U,      S' = diag(exp(G_C)) (S + K~^T U)
-// with S the fp32 state at the chunk start.  The README credits its chunk
-// speed-up to computing the cumulative sum as a batched matmul; here that is
-// one pair of tensor-core MMAs per chunk.
+// with S the fp32 state at the chunk start.
 //
 // One CTA (13 warps) owns one (b, h, NV-column slice of d_v) and walks the
 // T/64 chunks in order as a pipeline:
 //   producer warp 12 TMA loads (128B swizzle) of q, k, b (double buffered),
-//                   log_alpha, w and v (single buffered), L2 prefetch ahead.
+//                   log_alpha, w and v (single buffered, each refilled as soon
+//                   as its last reader is done), L2 prefetch ahead.
 //   key warps 0-7   chunk m, everything that does not depend on the state:
-//       MMA_G  G = L log_alpha -> TMEM (two M=64 MMAs: channels 0-63 in the
-//              lower half-lanes, 64-127 in the upper half-lanes, so one
-//              warp-wide TMEM load hands every thread one row x 64 channels)
-//       prep   Q~, E, K~ computed in place in the TMA tiles; W.V in place in
-//              the v tile; exp(G_C) for the state update
+//       prep   G by a running fp32 sum per channel pair, then Q~, E, K~ in
+//              place in the TMA tiles and exp(G_C) for the state update
+//       W.V    in place in the v tile
 //       MMA1   [Q~; E] K~^T -> TMEM (rows 0-63 P', rows 64-127 A')
 //       solve  T = (I + A)^{-1} in fp32 on CUDA cores (16x16 diagonal blocks
 //              by forward substitution, off-diagonal blocks by block products)
 //       MMA2   [. ; T] E       -> rows 64-127 = T E, back to bf16 over E
 //       MMA3   [. ; T] (W.V)   -> rows 64-127 = T (W.V)
+//     as a two-stage pipeline: warps 0-3 solve chunk m while warps 4-7 run
+//     the prep of chunk m+1 (exp(G_C) is triple buffered for that)
 //   chain warps 8-11 chunk m-1, the sequential state pass:
 //       MMA_s  [Q~; T E] S -> X (rows 0-63 Q~ S, rows 64-127 T E S)
 //       U      = T (W.V) - T E S  (bf16 into shared memory)
@@ -54,26 +53,27 @@ struct TcCfg {
     static constexpr uint32_t OFF_QE1 = 32768;
     static constexpr uint32_t OFF_K0 = 65536;              // K tile [kb][64 i][64 c]
     static constexpr uint32_t OFF_K1 = 81920;
-    static constexpr uint32_t OFF_LA = 98304;              // log_alpha [kb][64 s][64 c]; solve scratch
-    static constexpr uint32_t OFF_T = OFF_LA + 16384;      // T [64 r][64 i]; its first KB also scratch
-    static constexpr uint32_t OFF_W = OFF_T + 8192;        // w [jb][64 i][64 j]
-    static constexpr uint32_t OFF_V = OFF_W + VB * 8192u;  // v -> W.V
+    static constexpr uint32_t OFF_LA = 98304;              // log_alpha [kb][64 s][64 c]
+    static constexpr uint32_t OFF_W = OFF_LA + 16384;      // w [jb][64 i][64 j] (16 KB reserved); solve scratch
+    static constexpr uint32_t OFF_T = OFF_W + 16384;       // T [64 r][64 i]; its first KB also scratch
+    static constexpr uint32_t OFF_V = OFF_T + 8192;        // v -> W.V
     static constexpr uint32_t OFF_P0 = OFF_V + VB * 8192u; // P [64 r][64 i], stage 0
     static constexpr uint32_t OFF_P1 = OFF_P0 + 8192;      // P, stage 1
     static constexpr uint32_t OFF_S = OFF_P1 + 8192;       // bf16 S [jb][128 c][64 j]
     static constexpr uint32_t OFF_U = OFF_S + VB * 16384u; // U [jb][64 i][64 j]
-    static constexpr uint32_t OFF_L = OFF_U + VB * 8192u;  // L [64 r][64 s]
-    static constexpr uint32_t OFF_GC = OFF_L + 8192;       // exp(G_C) [2][128]
-    static constexpr uint32_t OFF_BAR = OFF_GC + 1024;
-    static constexpr uint32_t OFF_TMEMP = OFF_BAR + 256;
+    static constexpr uint32_t OFF_CARRY = OFF_U + VB * 8192u;   // cumsum carries [row block][128]
+    static constexpr uint32_t OFF_GC = OFF_CARRY + 2048;         // exp(G_C) [3][128]
+    static constexpr uint32_t OFF_BAR = OFF_GC + 1536;
+    static constexpr uint32_t OFF_TMEMP = OFF_BAR + 256;   // up to 32 mbarriers
     static constexpr uint32_t SMEM_BYTES = OFF_TMEMP + 16;
     static constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
-    // fp32 solve scratch A/T [64][68], in the log_alpha tile (dead once MMA_G
-    // has run) and the first KB of the T tile (rewritten after the solve)
+    // fp32 solve scratch A/T [64][68], in the w tile (dead once W.V is formed)
+    // and the first KB of the T tile (rewritten after the solve); the
+    // log_alpha tile is then free as soon as MMA_G has run
     static constexpr int LDA = 68;
-    static constexpr uint32_t OFF_SCR = OFF_LA;
+    static constexpr uint32_t OFF_SCR = OFF_W;
     static_assert(64 * LDA * 4 <= 16384 + 8192, "solve scratch");
-    // TMEM columns: [KT 128: G, then P'/A', then T E][T(W.V) NV][X NV][S NV]
+    // TMEM columns: [KT 128: P'/A', then T E][T(W.V) NV][X NV][S NV]
     static constexpr uint32_t T_KT = 0, T_UT = 128, T_X = 128 + NV, T_S = 128 + 2 * NV;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int PREFETCH = 3;
@@ -100,22 +100,63 @@ constexpr int kKeyThreads = 256;     // warps 0-7
 constexpr int kChainThreads = 128;   // warps 8-11
 constexpr int kTcThreads = kKeyThreads + kChainThreads + 32;   // + producer warp 12
 
+// fp32 -> tf32 (round to nearest, ties away from zero), as a tensor-core operand.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// D += A B for one m16n8k8 tile (tf32 inputs, fp32 accumulation), warp-wide.
+// Fragments (g = lane / 4, q = lane % 4): a = A[g][q], A[g+8][q], A[g][q+4],
+// A[g+8][q+4];  b = B[q][g], B[q+4][g];  d = D[g][2q], D[g][2q+1], D[g+8][2q],
+// D[g+8][2q+1].
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// One warp: C (16 x 16, row stride LDA) = sign * Am (16 x K) Bm (K x 16), all in
+// fp32 shared memory with row stride LDA, products in tf32 on the tensor cores.
+template <int LDA, int K>
+__device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, float *Cm, float sign, int lane) {
+    const int g = lane >> 2, q = lane & 3;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a[4] = {to_tf32(Am[g * LDA + k0 + q]), to_tf32(Am[(g + 8) * LDA + k0 + q]),
+                               to_tf32(Am[g * LDA + k0 + q + 4]), to_tf32(Am[(g + 8) * LDA + k0 + q + 4])};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t bf[2] = {to_tf32(Bm[(k0 + q) * LDA + 8 * nt + g]), to_tf32(Bm[(k0 + q + 4) * LDA + 8 * nt + g])};
+            mma_tf32(acc[nt], a, bf);
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        *reinterpret_cast<float2 *>(Cm + g * LDA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
+        *reinterpret_cast<float2 *>(Cm + (g + 8) * LDA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][2], sign * acc[nt][3]);
+    }
+}
+
 // T = (I + A)^{-1} for a strictly lower 64x64 A held in fp32 in sA (row
-// stride LDA), in place, by the 256 key threads:
+// stride LDA), in place, by 128 threads (4 warps):
 //   1. each 16x16 diagonal block D_k = (I + A_kk)^{-1} by right-looking
-//      forward substitution, one column per thread (threads 0-63);
+//      forward substitution in fp32, one column per thread (threads 0-63);
 //   2. 16 -> 32: T_{2p+1,2p} = -D_{2p+1} (A_{2p+1,2p} D_{2p}), p = 0, 1
-//      (threads 0-63);
+//      (warp p);
 //   3. 32 -> 64: T_ba = -T_b (A_ba T_a) with a = rows/cols 0-31, b = 32-63
-//      (threads 0-127).
-// Block products keep two rows of the left factor in registers per thread
-// and stream one float4 of the right factor per step, so each 128-bit
-// shared-memory load feeds eight FMAs.
-// The intermediate products go to the upper-right 32x32 block, which T
-// leaves zero; readers of T must mask columns above the diagonal.
-// Barriers are named barrier 1 (256 threads).
+//      (warp w: rows 16 (w % 2), columns 16 (w / 2) of each product).
+// The block products run on the tensor cores (mma.sync, tf32 inputs, fp32
+// accumulation); T is rounded to bf16 afterwards, which dominates the tf32
+// input rounding.  The intermediate products go to the upper-right 32x32
+// block, which T leaves zero; everywhere else above the diagonal the scratch
+// is exactly zero (given an A that is), so readers of T only zero that
+// block.  `bar` is a named barrier over exactly these 128 threads.
 template <int LDA>
-__device__ __forceinline__ void unit_lower_inverse64(float *sA, int t) {
+__device__ __forceinline__ void unit_lower_inverse64(float *sA, int t, int bar) {
+    const int w = t >> 5, lane = t & 31;
     {   // 1. diagonal blocks
         float x[16];
         const int R = (t >> 4) * 16, j = t & 15;
@@ -131,122 +172,138 @@ __device__ __forceinline__ void unit_lower_inverse64(float *sA, int t) {
                 for (int r = i + 1; r < 16; ++r) sacc[r] = fmaf(-blk[r * LDA + i], x[i], sacc[r]);
             }
         }
-        named_bar(1, kKeyThreads);
+        named_bar(bar, 128);
         if (t < 64) {
 #pragma unroll
             for (int r = 0; r < 16; ++r) sA[(R + r) * LDA + R + j] = x[r];
         }
-        named_bar(1, kKeyThreads);
+        named_bar(bar, 128);
     }
-    {   // 2. 16 -> 32 (threads 0-63: two rows x one float4 each); products in the
-        //    upper-right block, rows 16p + r, cols 32 + 4c4
-        const int p = (t >> 5) & 1, r = 2 * ((t >> 2) & 7), c4 = t & 3;
-        const int R = 32 * p;   // block (2p+1, 2p) lives at rows R+16.., cols R..
-        if (t < 64) {
-            float a0[16], a1[16];   // rows r, r+1 of A_{2p+1,2p}
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (R + 16 + r) * LDA + R + 4 * q);
-                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (R + 17 + r) * LDA + R + 4 * q);
-                a0[4 * q] = v0.x; a0[4 * q + 1] = v0.y; a0[4 * q + 2] = v0.z; a0[4 * q + 3] = v0.w;
-                a1[4 * q] = v1.x; a1[4 * q + 1] = v1.y; a1[4 * q + 2] = v1.z; a1[4 * q + 3] = v1.w;
-            }
-            const float *dcol = sA + R * LDA + R + 4 * c4;
-            float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float4 d = *reinterpret_cast<const float4 *>(dcol + k * LDA);
-                y0.x = fmaf(a0[k], d.x, y0.x); y0.y = fmaf(a0[k], d.y, y0.y);
-                y0.z = fmaf(a0[k], d.z, y0.z); y0.w = fmaf(a0[k], d.w, y0.w);
-                y1.x = fmaf(a1[k], d.x, y1.x); y1.y = fmaf(a1[k], d.y, y1.y);
-                y1.z = fmaf(a1[k], d.z, y1.z); y1.w = fmaf(a1[k], d.w, y1.w);
-            }
-            *reinterpret_cast<float4 *>(sA + (16 * p + r) * LDA + 32 + 4 * c4) = y0;
-            *reinterpret_cast<float4 *>(sA + (16 * p + r + 1) * LDA + 32 + 4 * c4) = y1;
-        }
-        named_bar(1, kKeyThreads);
-        if (t < 64) {
-            float d0[16], d1[16];   // rows r, r+1 of D_{2p+1}
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (R + 16 + r) * LDA + R + 16 + 4 * q);
-                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (R + 17 + r) * LDA + R + 16 + 4 * q);
-                d0[4 * q] = v0.x; d0[4 * q + 1] = v0.y; d0[4 * q + 2] = v0.z; d0[4 * q + 3] = v0.w;
-                d1[4 * q] = v1.x; d1[4 * q + 1] = v1.y; d1[4 * q + 2] = v1.z; d1[4 * q + 3] = v1.w;
-            }
-            const float *ycol = sA + (16 * p) * LDA + 32 + 4 * c4;
-            float4 z0 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = z0;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float4 y = *reinterpret_cast<const float4 *>(ycol + k * LDA);
-                z0.x = fmaf(d0[k], y.x, z0.x); z0.y = fmaf(d0[k], y.y, z0.y);
-                z0.z = fmaf(d0[k], y.z, z0.z); z0.w = fmaf(d0[k], y.w, z0.w);
-                z1.x = fmaf(d1[k], y.x, z1.x); z1.y = fmaf(d1[k], y.y, z1.y);
-                z1.z = fmaf(d1[k], y.z, z1.z); z1.w = fmaf(d1[k], y.w, z1.w);
-            }
-            *reinterpret_cast<float4 *>(sA + (R + 16 + r) * LDA + R + 4 * c4) = make_float4(-z0.x, -z0.y, -z0.z, -z0.w);
-            *reinterpret_cast<float4 *>(sA + (R + 17 + r) * LDA + R + 4 * c4) = make_float4(-z1.x, -z1.y, -z1.z, -z1.w);
-        }
-        named_bar(1, kKeyThreads);
+    if (w < 2) {   // 2. 16 -> 32, warp p = w; Y_p in rows 16p.., cols 32..
+        const int R = 32 * w;
+        float *Y = sA + (16 * w) * LDA + 32;
+        warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R, sA + R * LDA + R, Y, 1.f, lane);
+        __syncwarp();
+        warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R + 16, Y, sA + (R + 16) * LDA + R, -1.f, lane);
     }
-    {   // 3. 32 -> 64 (threads 0-127: two rows x one float4 each); Y in the
-        //    upper-right block, rows r, cols 32 + 4c4
-        const int r = 2 * (t >> 3), c4 = t & 7;
-        if (t < 128) {
-            float a0[32], a1[32];   // rows r, r+1 of A_ba
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (32 + r) * LDA + 4 * q);
-                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (33 + r) * LDA + 4 * q);
-                a0[4 * q] = v0.x; a0[4 * q + 1] = v0.y; a0[4 * q + 2] = v0.z; a0[4 * q + 3] = v0.w;
-                a1[4 * q] = v1.x; a1[4 * q + 1] = v1.y; a1[4 * q + 2] = v1.z; a1[4 * q + 3] = v1.w;
-            }
-            const float *tcol = sA + 4 * c4;
-            float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {   // Y = A_ba T_a
-                const float4 tv = *reinterpret_cast<const float4 *>(tcol + k * LDA);
-                y0.x = fmaf(a0[k], tv.x, y0.x); y0.y = fmaf(a0[k], tv.y, y0.y);
-                y0.z = fmaf(a0[k], tv.z, y0.z); y0.w = fmaf(a0[k], tv.w, y0.w);
-                y1.x = fmaf(a1[k], tv.x, y1.x); y1.y = fmaf(a1[k], tv.y, y1.y);
-                y1.z = fmaf(a1[k], tv.z, y1.z); y1.w = fmaf(a1[k], tv.w, y1.w);
-            }
-            *reinterpret_cast<float4 *>(sA + r * LDA + 32 + 4 * c4) = y0;
-            *reinterpret_cast<float4 *>(sA + (r + 1) * LDA + 32 + 4 * c4) = y1;
-        }
-        named_bar(1, kKeyThreads);
-        if (t < 128) {
-            float d0[32], d1[32];   // rows r, r+1 of T_b (zero above the diagonal)
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float4 v0 = *reinterpret_cast<const float4 *>(sA + (32 + r) * LDA + 32 + 4 * q);
-                const float4 v1 = *reinterpret_cast<const float4 *>(sA + (33 + r) * LDA + 32 + 4 * q);
-                d0[4 * q] = v0.x; d0[4 * q + 1] = v0.y; d0[4 * q + 2] = v0.z; d0[4 * q + 3] = v0.w;
-                d1[4 * q] = v1.x; d1[4 * q + 1] = v1.y; d1[4 * q + 2] = v1.z; d1[4 * q + 3] = v1.w;
-            }
-            const float *ycol = sA + 32 + 4 * c4;
-            float4 z0 = make_float4(0.f, 0.f, 0.f, 0.f), z1 = z0;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {   // T_ba = -T_b Y
-                const float4 y = *reinterpret_cast<const float4 *>(ycol + k * LDA);
-                z0.x = fmaf(d0[k], y.x, z0.x); z0.y = fmaf(d0[k], y.y, z0.y);
-                z0.z = fmaf(d0[k], y.z, z0.z); z0.w = fmaf(d0[k], y.w, z0.w);
-                z1.x = fmaf(d1[k], y.x, z1.x); z1.y = fmaf(d1[k], y.y, z1.y);
-                z1.z = fmaf(d1[k], y.z, z1.z); z1.w = fmaf(d1[k], y.w, z1.w);
-            }
-            *reinterpret_cast<float4 *>(sA + (32 + r) * LDA + 4 * c4) = make_float4(-z0.x, -z0.y, -z0.z, -z0.w);
-            *reinterpret_cast<float4 *>(sA + (33 + r) * LDA + 4 * c4) = make_float4(-z1.x, -z1.y, -z1.z, -z1.w);
-        }
-        named_bar(1, kKeyThreads);
+    named_bar(bar, 128);
+    {   // 3. 32 -> 64: Y = A_ba T_a into rows 0-31, cols 32-63; then T_ba = -T_b Y
+        const int rm = 16 * (w & 1), cn = 16 * (w >> 1);
+        warp_gemm16<LDA, 32>(sA + (32 + rm) * LDA, sA + cn, sA + rm * LDA + 32 + cn, 1.f, lane);
+        named_bar(bar, 128);
+        warp_gemm16<LDA, 32>(sA + (32 + rm) * LDA + 32, sA + 32 + cn, sA + (32 + rm) * LDA + cn, -1.f, lane);
+        named_bar(bar, 128);
     }
 }
 
-// 8 bf16 products of two 16-byte vectors, rounded back to bf16.
+// 8 bf16 products of two 16-byte vectors, rounded back to bf16 (packed bf16x2
+// multiplies: the exact product rounded once, as fp32 multiply + rounding).
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
 __device__ __forceinline__ uint4 mul_bf16x8(const uint4 &a, const uint4 &b) {
-    return make_uint4(pack_bf16x2(bf16_lo(a.x) * bf16_lo(b.x), bf16_hi(a.x) * bf16_hi(b.x)),
-                      pack_bf16x2(bf16_lo(a.y) * bf16_lo(b.y), bf16_hi(a.y) * bf16_hi(b.y)),
-                      pack_bf16x2(bf16_lo(a.z) * bf16_lo(b.z), bf16_hi(a.z) * bf16_hi(b.z)),
-                      pack_bf16x2(bf16_lo(a.w) * bf16_lo(b.w), bf16_hi(a.w) * bf16_hi(b.w)));
+    return make_uint4(mul_bf16x2(a.x, b.x), mul_bf16x2(a.y, b.y), mul_bf16x2(a.z, b.z), mul_bf16x2(a.w, b.w));
+}
+// 2^x (MUFU approximation, flush-to-zero).
+__device__ __forceinline__ float ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Prep of one chunk by 128 threads (thread g): the per-channel cumulative
+// log-decay G (fp32, in row order, kept as G log2(e)) and, in place in the TMA tiles,
+//     Q~ = q.exp(G),  E = b.k.exp(G),  K~ = k.exp(-G),
+// plus exp(G_C) (last row) into gc.  Thread g owns the channel quad
+// p = g % (DK/4) over a block of R consecutive rows; the running sum enters a
+// block with the totals of the blocks above it (exchanged through `carry` and
+// named barrier `bar` over the 128 threads).  A half-warp covers 16
+// consecutive quads = one 128-byte swizzled row, so the 8-byte shared
+// accesses are conflict-free.  Thread 0 arrives on `la_free` once every thread
+// holds its log_alpha values.
+template <int DK>
+__device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, uint32_t ola, float *gc,
+                                           float *carry, uint64_t *la_free, int g, int bar) {
+    constexpr int NP = DK / 4;      // channel quads
+    constexpr int NB = 128 / NP;    // row blocks
+    constexpr int R = 64 / NB;      // rows per thread
+    static_assert(NB * R == 64 && NB <= 8, "prep split");
+    const int p = g % NP, hb = g / NP;
+    const int kb = p >> 4, cb = (p & 15) * 8;   // channel block, byte in the 128-byte row
+    const uint8_t *la_t = smem + ola + kb * 8192;
+    uint8_t *q_t = smem + oqe + kb * 16384, *e_t = q_t + 8192, *k_t = smem + okt + kb * 8192;
+    auto off = [&](int r) { return r * 128 + ((((cb >> 4) ^ r) & 7) << 4) + (cb & 15); };
+    // running sums in log2 units (G log2(e)), so that exp(+-G) = 2^(+-sum)
+    constexpr float kLog2e = 1.4426950408889634f;
+    uint2 law[R];
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        law[i] = *reinterpret_cast<const uint2 *>(la_t + off(hb * R + i));
+        sum[0] = fmaf(bf16_lo(law[i].x), kLog2e, sum[0]);
+        sum[1] = fmaf(bf16_hi(law[i].x), kLog2e, sum[1]);
+        sum[2] = fmaf(bf16_lo(law[i].y), kLog2e, sum[2]);
+        sum[3] = fmaf(bf16_hi(law[i].y), kLog2e, sum[3]);
+    }
+    reinterpret_cast<float4 *>(carry)[hb * NP + p] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+    named_bar(bar, 128);
+    if (g == 0) mbar_arrive(la_free);   // log_alpha is in registers: the tile may be refilled
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sum[e] = 0.f;
+#pragma unroll
+    for (int h2 = 0; h2 < NB - 1; ++h2) {
+        if (h2 < hb) {
+            const float4 c4 = reinterpret_cast<const float4 *>(carry)[h2 * NP + p];
+            sum[0] += c4.x;
+            sum[1] += c4.y;
+            sum[2] += c4.z;
+            sum[3] += c4.w;
+        }
+    }
+    // rows in batches: the tiles are rewritten in place, so loads of a batch
+    // cannot be hoisted above the previous batch's stores by the compiler
+    constexpr int RB = 2;
+#pragma unroll
+    for (int i0 = 0; i0 < R; i0 += RB) {
+        uint2 qw[RB], kw[RB], bw[RB];
+        int o[RB];
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            o[j] = off(hb * R + i0 + j);
+            qw[j] = *reinterpret_cast<const uint2 *>(q_t + o[j]);
+            kw[j] = *reinterpret_cast<const uint2 *>(k_t + o[j]);
+            bw[j] = *reinterpret_cast<const uint2 *>(e_t + o[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+            const uint2 la2 = law[i0 + j];
+            sum[0] = fmaf(bf16_lo(la2.x), kLog2e, sum[0]);
+            sum[1] = fmaf(bf16_hi(la2.x), kLog2e, sum[1]);
+            sum[2] = fmaf(bf16_lo(la2.y), kLog2e, sum[2]);
+            sum[3] = fmaf(bf16_hi(la2.y), kLog2e, sum[3]);
+            const uint32_t qv[2] = {qw[j].x, qw[j].y}, kv[2] = {kw[j].x, kw[j].y}, bv[2] = {bw[j].x, bw[j].y};
+            uint32_t oq[2], oe[2], ok[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float ga0 = ex2(sum[2 * h]), ga1 = ex2(sum[2 * h + 1]);
+                const float iv0 = ex2(-sum[2 * h]), iv1 = ex2(-sum[2 * h + 1]);
+                const float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
+                oq[h] = pack_bf16x2(bf16_lo(qv[h]) * ga0, bf16_hi(qv[h]) * ga1);
+                oe[h] = pack_bf16x2(bf16_lo(bv[h]) * k0 * ga0, bf16_hi(bv[h]) * k1 * ga1);
+                ok[h] = pack_bf16x2(k0 * iv0, k1 * iv1);
+            }
+            *reinterpret_cast<uint2 *>(q_t + o[j]) = make_uint2(oq[0], oq[1]);
+            *reinterpret_cast<uint2 *>(e_t + o[j]) = make_uint2(oe[0], oe[1]);
+            *reinterpret_cast<uint2 *>(k_t + o[j]) = make_uint2(ok[0], ok[1]);
+        }
+    }
+    if (hb == NB - 1) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) gc[4 * p + e] = ex2(sum[e]);
+    }
+    fence_proxy_async_smem();
 }
 
 template <int DK, int NV>
@@ -268,35 +325,31 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const long head = (long)bb * H + h;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-    uint64_t *qkb_full = bars + 0;    // [2] TMA q, k, b of a chunk landed (stage)
-    uint64_t *lw_full = bars + 2;     // TMA log_alpha, w landed
+    uint64_t *qb_full = bars + 0;     // [2] TMA q, b of a chunk landed (stage)
+    uint64_t *la_full = bars + 2;     // TMA log_alpha landed
     uint64_t *v_full = bars + 3;      // TMA v landed
-    uint64_t *lw_free = bars + 4;     // key done with log_alpha/w tiles (and the solve scratch)
+    uint64_t *la_free = bars + 4;     // the prep holds log_alpha in registers
     uint64_t *v_free = bars + 5;      // key done with W.V (MMA3 complete)
+    uint64_t *w_full = bars + 19;     // TMA w landed
+    uint64_t *w_free = bars + 20;     // key done with the w tile (W.V formed, solve scratch released)
+    uint64_t *k_full = bars + 21;     // [2] TMA k of a chunk landed (stage)
+    uint64_t *empty_k = bars + 23;    // [2] chain's MMA_u done: K~ tile of the stage free
+    uint64_t *empty_pg = bars + 25;   // [2] chain done with P of the stage
     uint64_t *full = bars + 6;        // [2] key products of a chunk ready
-    uint64_t *empty = bars + 8;       // [2] chain done with a stage
+    uint64_t *empty_qe = bars + 8;    // [2] chain's MMA_s done: Q~/(T E) tiles of the stage free
     uint64_t *utfree = bars + 10;     // chain read T(W.V) and MMA_s done
-    uint64_t *bG = bars + 11, *bk1 = bars + 12, *bk2 = bars + 13;
+    uint64_t *bk1 = bars + 12, *bk2 = bars + 13;
     uint64_t *bc1 = bars + 14, *bc2 = bars + 15, *bc3 = bars + 16;
-    uint64_t *drain = bars + 17;      // [2]
+    uint64_t *drain = bars + 17;      // [2] teardown: key and chain MMA issuers
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_TMEMP);
     float *gC = reinterpret_cast<float *>(smem + Cfg::OFF_GC);
     float *sA = reinterpret_cast<float *>(smem + Cfg::OFF_SCR);
 
     // ---------------------------------------------------------------- setup
-    for (uint32_t off = tid * 16u; off < Cfg::OFF_L; off += kTcThreads * 16u) st_shared_v4(sb + off, 0u, 0u, 0u, 0u);
-    for (int i = tid; i < 512; i += kTcThreads) {   // L: lower-triangular ones, K-major [r][s]
-        const int r = i >> 3, ch = i & 7;
-        uint32_t p[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int s0 = ch * 8 + 2 * e;
-            p[e] = pack_bf16x2(s0 <= r ? 1.f : 0.f, s0 + 1 <= r ? 1.f : 0.f);
-        }
-        st_shared_v4(sb + Cfg::OFF_L + sw128_chunk(r, ch), p[0], p[1], p[2], p[3]);
-    }
+    for (uint32_t off = tid * 16u; off < Cfg::OFF_CARRY; off += kTcThreads * 16u) st_shared_v4(sb + off, 0u, 0u, 0u, 0u);
+    for (int i = tid; i < 3 * 128; i += kTcThreads) gC[i] = 1.f;   // channels >= d_k keep exp(G_C) = 1
     if (tid == 0) {
-        for (int i = 0; i < 19; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 27; ++i) mbar_init(bars + i, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -334,34 +387,48 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             };
             for (int p = 0; p < Cfg::PREFETCH && p < NC; ++p) prefetch(p);
-            int nq = 0, nl = 0, nv = 0;   // next chunk to load for each group
+            int nq = 0, nk = 0, nl = 0, nw = 0, nv = 0;   // next chunk to load for each group
             uint64_t t0 = globaltimer_ns();
-            while (nq < NC || nl < NC || nv < NC) {
+            while (nq < NC || nk < NC || nl < NC || nw < NC || nv < NC) {
                 bool progress = false;
-                if (nq < NC && (nq < 2 || mbar_try_wait(&empty[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
+                if (nq < NC && (nq < 2 || mbar_test_wait(&empty_qe[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
                     const int s = nq & 1, r = nq * 64;
-                    const uint32_t oqe = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, ok = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
-                    mbar_arrive_expect_tx(&qkb_full[s], 3u * Cfg::KEY_TILE);
+                    const uint32_t oqe = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0;
+                    mbar_arrive_expect_tx(&qb_full[s], 2u * Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb) {
-                        tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qkb_full[s], kb * 64, h, r, bb);
-                        tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qkb_full[s], kb * 64, h, r, bb);
-                        tma_load_4d(smem + ok + kb * 8192, &tm_k, &qkb_full[s], kb * 64, h, r, bb);
+                        tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qb_full[s], kb * 64, h, r, bb);
+                        tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qb_full[s], kb * 64, h, r, bb);
                     }
                     if (nq + Cfg::PREFETCH < NC) prefetch(nq + Cfg::PREFETCH);
                     ++nq;
                     progress = true;
                 }
-                if (nl < NC && nl < nq && (nl < 1 || mbar_try_wait(lw_free, static_cast<uint32_t>((nl - 1) & 1)))) {
-                    const int r = nl * 64;
-                    mbar_arrive_expect_tx(lw_full, Cfg::KEY_TILE + Cfg::VAL_TILE);
+                if (nk < NC && (nk < 2 || mbar_test_wait(&empty_k[nk & 1], static_cast<uint32_t>(((nk >> 1) - 1) & 1)))) {
+                    const int s = nk & 1, r = nk * 64;
+                    const uint32_t ok = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
+                    mbar_arrive_expect_tx(&k_full[s], Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_4d(smem + Cfg::OFF_LA + kb * 8192, &tm_la, lw_full, kb * 64, h, r, bb);
-                    for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_load_4d(smem + Cfg::OFF_W + vb * 8192, &tm_w, lw_full, j0 + vb * 64, h, r, bb);
+                        tma_load_4d(smem + ok + kb * 8192, &tm_k, &k_full[s], kb * 64, h, r, bb);
+                    ++nk;
+                    progress = true;
+                }
+                if (nl < NC && (nl < 1 || mbar_test_wait(la_free, static_cast<uint32_t>((nl - 1) & 1)))) {
+                    const int r = nl * 64;
+                    mbar_arrive_expect_tx(la_full, Cfg::KEY_TILE);
+                    for (int kb = 0; kb < DK / 64; ++kb)
+                        tma_load_4d(smem + Cfg::OFF_LA + kb * 8192, &tm_la, la_full, kb * 64, h, r, bb);
                     ++nl;
                     progress = true;
                 }
-                if (nv < NC && nv < nq && (nv < 1 || mbar_try_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
+                if (nw < NC && (nw < 1 || mbar_test_wait(w_free, static_cast<uint32_t>((nw - 1) & 1)))) {
+                    const int r = nw * 64;
+                    mbar_arrive_expect_tx(w_full, Cfg::VAL_TILE);
+                    for (int vb = 0; vb < Cfg::VB; ++vb)
+                        tma_load_4d(smem + Cfg::OFF_W + vb * 8192, &tm_w, w_full, j0 + vb * 64, h, r, bb);
+                    ++nw;
+                    progress = true;
+                }
+                if (nv < NC && (nv < 1 || mbar_test_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
                     const int r = nv * 64;
                     mbar_arrive_expect_tx(v_full, Cfg::VAL_TILE);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
@@ -376,77 +443,28 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (tid < kKeyThreads) {
         // ============================================================ key side
+        // Two-stage pipeline over chunks: while warps 0-3 (group A) invert
+        // I + A of chunk m, warps 4-7 (group B) prepare chunk m+1; everything
+        // else is done by all eight warps.
         const int t = tid, l = tid & 31, kq = warp & 3, kh = warp >> 2;   // lane quarter, column half
-        const int prow = 16 * kq + (l & 15), phf = l >> 4;   // prep: row, channel half
-        uint32_t phG = 0, ph1 = 0, ph2 = 0;
-        for (int m = 0; m < NC; ++m) {
+        const bool grp_b = t >= 128;
+        uint32_t ph1 = 0, ph2 = 0;
+        float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
+        // prologue: prep of chunk 0 (group B)
+        if (NC > 0) {
+            bool ok = mbar_wait(la_full, 0u, wait_ns);
+            ok = ok && mbar_wait(&qb_full[0], 0u, wait_ns);
+            ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
+            if (group_any(1, kKeyThreads, !ok)) failed = true;
+            else if (grp_b) prep_chunk<DK>(smem, Cfg::OFF_QE0, Cfg::OFF_K0, Cfg::OFF_LA, gC, carry, la_free, t - 128, 4);
+        }
+        for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
             const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
             const uint32_t OP = s ? Cfg::OFF_P1 : Cfg::OFF_P0;
-            // ------------------------------------------------- MMA_G (cumsum)
-            {
-                const bool ok = mbar_wait(lw_full, static_cast<uint32_t>(m & 1), wait_ns);
-                if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
-            }
-            if (t == 0) {
-                tc_fence_after();
-                const uint32_t idg = idesc_bf16(64, 64, false, true);
-                for (int kb = 0; kb < DK / 64; ++kb)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(t_KT + (static_cast<uint32_t>(16 * kb) << 16), sdesc_sw128(sb + Cfg::OFF_L + ks * 32, 16, 1024),
-                                  sdesc_sw128(sb + Cfg::OFF_LA + kb * 8192 + ks * 2048, 8192, 1024), idg,
-                                  ks > 0 ? 1u : 0u);
-                umma_commit(bG);
-            }
-            {
-                bool ok = mbar_wait(&qkb_full[s], static_cast<uint32_t>((m >> 1) & 1), wait_ns);
-                ok = ok && mbar_wait(bG, phG, wait_ns);
-                phG ^= 1u;
-                if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
-            }
-            tc_fence_after();
-            // ------------------------------------------------------ prep
-            // thread: row prow, channels phf*64 + 32*kh + [0, 32)
-            {
-                float gv[32];
-                tmem_ld32(t_KT + lane_q + 32 * kh, gv);
-                if (phf < DK / 64) {
-                    const uint32_t qb = sb + OQE + phf * 16384, eb = qb + 8192, kb = sb + OK + phf * 8192;
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const uint32_t co = sw128_chunk(prow, 4 * kh + jj);
-                        uint32_t q0, q1, q2, q3, k0, k1, k2, k3, b0, b1, b2, b3;
-                        ld_shared_v4(qb + co, q0, q1, q2, q3);
-                        ld_shared_v4(kb + co, k0, k1, k2, k3);
-                        ld_shared_v4(eb + co, b0, b1, b2, b3);
-                        const uint32_t qw[4] = {q0, q1, q2, q3}, kw[4] = {k0, k1, k2, k3}, bw[4] = {b0, b1, b2, b3};
-                        uint32_t oq[4], oe[4], okk[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float g0 = gv[8 * jj + 2 * e], g1 = gv[8 * jj + 2 * e + 1];
-                            const float ga0 = __expf(g0), ga1 = __expf(g1);
-                            const float iv0 = __expf(-g0), iv1 = __expf(-g1);
-                            const float kv0 = bf16_lo(kw[e]), kv1 = bf16_hi(kw[e]);
-                            oq[e] = pack_bf16x2(bf16_lo(qw[e]) * ga0, bf16_hi(qw[e]) * ga1);
-                            oe[e] = pack_bf16x2(bf16_lo(bw[e]) * kv0 * ga0, bf16_hi(bw[e]) * kv1 * ga1);
-                            okk[e] = pack_bf16x2(kv0 * iv0, kv1 * iv1);
-                        }
-                        st_shared_v4(qb + co, oq[0], oq[1], oq[2], oq[3]);
-                        st_shared_v4(eb + co, oe[0], oe[1], oe[2], oe[3]);
-                        st_shared_v4(kb + co, okk[0], okk[1], okk[2], okk[3]);
-                    }
-                    if (prow == 63) {
-#pragma unroll
-                        for (int ch = 0; ch < 32; ++ch) gC[s * 128 + phf * 64 + 32 * kh + ch] = __expf(gv[ch]);
-                    }
-                } else if (prow == 63) {
-                    for (int ch = 0; ch < 32; ++ch) gC[s * 128 + phf * 64 + 32 * kh + ch] = 1.f;
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(1, kKeyThreads);
+            // prep of chunk m is complete: chunk 0 here, later chunks before the
+            // barriers that close the previous iteration
+            if (m == 0) named_bar(1, kKeyThreads);
             // ---------------------------------------------------------- MMA1
             if (t == 0) {
                 tc_fence_after();
@@ -458,10 +476,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                               ks > 0 ? 1u : 0u);
                 umma_commit(bk1);
             }
-            // W.V in place in the v tile while MMA1 runs (the solve scratch does not
-            // touch the w tile)
+            // W.V in place in the v tile while MMA1 runs (the solve scratch overlaps
+            // the w tile, so this comes first)
             {
-                const bool ok = mbar_wait(v_full, static_cast<uint32_t>(m & 1), wait_ns);
+                bool ok = mbar_wait(v_full, static_cast<uint32_t>(m & 1), wait_ns);
+                ok = ok && mbar_wait(w_full, static_cast<uint32_t>(m & 1), wait_ns);
                 if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
 #pragma unroll
                 for (int it = 0; it < Cfg::VAL_TILE / 16 / kKeyThreads; ++it) {
@@ -474,8 +493,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             {
-                const bool ok = mbar_wait(bk1, ph1, wait_ns);
+                bool ok = mbar_wait(bk1, ph1, wait_ns);
                 ph1 ^= 1u;
+                // P of this stage was last read by the chain two chunks ago
+                if (m >= 2) ok = ok && mbar_wait(&empty_pg[s], static_cast<uint32_t>(((m >> 1) - 1) & 1), wait_ns);
                 if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
             }
             tc_fence_after();
@@ -484,46 +505,71 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             {
                 float x[32];
                 tmem_ld32(t_KT + lane_q + 32 * kh, x);
-                if (kq < 2) {
-                    const int r = 32 * kq + l;
+                // warp-uniform block position: columns 32 kh.. against rows 32 (kq % 2)..;
+                // only the diagonal block needs per-element masks
+                const int rb = kq & 1, r = 32 * rb + l;
+                if (kq < 2) {   // P = lower(Q~ K~^T), diagonal included
+                    if (kh > rb) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t pp[4];
+                        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                    } else if (kh == rb) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 32 * kh + q4 * 8 + 2 * e;
-                            pp[e] = pack_bf16x2(i <= r ? x[q4 * 8 + 2 * e] : 0.f, i + 1 <= r ? x[q4 * 8 + 2 * e + 1] : 0.f);
-                        }
-                        st_shared_v4(sb + OP + sw128_chunk(r, 4 * kh + q4), pp[0], pp[1], pp[2], pp[3]);
+                        for (int e = 0; e < 32; ++e) x[e] = e <= l ? x[e] : 0.f;
                     }
-                } else {
-                    const int r = 32 * (kq - 2) + l;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const int i = 32 * kh + e;
-                        *reinterpret_cast<float4 *>(sA + r * Cfg::LDA + i) =
-                            make_float4(i < r ? x[e] : 0.f, i + 1 < r ? x[e + 1] : 0.f, i + 2 < r ? x[e + 2] : 0.f,
-                                        i + 3 < r ? x[e + 3] : 0.f);
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        st_shared_v4(sb + OP + sw128_chunk(r, 4 * kh + q4), pack_bf16x2(x[8 * q4], x[8 * q4 + 1]),
+                                     pack_bf16x2(x[8 * q4 + 2], x[8 * q4 + 3]), pack_bf16x2(x[8 * q4 + 4], x[8 * q4 + 5]),
+                                     pack_bf16x2(x[8 * q4 + 6], x[8 * q4 + 7]));
+                } else {        // A = strict_lower(E K~^T), fp32 into the solve scratch
+                    if (kh > rb) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                    } else if (kh == rb) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = e < l ? x[e] : 0.f;
                     }
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(sA + r * Cfg::LDA + 32 * kh + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
                 }
             }
             tc_fence_before();
             named_bar(1, kKeyThreads);
-            // ------------------------------------------ T = (I + A)^{-1}
-            unit_lower_inverse64<Cfg::LDA>(sA, t);
+            // ------------- group A: T = (I + A)^{-1};  group B: prep of chunk m+1
+            bool ok_b = true;
+            if (!grp_b) {
+                unit_lower_inverse64<Cfg::LDA>(sA, t, 3);
+            } else if (m + 1 < NC) {
+                const int sn = (m + 1) & 1;
+                const uint32_t pn = static_cast<uint32_t>(((m + 1) >> 1) & 1);
+                ok_b = mbar_wait(la_full, static_cast<uint32_t>((m + 1) & 1), wait_ns);
+                ok_b = ok_b && mbar_wait(&qb_full[sn], pn, wait_ns);
+                ok_b = ok_b && mbar_wait(&k_full[sn], pn, wait_ns);
+                ok_b = !group_any(4, 128, !ok_b);
+                if (ok_b)
+                    prep_chunk<DK>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, sn ? Cfg::OFF_K1 : Cfg::OFF_K0, Cfg::OFF_LA,
+                                        gC + ((m + 1) % 3) * 128, carry, la_free, t - 128, 4);
+            }
+            if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
                 // the scratch's last rows overlap the T tile
                 uint32_t tp[2][4];
 #pragma unroll
                 for (int it = 0; it < 2; ++it) {
                     const int idx = t + it * kKeyThreads, r = idx >> 3, ch = idx & 7, c0 = 8 * ch;
-                    const float4 a = *reinterpret_cast<const float4 *>(sA + r * Cfg::LDA + c0);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(sA + r * Cfg::LDA + c0 + 4);
-                    // T is unit lower triangular; the scratch above the diagonal is not T
-                    tp[it][0] = pack_bf16x2(c0 <= r ? a.x : 0.f, c0 + 1 <= r ? a.y : 0.f);
-                    tp[it][1] = pack_bf16x2(c0 + 2 <= r ? a.z : 0.f, c0 + 3 <= r ? a.w : 0.f);
-                    tp[it][2] = pack_bf16x2(c0 + 4 <= r ? b4.x : 0.f, c0 + 5 <= r ? b4.y : 0.f);
-                    tp[it][3] = pack_bf16x2(c0 + 6 <= r ? b4.z : 0.f, c0 + 7 <= r ? b4.w : 0.f);
+                    // T is unit lower triangular: the scratch above the diagonal is zero
+                    // except the upper-right 32x32 block, which holds the solve's products
+                    if (r < 32 && c0 >= 32) {
+                        tp[it][0] = tp[it][1] = tp[it][2] = tp[it][3] = 0u;
+                    } else {
+                        const float4 a = *reinterpret_cast<const float4 *>(sA + r * Cfg::LDA + c0);
+                        const float4 b4 = *reinterpret_cast<const float4 *>(sA + r * Cfg::LDA + c0 + 4);
+                        tp[it][0] = pack_bf16x2(a.x, a.y);
+                        tp[it][1] = pack_bf16x2(a.z, a.w);
+                        tp[it][2] = pack_bf16x2(b4.x, b4.y);
+                        tp[it][3] = pack_bf16x2(b4.z, b4.w);
+                    }
                 }
                 named_bar(1, kKeyThreads);
 #pragma unroll
@@ -534,7 +580,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             fence_proxy_async_smem();
             named_bar(1, kKeyThreads);
-            if (t == 0) mbar_arrive(lw_free);   // log_alpha (scratch) and w tiles are free
+            if (t == 0) mbar_arrive(w_free);   // w tile (solve scratch) is free
             // the chain must have read T(W.V) and run MMA_s of the previous chunk
             if (m >= 1) {
                 const bool ok = mbar_wait(utfree, static_cast<uint32_t>((m - 1) & 1), wait_ns);
@@ -641,6 +687,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ph1 ^= 1u;
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
+            if (t == 0) mbar_arrive(&empty_qe[s]);   // MMA_s has read Q~ and T E of this stage
             tc_fence_after();
             if ((warp & 3) >= 2) {
                 const int r = t - 64;   // U row r (TMEM lanes 64-127)
@@ -686,10 +733,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ph2 ^= 1u;
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
+            if (t == 0) mbar_arrive(&empty_k[s]);    // MMA_u has read K~ of this stage
             tc_fence_after();
             {
                 const int c = t;
-                const float gcv = gC[s * 128 + c];
+                const float gcv = gC[(n % 3) * 128 + c];
                 const bool last = (n + 1 == NC);
 #pragma unroll 1
                 for (int jc = 0; jc < NV / 32; ++jc) {
@@ -746,7 +794,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(2, kChainThreads);
-            if (t == 0) mbar_arrive(&empty[s]);
+            if (t == 0) mbar_arrive(&empty_pg[s]);
         }
         if (t == 0) {
             umma_commit(&drain[1]);
