@@ -10,9 +10,10 @@
 //
 // One CTA (13 warps) owns one (b, h, NV-column slice of d_v) and walks the
 // T/64 chunks in order as a pipeline:
-//   producer warp 12 TMA loads (128B swizzle) of q, k, b (double buffered),
-//                   log_alpha, w and v (single buffered, each refilled as soon
-//                   as its last reader is done), L2 prefetch ahead.
+//   producer warp 12 TMA loads (128B swizzle) of q, b (double buffered), k
+//                   (triple buffered), w and v (single buffered, each refilled
+//                   as soon as its last reader is done), L2 prefetch ahead;
+//                   log_alpha goes straight to the prep threads' registers.
 //   key warps 0-7   chunk m, everything that does not depend on the state:
 //       prep   G by a running fp32 sum per channel pair, then Q~, E, K~ in
 //              place in the TMA tiles and exp(G_C) for the state update
@@ -51,10 +52,8 @@ struct TcCfg {
     // 64 channels), so [Q; E] is a 128-row K-major operand per channel block.
     static constexpr uint32_t OFF_QE0 = 0;
     static constexpr uint32_t OFF_QE1 = 32768;
-    static constexpr uint32_t OFF_K0 = 65536;              // K tile [kb][64 i][64 c]
-    static constexpr uint32_t OFF_K1 = 81920;
-    static constexpr uint32_t OFF_LA = 98304;              // log_alpha [kb][64 s][64 c]
-    static constexpr uint32_t OFF_W = OFF_LA + 16384;      // w [jb][64 i][64 j] (16 KB reserved); solve scratch
+    static constexpr uint32_t OFF_K = 65536;               // K tiles [3 stages][kb][64 i][64 c]
+    static constexpr uint32_t OFF_W = OFF_K + 3 * 16384;   // w [jb][64 i][64 j] (16 KB reserved); solve scratch
     static constexpr uint32_t OFF_T = OFF_W + 16384;       // T [64 r][64 i]; its first KB also scratch
     static constexpr uint32_t OFF_V = OFF_T + 8192;        // v -> W.V
     static constexpr uint32_t OFF_P0 = OFF_V + VB * 8192u; // P [64 r][64 i], stage 0
@@ -213,43 +212,54 @@ __device__ __forceinline__ float ex2(float x) {
     return r;
 }
 
+// log_alpha of one chunk for the prep thread g (channel quad p = g % (DK/4),
+// rows R hb .. R hb + R - 1 with hb = g / (DK/4)), straight from HBM into
+// registers; rows past T read as zero (no decay on padding).
+template <int DK>
+struct PrepLA {
+    static constexpr int NP = DK / 4, NB = 128 / NP, R = 64 / NB;
+    uint2 v[R];
+    __device__ __forceinline__ void load(const __nv_bfloat16 *la, int bb, int n, int h, int T, int H, int g) {
+        const int p = g % NP, hb = g / NP;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int r = n * 64 + hb * R + i;
+            v[i] = r < T ? __ldg(reinterpret_cast<const uint2 *>(la + (((long)bb * T + r) * H + h) * DK + 4 * p))
+                         : make_uint2(0u, 0u);
+        }
+    }
+};
+
 // Prep of one chunk by 128 threads (thread g): the per-channel cumulative
 // log-decay G (fp32, in row order, kept as G log2(e)) and, in place in the TMA tiles,
 //     Q~ = q.exp(G),  E = b.k.exp(G),  K~ = k.exp(-G),
 // plus exp(G_C) (last row) into gc.  Thread g owns the channel quad
-// p = g % (DK/4) over a block of R consecutive rows; the running sum enters a
-// block with the totals of the blocks above it (exchanged through `carry` and
-// named barrier `bar` over the 128 threads).  A half-warp covers 16
-// consecutive quads = one 128-byte swizzled row, so the 8-byte shared
-// accesses are conflict-free.  Thread 0 arrives on `la_free` once every thread
-// holds its log_alpha values.
+// p = g % (DK/4) over a block of R consecutive rows (its log_alpha values in
+// `law`); the running sum enters a block with the totals of the blocks above
+// it (exchanged through `carry` and named barrier `bar` over the 128
+// threads).  A half-warp covers 16 consecutive quads = one 128-byte swizzled
+// row, so the 8-byte shared accesses are conflict-free.
 template <int DK>
-__device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, uint32_t ola, float *gc,
-                                           float *carry, uint64_t *la_free, int g, int bar) {
-    constexpr int NP = DK / 4;      // channel quads
-    constexpr int NB = 128 / NP;    // row blocks
-    constexpr int R = 64 / NB;      // rows per thread
+__device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLA<DK> &law,
+                                           float *gc, float *carry, int g, int bar) {
+    constexpr int NP = PrepLA<DK>::NP, NB = PrepLA<DK>::NB, R = PrepLA<DK>::R;
     static_assert(NB * R == 64 && NB <= 8, "prep split");
     const int p = g % NP, hb = g / NP;
     const int kb = p >> 4, cb = (p & 15) * 8;   // channel block, byte in the 128-byte row
-    const uint8_t *la_t = smem + ola + kb * 8192;
     uint8_t *q_t = smem + oqe + kb * 16384, *e_t = q_t + 8192, *k_t = smem + okt + kb * 8192;
     auto off = [&](int r) { return r * 128 + ((((cb >> 4) ^ r) & 7) << 4) + (cb & 15); };
     // running sums in log2 units (G log2(e)), so that exp(+-G) = 2^(+-sum)
     constexpr float kLog2e = 1.4426950408889634f;
-    uint2 law[R];
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-        law[i] = *reinterpret_cast<const uint2 *>(la_t + off(hb * R + i));
-        sum[0] = fmaf(bf16_lo(law[i].x), kLog2e, sum[0]);
-        sum[1] = fmaf(bf16_hi(law[i].x), kLog2e, sum[1]);
-        sum[2] = fmaf(bf16_lo(law[i].y), kLog2e, sum[2]);
-        sum[3] = fmaf(bf16_hi(law[i].y), kLog2e, sum[3]);
+        sum[0] = fmaf(bf16_lo(law.v[i].x), kLog2e, sum[0]);
+        sum[1] = fmaf(bf16_hi(law.v[i].x), kLog2e, sum[1]);
+        sum[2] = fmaf(bf16_lo(law.v[i].y), kLog2e, sum[2]);
+        sum[3] = fmaf(bf16_hi(law.v[i].y), kLog2e, sum[3]);
     }
     reinterpret_cast<float4 *>(carry)[hb * NP + p] = make_float4(sum[0], sum[1], sum[2], sum[3]);
     named_bar(bar, 128);
-    if (g == 0) mbar_arrive(la_free);   // log_alpha is in registers: the tile may be refilled
 #pragma unroll
     for (int e = 0; e < 4; ++e) sum[e] = 0.f;
 #pragma unroll
@@ -278,7 +288,7 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
         }
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
-            const uint2 la2 = law[i0 + j];
+            const uint2 la2 = law.v[i0 + j];
             sum[0] = fmaf(bf16_lo(la2.x), kLog2e, sum[0]);
             sum[1] = fmaf(bf16_hi(la2.x), kLog2e, sum[1]);
             sum[2] = fmaf(bf16_lo(la2.y), kLog2e, sum[2]);
@@ -309,8 +319,8 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
 template <int DK, int NV>
 __global__ void __launch_bounds__(kTcThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_b,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16 *__restrict__ la,
                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T,
                     int T, int H, int d_v, unsigned long long wait_ns) {
     using Cfg = TcCfg<DK, NV>;
@@ -325,22 +335,21 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const long head = (long)bb * H + h;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
-    uint64_t *qb_full = bars + 0;     // [2] TMA q, b of a chunk landed (stage)
-    uint64_t *la_full = bars + 2;     // TMA log_alpha landed
-    uint64_t *v_full = bars + 3;      // TMA v landed
-    uint64_t *la_free = bars + 4;     // the prep holds log_alpha in registers
-    uint64_t *v_free = bars + 5;      // key done with W.V (MMA3 complete)
-    uint64_t *w_full = bars + 19;     // TMA w landed
-    uint64_t *w_free = bars + 20;     // key done with the w tile (W.V formed, solve scratch released)
-    uint64_t *k_full = bars + 21;     // [2] TMA k of a chunk landed (stage)
-    uint64_t *empty_k = bars + 23;    // [2] chain's MMA_u done: K~ tile of the stage free
-    uint64_t *empty_pg = bars + 25;   // [2] chain done with P of the stage
-    uint64_t *full = bars + 6;        // [2] key products of a chunk ready
-    uint64_t *empty_qe = bars + 8;    // [2] chain's MMA_s done: Q~/(T E) tiles of the stage free
-    uint64_t *utfree = bars + 10;     // chain read T(W.V) and MMA_s done
-    uint64_t *bk1 = bars + 12, *bk2 = bars + 13;
-    uint64_t *bc1 = bars + 14, *bc2 = bars + 15, *bc3 = bars + 16;
-    uint64_t *drain = bars + 17;      // [2] teardown: key and chain MMA issuers
+    uint64_t *qb_full = bars + 0;     // [2] TMA q, b of a chunk landed (stage m % 2)
+    uint64_t *k_full = bars + 2;      // [3] TMA k of a chunk landed (stage m % 3)
+    uint64_t *v_full = bars + 5;      // TMA v landed
+    uint64_t *w_full = bars + 6;      // TMA w landed
+    uint64_t *v_free = bars + 7;      // key done with W.V (MMA3 complete)
+    uint64_t *w_free = bars + 8;      // key done with the w tile (W.V formed, solve scratch released)
+    uint64_t *full = bars + 9;        // [2] key products of a chunk ready
+    uint64_t *empty_qe = bars + 11;   // [2] chain's MMA_s done: Q~/(T E) tiles of the stage free
+    uint64_t *empty_k = bars + 13;    // [3] chain's MMA_u done: K~ tile of the stage free
+    uint64_t *empty_pg = bars + 16;   // [2] chain done with P of the stage
+    uint64_t *utfree = bars + 18;     // chain read T(W.V) and MMA_s done
+    uint64_t *bk1 = bars + 19, *bk2 = bars + 20;
+    uint64_t *bc1 = bars + 21, *bc2 = bars + 22, *bc3 = bars + 23;
+    uint64_t *drain = bars + 24;      // [2] teardown: key and chain MMA issuers
+    constexpr int kNumBars = 26;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_TMEMP);
     float *gC = reinterpret_cast<float *>(smem + Cfg::OFF_GC);
     float *sA = reinterpret_cast<float *>(smem + Cfg::OFF_SCR);
@@ -349,7 +358,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     for (uint32_t off = tid * 16u; off < Cfg::OFF_CARRY; off += kTcThreads * 16u) st_shared_v4(sb + off, 0u, 0u, 0u, 0u);
     for (int i = tid; i < 3 * 128; i += kTcThreads) gC[i] = 1.f;   // channels >= d_k keep exp(G_C) = 1
     if (tid == 0) {
-        for (int i = 0; i < 27; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -376,7 +385,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             auto prefetch = [&](int n) {
                 const int r = n * 64;
                 for (int kb = 0; kb < DK / 64; ++kb) {
-                    tma_prefetch_l2_4d(&tm_la, kb * 64, h, r, bb);
                     tma_prefetch_l2_4d(&tm_q, kb * 64, h, r, bb);
                     tma_prefetch_l2_4d(&tm_k, kb * 64, h, r, bb);
                     tma_prefetch_l2_4d(&tm_b, kb * 64, h, r, bb);
@@ -387,9 +395,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             };
             for (int p = 0; p < Cfg::PREFETCH && p < NC; ++p) prefetch(p);
-            int nq = 0, nk = 0, nl = 0, nw = 0, nv = 0;   // next chunk to load for each group
+            int nq = 0, nk = 0, nw = 0, nv = 0;   // next chunk to load for each group
             uint64_t t0 = globaltimer_ns();
-            while (nq < NC || nk < NC || nl < NC || nw < NC || nv < NC) {
+            while (nq < NC || nk < NC || nw < NC || nv < NC) {
                 bool progress = false;
                 if (nq < NC && (nq < 2 || mbar_test_wait(&empty_qe[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
                     const int s = nq & 1, r = nq * 64;
@@ -403,21 +411,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ++nq;
                     progress = true;
                 }
-                if (nk < NC && (nk < 2 || mbar_test_wait(&empty_k[nk & 1], static_cast<uint32_t>(((nk >> 1) - 1) & 1)))) {
-                    const int s = nk & 1, r = nk * 64;
-                    const uint32_t ok = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
-                    mbar_arrive_expect_tx(&k_full[s], Cfg::KEY_TILE);
+                if (nk < NC && (nk < 3 || mbar_test_wait(&empty_k[nk % 3], static_cast<uint32_t>((nk / 3 - 1) & 1)))) {
+                    const int s3 = nk % 3, r = nk * 64;
+                    mbar_arrive_expect_tx(&k_full[s3], Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_4d(smem + ok + kb * 8192, &tm_k, &k_full[s], kb * 64, h, r, bb);
+                        tma_load_4d(smem + Cfg::OFF_K + s3 * 16384 + kb * 8192, &tm_k, &k_full[s3], kb * 64, h, r, bb);
                     ++nk;
-                    progress = true;
-                }
-                if (nl < NC && (nl < 1 || mbar_test_wait(la_free, static_cast<uint32_t>((nl - 1) & 1)))) {
-                    const int r = nl * 64;
-                    mbar_arrive_expect_tx(la_full, Cfg::KEY_TILE);
-                    for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_4d(smem + Cfg::OFF_LA + kb * 8192, &tm_la, la_full, kb * 64, h, r, bb);
-                    ++nl;
                     progress = true;
                 }
                 if (nw < NC && (nw < 1 || mbar_test_wait(w_free, static_cast<uint32_t>((nw - 1) & 1)))) {
@@ -450,21 +449,24 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool grp_b = t >= 128;
         uint32_t ph1 = 0, ph2 = 0;
         float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
+        PrepLA<DK> lan;   // group B: log_alpha of the next chunk to prepare
         // prologue: prep of chunk 0 (group B)
         if (NC > 0) {
-            bool ok = mbar_wait(la_full, 0u, wait_ns);
-            ok = ok && mbar_wait(&qb_full[0], 0u, wait_ns);
+            if (grp_b) lan.load(la, bb, 0, h, T, H, t - 128);
+            bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK>(smem, Cfg::OFF_QE0, Cfg::OFF_K0, Cfg::OFF_LA, gC, carry, la_free, t - 128, 4);
+            else if (grp_b) prep_chunk<DK>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4);
         }
         for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
-            const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
+            const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = Cfg::OFF_K + (m % 3) * 16384u;
             const uint32_t OP = s ? Cfg::OFF_P1 : Cfg::OFF_P0;
             // prep of chunk m is complete: chunk 0 here, later chunks before the
             // barriers that close the previous iteration
             if (m == 0) named_bar(1, kKeyThreads);
+            // log_alpha of chunk m+1, a whole iteration ahead of its use
+            if (grp_b && m + 1 < NC) lan.load(la, bb, m + 1, h, T, H, t - 128);
             // ---------------------------------------------------------- MMA1
             if (t == 0) {
                 tc_fence_after();
@@ -541,15 +543,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!grp_b) {
                 unit_lower_inverse64<Cfg::LDA>(sA, t, 3);
             } else if (m + 1 < NC) {
-                const int sn = (m + 1) & 1;
-                const uint32_t pn = static_cast<uint32_t>(((m + 1) >> 1) & 1);
-                ok_b = mbar_wait(la_full, static_cast<uint32_t>((m + 1) & 1), wait_ns);
-                ok_b = ok_b && mbar_wait(&qb_full[sn], pn, wait_ns);
-                ok_b = ok_b && mbar_wait(&k_full[sn], pn, wait_ns);
+                const int sn = (m + 1) & 1, s3n = (m + 1) % 3;
+                ok_b = mbar_wait(&qb_full[sn], static_cast<uint32_t>(((m + 1) >> 1) & 1), wait_ns);
+                ok_b = ok_b && mbar_wait(&k_full[s3n], static_cast<uint32_t>(((m + 1) / 3) & 1), wait_ns);
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
-                    prep_chunk<DK>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, sn ? Cfg::OFF_K1 : Cfg::OFF_K0, Cfg::OFF_LA,
-                                        gC + ((m + 1) % 3) * 128, carry, la_free, t - 128, 4);
+                    prep_chunk<DK>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
+                                   gC + ((m + 1) % 3) * 128, carry, t - 128, 4);
             }
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
@@ -666,7 +666,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint32_t ph1 = 0, ph2 = 0, ph3 = 0;
         for (int n = 0; n < NC; ++n) {
             const int s = n & 1;
-            const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = s ? Cfg::OFF_K1 : Cfg::OFF_K0;
+            const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = Cfg::OFF_K + (n % 3) * 16384u;
             const uint32_t OP = s ? Cfg::OFF_P1 : Cfg::OFF_P0;
             {
                 const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((n >> 1) & 1), wait_ns);
@@ -733,7 +733,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ph2 ^= 1u;
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
-            if (t == 0) mbar_arrive(&empty_k[s]);    // MMA_u has read K~ of this stage
+            if (t == 0) mbar_arrive(&empty_k[n % 3]);   // MMA_u has read K~ of this stage
             tc_fence_after();
             {
                 const int c = t;

@@ -75,17 +75,17 @@ template <int DK, int NV>
 gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void *la, const void *b, const void *w,
                         const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st) {
     using Cfg = TcCfg<DK, NV>;
-    CUtensorMap tq, tk, tla, tb, tv, tw;
+    CUtensorMap tq, tk, tb, tv, tw;
     if (!make_token_map(&tq, q, B, T, H, DK) || !make_token_map(&tk, k, B, T, H, DK) ||
-        !make_token_map(&tla, la, B, T, H, DK) || !make_token_map(&tb, b, B, T, H, DK) ||
-        !make_token_map(&tv, v, B, T, H, d_v) || !make_token_map(&tw, w, B, T, H, d_v))
+        !make_token_map(&tb, b, B, T, H, DK) || !make_token_map(&tv, v, B, T, H, d_v) ||
+        !make_token_map(&tw, w, B, T, H, d_v))
         return GDN2_ERR_CUDA;
     auto kern = chunk_fwd_tc_kernel<DK, NV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
     dim3 grid(d_v / NV, H, B);
-    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tla, tb, tv, tw, S0, static_cast<__nv_bfloat16 *>(o), S_T, T,
-                                             H, d_v, kWaitNs);
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, static_cast<const __nv_bfloat16 *>(la), S0,
+                                                    static_cast<__nv_bfloat16 *>(o), S_T, T, H, d_v, kWaitNs);
     return from_cuda(cudaGetLastError());
 }
 
