@@ -15,7 +15,9 @@ Pins: every function here is checked in ``tests/test_oracle_pins.py`` against
 an explicit d_k x d_k matrix brute force, the linear-attention and
 gated-linear-attention closed forms, separately written KDA and Gated DeltaNet
 recurrences, a hand-derived worked example, and invariants (delta-write,
-state split, linearity, w/v symmetry).
+state split, linearity, w/v symmetry).  The optional input prep and output
+epilogue are pinned in ``tests/test_oracle_fused_pins.py`` (hand-worked
+values, closed forms of sigmoid and SiLU, scale and sign invariances).
 """
 from __future__ import annotations
 
@@ -47,6 +49,11 @@ def open_library(path: str):
     lib.gdn2_oracle_forward.argtypes = [P, P, P, P, P, P, P, P, P, P,
                                         I, I, I, I, I, P, I, I]
     lib.gdn2_oracle_forward.restype = I
+    D = ctypes.c_double
+    lib.gdn2_oracle_forward_ex.argtypes = [P, P, P, P, P, P, P, P, P, P,
+                                           I, I, I, I, I, P, I, I,
+                                           I, D, P, P, D]
+    lib.gdn2_oracle_forward_ex.restype = I
     lib.gdn2_oracle_max_threads.restype = I
     return lib
 
@@ -74,7 +81,9 @@ def _ptr(a):
 
 
 def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
-            want_state: bool = True, want_smax: bool = False, lib=None):
+            want_state: bool = True, want_smax: bool = False, lib=None, *,
+            prep: bool = False, allow_neg_eigval: bool = False, l2_eps: float = 1e-6,
+            gate=None, norm_weight=None, norm_eps: float = 1e-5):
     """Run the recurrence in fp64.
 
     q, k, log_alpha, b : [B, T, H, d_k];  v, w : [B, T, H, d_v] (any float
@@ -83,6 +92,14 @@ def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
     indices, or None for all.  Returns (o, S_T[, smax]) with
     o : [n_heads, T, d_v] and S_T : [n_heads, d_k, d_v] (float64), heads in
     the order requested.
+
+    prep=True takes q, k, b, w as raw: q and k are L2-normalised over d_k
+    (x / sqrt(sum x^2 + l2_eps)), b = sigmoid(b) (2 sigmoid(b) with
+    allow_neg_eigval) and w = sigmoid(w), all in double (burn-gdn2 README,
+    "Architecture" L2-Norm; "Configuration" allow_neg_eigval).  gate
+    [B, T, H, d_v] with norm_weight [d_v] returns the gated RMS norm
+    o / sqrt(mean(o^2) + norm_eps) * norm_weight * silu(gate) per (token, head)
+    instead of o (README "Architecture": Gated RMS Norm <- SiLU Gate).
     """
     q, k, v, la, b, w = (_f32(x) for x in (q, k, v, log_alpha, b, w))
     B, T, H, dk = q.shape
@@ -106,9 +123,21 @@ def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
     o = np.empty((nh, T, dv), dtype=np.float64)
     st = np.empty((nh, dk, dv), dtype=np.float64) if want_state else None
     sm = np.empty((nh,), dtype=np.float64) if want_smax else None
-    rc = (lib or _load()).gdn2_oracle_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w),
-                                     _ptr(s0), _ptr(o), _ptr(st), _ptr(sm),
-                                     B, T, H, dk, dv, _ptr(hl), nh, int(n_threads))
+    g = None
+    wt = None
+    if gate is not None:
+        g = _f32(gate)
+        assert g.shape == (B, T, H, dv), g.shape
+        assert norm_weight is not None, "the epilogue needs norm_weight"
+        if hasattr(norm_weight, "detach"):
+            norm_weight = norm_weight.detach().double().cpu().numpy()
+        wt = np.ascontiguousarray(np.asarray(norm_weight, dtype=np.float64))
+        assert wt.shape == (dv,), wt.shape
+    pflag = (1 | (2 if allow_neg_eigval else 0)) if prep else 0
+    rc = (lib or _load()).gdn2_oracle_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w),
+                                        _ptr(s0), _ptr(o), _ptr(st), _ptr(sm),
+                                        B, T, H, dk, dv, _ptr(hl), nh, int(n_threads),
+                                        pflag, float(l2_eps), _ptr(g), _ptr(wt), float(norm_eps))
     if rc != 0:
         raise ValueError("gdn2 oracle rejected its arguments")
     if want_smax:
@@ -116,15 +145,20 @@ def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
     return o, st
 
 
-def decode_steps(q, k, v, log_alpha, b, w, S0, heads=None, n_threads: int = 0):
+def decode_steps(q, k, v, log_alpha, b, w, S0, heads=None, n_threads: int = 0, *,
+                 prep: bool = False, allow_neg_eigval: bool = False, l2_eps: float = 1e-6,
+                 gate=None, norm_weight=None, norm_eps: float = 1e-5):
     """Token-by-token decode over a step axis.
 
     Inputs are [steps, B, H, d] (one token per step and sequence), S0 is
     [B, H, d_k, d_v].  Returns (o [n_heads, steps, d_v], S [n_heads, d_k, d_v]).
     Decode is the same recurrence run one token at a time, so this is the
-    forward pass with the step axis taken as time.
+    forward pass with the step axis taken as time (prep and epilogue as in
+    ``forward``).
     """
     def tb(x):
         return np.ascontiguousarray(np.swapaxes(_f32(x), 0, 1))
     return forward(tb(q), tb(k), tb(v), tb(log_alpha), tb(b), tb(w), S0=S0,
-                   heads=heads, n_threads=n_threads)
+                   heads=heads, n_threads=n_threads, prep=prep, allow_neg_eigval=allow_neg_eigval,
+                   l2_eps=l2_eps, gate=None if gate is None else tb(gate), norm_weight=norm_weight,
+                   norm_eps=norm_eps)

@@ -37,6 +37,19 @@
  * largest |S_t[i][j]| seen over the run, so state growth is visible.
  *
  * Returns 0 on success, -1 on bad arguments or allocation failure.
+ *
+ * gdn2_oracle_forward_ex adds the two steps around the recurrence that the
+ * README's "Architecture" diagram draws next to it, each optional:
+ *   input prep  (the "L2-Norm" after the projections; "Configuration",
+ *                allow_neg_eigval "b x 2"):
+ *       q = q_raw / sqrt(sum_i q_raw_i^2 + l2_eps), k likewise (over d_k),
+ *       b = sigmoid(b_raw) (times 2 with allow_neg_eigval), w = sigmoid(w_raw);
+ *   output epilogue ("Gated RMS Norm <- SiLU Gate"; "Configuration",
+ *                norm_eps):
+ *       y_j = o_j / sqrt(mean_j o_j^2 + norm_eps) * weight_j * silu(g_j),
+ *       silu(x) = x / (1 + exp(-x)), per (token, head) over d_v.
+ * Readings: the L2 epsilon (not on the pages) is an argument; the RMS norm
+ * is taken per head over d_v with one weight vector [d_v] for all heads.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -45,22 +58,54 @@
 #include <omp.h>
 #endif
 
+typedef struct {
+    int prep;              /* q, k, b, w are raw: L2-normalise q, k; sigmoid b, w */
+    int neg_eigval;        /* with prep: b = 2 sigmoid(b_raw) */
+    double l2_eps;
+    const float *gate;     /* NULL: no epilogue; else [B, T, H, d_v] */
+    const double *weight;  /* [d_v] */
+    double norm_eps;
+} fuse_t;
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* q, k, b (d_k) and w (d_v) of one token as doubles, prepared if asked */
+static void token_inputs(const float *qt, const float *kt, const float *bt, const float *wt,
+                         double *qd, double *kd, double *bd, double *wd, long dk, long dv,
+                         const fuse_t *f)
+{
+    for (long i = 0; i < dk; ++i) { qd[i] = qt[i]; kd[i] = kt[i]; bd[i] = bt[i]; }
+    for (long j = 0; j < dv; ++j) wd[j] = wt[j];
+    if (!f->prep) return;
+    double sq = 0.0, sk = 0.0;
+    for (long i = 0; i < dk; ++i) { sq += qd[i] * qd[i]; sk += kd[i] * kd[i]; }
+    const double nq = sqrt(sq + f->l2_eps), nk = sqrt(sk + f->l2_eps);
+    for (long i = 0; i < dk; ++i) {
+        qd[i] /= nq;
+        kd[i] /= nk;
+        bd[i] = (f->neg_eigval ? 2.0 : 1.0) * sigmoid(bd[i]);
+    }
+    for (long j = 0; j < dv; ++j) wd[j] = sigmoid(wd[j]);
+}
+
 static int run_head(const float *q, const float *k, const float *v,
-                    const float *la, const float *b, const float *w,
+                    const float *la, const float *b, const float *w, const float *g,
                     const double *S0, double *o, double *S_T, double *smax,
-                    long T, long H, long dk, long dv)
+                    long T, long H, long dk, long dv, const fuse_t *f)
 {
     double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
     double *r = (double *)malloc(sizeof(double) * (size_t)dv);
     double *u = (double *)malloc(sizeof(double) * (size_t)dv);
-    if (!S || !r || !u) { free(S); free(r); free(u); return -1; }
+    double *tk = (double *)malloc(sizeof(double) * (size_t)(3 * dk + dv));
+    if (!S || !r || !u || !tk) { free(S); free(r); free(u); free(tk); return -1; }
+    double *qd = tk, *kd = tk + dk, *bd = tk + 2 * dk, *wd = tk + 3 * dk;
     if (S0) memcpy(S, S0, sizeof(double) * (size_t)(dk * dv));
     else    memset(S, 0, sizeof(double) * (size_t)(dk * dv));
     double big = 0.0;
     const long sk = H * dk, sv = H * dv;   /* stride between tokens */
     for (long t = 0; t < T; ++t) {
-        const float *qt = q + t * sk, *kt = k + t * sk, *lat = la + t * sk,
-                    *bt = b + t * sk, *vt = v + t * sv, *wt = w + t * sv;
+        const float *lat = la + t * sk, *vt = v + t * sv;
+        token_inputs(q + t * sk, k + t * sk, b + t * sk, w + t * sv, qd, kd, bd, wd, dk, dv, f);
         /* diag(alpha_t) S_{t-1} */
         for (long i = 0; i < dk; ++i) {
             const double a = exp((double)lat[i]);
@@ -70,14 +115,14 @@ static int run_head(const float *q, const float *k, const float *v,
         /* r = (b_t . k_t)^T (decayed S) */
         for (long j = 0; j < dv; ++j) r[j] = 0.0;
         for (long i = 0; i < dk; ++i) {
-            const double bk = (double)bt[i] * (double)kt[i];
+            const double bk = bd[i] * kd[i];
             const double *row = S + i * dv;
             for (long j = 0; j < dv; ++j) r[j] += bk * row[j];
         }
         /* u = w_t . v_t - r ;  S += k_t u^T */
-        for (long j = 0; j < dv; ++j) u[j] = (double)wt[j] * (double)vt[j] - r[j];
+        for (long j = 0; j < dv; ++j) u[j] = wd[j] * (double)vt[j] - r[j];
         for (long i = 0; i < dk; ++i) {
-            const double ki = (double)kt[i];
+            const double ki = kd[i];
             double *row = S + i * dv;
             for (long j = 0; j < dv; ++j) {
                 row[j] += ki * u[j];
@@ -89,25 +134,38 @@ static int run_head(const float *q, const float *k, const float *v,
         double *ot = o + t * dv;
         for (long j = 0; j < dv; ++j) ot[j] = 0.0;
         for (long i = 0; i < dk; ++i) {
-            const double qi = (double)qt[i];
+            const double qi = qd[i];
             const double *row = S + i * dv;
             for (long j = 0; j < dv; ++j) ot[j] += qi * row[j];
+        }
+        /* y = RMSNorm(o_t) . weight . silu(g_t) */
+        if (g) {
+            const float *gt = g + t * sv;
+            double ms = 0.0;
+            for (long j = 0; j < dv; ++j) ms += ot[j] * ot[j];
+            const double inv = 1.0 / sqrt(ms / (double)dv + f->norm_eps);
+            for (long j = 0; j < dv; ++j) {
+                const double gj = (double)gt[j];
+                ot[j] = ot[j] * inv * f->weight[j] * (gj * sigmoid(gj));
+            }
         }
     }
     if (S_T) memcpy(S_T, S, sizeof(double) * (size_t)(dk * dv));
     if (smax) *smax = big;
-    free(S); free(r); free(u);
+    free(S); free(r); free(u); free(tk);
     return 0;
 }
 
-int gdn2_oracle_forward(const float *q, const float *k, const float *v,
+static int forward_impl(const float *q, const float *k, const float *v,
                         const float *log_alpha, const float *b, const float *w,
                         const double *S0, double *o, double *S_T, double *smax,
                         int B, int T, int H, int d_k, int d_v,
-                        const int *heads, int n_heads, int n_threads)
+                        const int *heads, int n_heads, int n_threads, const fuse_t *f)
 {
     if (!q || !k || !v || !log_alpha || !b || !w || !o) return -1;
     if (B <= 0 || T < 0 || H <= 0 || d_k <= 0 || d_v <= 0) return -1;
+    if (f->gate && !f->weight) return -1;
+    if (f->prep && !(f->l2_eps >= 0.0)) return -1;
     const long nh = heads ? n_heads : (long)B * H;
     if (nh < 0) return -1;
     int bad = 0;
@@ -122,13 +180,41 @@ int gdn2_oracle_forward(const float *q, const float *k, const float *v,
         const long tok0 = bi * (long)T * H + hi;      /* (b, t=0, h) row */
         const long off_k = tok0 * d_k, off_v = tok0 * d_v;
         bad |= run_head(q + off_k, k + off_k, v + off_v, log_alpha + off_k,
-                        b + off_k, w + off_v,
+                        b + off_k, w + off_v, f->gate ? f->gate + off_v : NULL,
                         S0 ? S0 + bh * (long)d_k * d_v : NULL,
                         o + n * (long)T * d_v,
                         S_T ? S_T + n * (long)d_k * d_v : NULL,
-                        smax ? smax + n : NULL, T, H, d_k, d_v) != 0;
+                        smax ? smax + n : NULL, T, H, d_k, d_v, f) != 0;
     }
     return bad ? -1 : 0;
+}
+
+int gdn2_oracle_forward(const float *q, const float *k, const float *v,
+                        const float *log_alpha, const float *b, const float *w,
+                        const double *S0, double *o, double *S_T, double *smax,
+                        int B, int T, int H, int d_k, int d_v,
+                        const int *heads, int n_heads, int n_threads)
+{
+    const fuse_t f = {0, 0, 0.0, NULL, NULL, 0.0};
+    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, d_k, d_v,
+                        heads, n_heads, n_threads, &f);
+}
+
+/* prep: 0 = inputs as given, 1 = raw q, k, b, w (see the header), 3 = raw and
+ * allow_neg_eigval.  gate (nullable) switches the output epilogue on; it needs
+ * weight [d_v]. */
+int gdn2_oracle_forward_ex(const float *q, const float *k, const float *v,
+                           const float *log_alpha, const float *b, const float *w,
+                           const double *S0, double *o, double *S_T, double *smax,
+                           int B, int T, int H, int d_k, int d_v,
+                           const int *heads, int n_heads, int n_threads,
+                           int prep, double l2_eps, const float *gate, const double *weight,
+                           double norm_eps)
+{
+    if (prep != 0 && prep != 1 && prep != 3) return -1;
+    const fuse_t f = {prep & 1, (prep >> 1) & 1, l2_eps, gate, weight, norm_eps};
+    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, d_k, d_v,
+                        heads, n_heads, n_threads, &f);
 }
 
 int gdn2_oracle_max_threads(void)

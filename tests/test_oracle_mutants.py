@@ -3,7 +3,8 @@
 Each case copies ``oracle/gdn2_oracle.c`` to a temporary directory, plants one
 mistake by text substitution (a dropped term, a wrong sign, a swapped
 operand), compiles it with gcc and checks that the brute-force / worked-example
-pins reject it.  Mistakes are planted only in these CPU copies.
+pins reject it (the input-prep and epilogue mistakes against the fused pins).
+Mistakes are planted only in these CPU copies.
 """
 import json
 import os
@@ -17,18 +18,28 @@ from test_oracle_pins import HERE, brute_force_head, head, rand_inputs, rel_err
 
 MUTANTS = {
     "write_sign": ("row[j] += ki * u[j];", "row[j] -= ki * u[j];"),
-    "erase_sign": ("u[j] = (double)wt[j] * (double)vt[j] - r[j];",
-                   "u[j] = (double)wt[j] * (double)vt[j] + r[j];"),
-    "erase_gate_dropped": ("const double bk = (double)bt[i] * (double)kt[i];",
-                           "const double bk = (double)kt[i];"),
+    "erase_sign": ("u[j] = wd[j] * (double)vt[j] - r[j];", "u[j] = wd[j] * (double)vt[j] + r[j];"),
+    "erase_gate_dropped": ("const double bk = bd[i] * kd[i];", "const double bk = kd[i];"),
     "decay_dropped": ("const double a = exp((double)lat[i]);", "const double a = 1.0;"),
     "decay_inverted": ("const double a = exp((double)lat[i]);",
                        "const double a = exp(-(double)lat[i]);"),
-    "write_gate_dropped": ("u[j] = (double)wt[j] * (double)vt[j] - r[j];",
-                           "u[j] = (double)vt[j] - r[j];"),
-    "query_is_key": ("const double qi = (double)qt[i];", "const double qi = (double)kt[i];"),
-    "erase_on_query": ("const double bk = (double)bt[i] * (double)kt[i];",
-                       "const double bk = (double)bt[i] * (double)qt[i];"),
+    "write_gate_dropped": ("u[j] = wd[j] * (double)vt[j] - r[j];", "u[j] = (double)vt[j] - r[j];"),
+    "query_is_key": ("const double qi = qd[i];", "const double qi = kd[i];"),
+    "erase_on_query": ("const double bk = bd[i] * kd[i];", "const double bk = bd[i] * qd[i];"),
+}
+
+# mistakes in the optional input prep and output epilogue
+FUSED_MUTANTS = {
+    "l2_without_sqrt": ("const double nq = sqrt(sq + f->l2_eps), nk = sqrt(sk + f->l2_eps);",
+                        "const double nq = sq + f->l2_eps, nk = sk + f->l2_eps;"),
+    "l2_key_skipped": ("kd[i] /= nk;", "kd[i] /= 1.0;"),
+    "logistic_sign": ("static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }",
+                      "static double sigmoid(double x) { return 1.0 / (1.0 + exp(x)); }"),
+    "neg_eigval_ignored": ("(f->neg_eigval ? 2.0 : 1.0)", "(1.0)"),
+    "write_gate_left_raw": ("for (long j = 0; j < dv; ++j) wd[j] = sigmoid(wd[j]);", ""),
+    "rms_sum_not_mean": ("sqrt(ms / (double)dv + f->norm_eps)", "sqrt(ms + f->norm_eps)"),
+    "silu_is_sigmoid": ("(gj * sigmoid(gj))", "sigmoid(gj)"),
+    "norm_weight_dropped": ("ot[j] * inv * f->weight[j] * ", "ot[j] * inv * "),
 }
 
 
@@ -52,6 +63,27 @@ def _pins_pass(lib) -> bool:
                 and np.allclose(ST[0], g["expected"]["S_T"], atol=1e-7))
 
 
+def _fused_pins_pass(lib) -> bool:
+    import test_oracle_fused_pins as fp
+
+    class _Mod:   # the oracle module's forward, bound to this library
+        @staticmethod
+        def forward(*a, **kw):
+            return oracle.forward(*a, lib=lib, **kw)
+
+    checks = [lambda: fp.test_input_prep_worked_example(_Mod, "plain"),
+              lambda: fp.test_input_prep_worked_example(_Mod, "neg_eigval"),
+              lambda: fp.test_output_epilogue_worked_example(_Mod),
+              lambda: fp.test_prep_is_scale_invariant_in_q_and_k(_Mod),
+              lambda: fp.test_epilogue_constant_row_and_zero_gate(_Mod)]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
 def _compile(src_text: str, tmp_path, name: str):
     c = tmp_path / f"{name}.c"
     so = tmp_path / f"{name}.so"
@@ -67,7 +99,8 @@ def oracle_source():
 
 
 def test_unmutated_copy_passes(oracle_source, tmp_path):
-    assert _pins_pass(_compile(oracle_source, tmp_path, "clean"))
+    lib = _compile(oracle_source, tmp_path, "clean")
+    assert _pins_pass(lib) and _fused_pins_pass(lib)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -76,3 +109,11 @@ def test_mutant_is_caught(oracle_source, tmp_path, name):
     assert oracle_source.count(old) == 1, f"mutation site for {name} not found"
     lib = _compile(oracle_source.replace(old, new), tmp_path, name)
     assert not _pins_pass(lib), f"pins did not catch mutant {name}"
+
+
+@pytest.mark.parametrize("name", sorted(FUSED_MUTANTS))
+def test_fused_mutant_is_caught(oracle_source, tmp_path, name):
+    old, new = FUSED_MUTANTS[name]
+    assert oracle_source.count(old) == 1, f"mutation site for {name} not found"
+    lib = _compile(oracle_source.replace(old, new), tmp_path, name)
+    assert not _fused_pins_pass(lib), f"fused pins did not catch mutant {name}"
