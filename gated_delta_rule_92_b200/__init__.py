@@ -26,8 +26,11 @@ IO_BF16 = 1
 STATUS_NAMES = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
                 3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT"}
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_decode_step",
+            "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex",
             "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_status_string",
             "gdn2_version")
+FUSE_INPUT_PREP = 1    # q, k, b, w are raw: L2-normalise q, k over d_k; b, w = sigmoid
+FUSE_NEG_EIGVAL = 2    # with FUSE_INPUT_PREP: b = 2 sigmoid(b)
 
 _lib = None
 
@@ -53,6 +56,12 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).restype = I
         L.gdn2_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.gdn2_decode_step.restype = I
+        F = ctypes.c_float
+        fuse_args = [I, F, P, P, F]
+        L.gdn2_chunk_fwd_ex.argtypes = chunk_args[:-1] + fuse_args + [P]
+        L.gdn2_chunk_fwd_ex.restype = I
+        L.gdn2_decode_step_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I] + fuse_args + [P]
+        L.gdn2_decode_step_ex.restype = I
         L.gdn2_device_status.argtypes = [P]
         L.gdn2_device_status.restype = I
         L.gdn2_selftest_wait_timeout.argtypes = [I, P]
@@ -105,7 +114,25 @@ def _check_state(S, shape, device):
         raise ValueError(f"state must be contiguous float32 {tuple(shape)} on {device}")
 
 
-def _chunk(fn_name, q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state):
+def _fuse_args(q, prep, allow_neg_eigval, l2_eps, gate, norm_weight, norm_eps, gate_shape):
+    """The fusion arguments of the _ex calls, checked and marshalled."""
+    flags = (FUSE_INPUT_PREP if prep else 0) | (FUSE_NEG_EIGVAL if (prep and allow_neg_eigval) else 0)
+    if allow_neg_eigval and not prep:
+        raise ValueError("allow_neg_eigval applies to the fused input prep (prep=True)")
+    if gate is not None:
+        _check_tokens((gate,), q.dtype, q.device)
+        if tuple(gate.shape) != tuple(gate_shape):
+            raise ValueError(f"gate must be {tuple(gate_shape)}")
+        if norm_weight is None or norm_weight.dtype != torch.float32 or not norm_weight.is_contiguous() \
+                or tuple(norm_weight.shape) != (gate_shape[-1],) or norm_weight.device != q.device:
+            raise ValueError("norm_weight must be a contiguous float32 [d_v] tensor on the device")
+    elif norm_weight is not None:
+        raise ValueError("norm_weight is only used with gate")
+    return [int(flags), ctypes.c_float(float(l2_eps)), _ptr(gate),
+            _ptr(norm_weight) if gate is not None else None, ctypes.c_float(float(norm_eps))]
+
+
+def _chunk(fn_name, q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state, fuse=None):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -123,9 +150,11 @@ def _chunk(fn_name, q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_st
     _check_tokens((o,), q.dtype, dev)
     _check_state(S_T, (B, H, dk, dv), dev)
     with torch.cuda.device(dev):
-        st = getattr(lib(), fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
-                                     _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk),
-                                     _io(q.dtype), _stream(stream))
+        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk), _io(q.dtype)]
+        if fuse is not None:
+            args += fuse(q, (B, T, H, dv))
+        st = getattr(lib(), fn_name)(*args, _stream(stream))
     if st != 0:
         raise Gdn2Error(st, fn_name)
     return o, S_T
@@ -137,6 +166,18 @@ def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int
     return _chunk("gdn2_chunk_fwd", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state)
 
 
+def chunk_fwd_ex(q, k, v, log_alpha, b, w, S0=None, *, prep: bool = False, allow_neg_eigval: bool = False,
+                 l2_eps: float = 1e-6, gate=None, norm_weight=None, norm_eps: float = 1e-5,
+                 o=None, S_T=None, chunk: int = 64, stream=None, want_state: bool = True):
+    """Chunk forward with the fused input prep (prep=True: raw q, k, b, w) and,
+    with gate [B,T,H,d_v] and norm_weight [d_v] fp32, the gated RMS-norm output
+    epilogue.  Returns (o or y, S_T)."""
+    fuse = lambda q_, shape: _fuse_args(q_, prep, allow_neg_eigval, l2_eps, gate, norm_weight,
+                                        norm_eps, shape)
+    return _chunk("gdn2_chunk_fwd_ex", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream,
+                  want_state, fuse)
+
+
 def chunk_fwd_cuda_core(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int = 64,
                         stream=None, want_state: bool = True):
     """The same forward on the CUDA-core (fp32 FFMA) chunk kernel."""
@@ -144,8 +185,7 @@ def chunk_fwd_cuda_core(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, 
                   want_state)
 
 
-def decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
-    """One token per sequence: S [B,H,d_k,d_v] fp32 is updated in place; returns o [B,H,d_v]."""
+def _decode(fn_name, q, k, v, log_alpha, b, w, S, o, stream, fuse=None):
     B, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -154,11 +194,29 @@ def decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
     if o is None:
         o = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
     with torch.cuda.device(dev):
-        st = lib().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
-                                    _ptr(S), _ptr(o), B, H, dk, dv, _io(q.dtype), _stream(stream))
+        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                _ptr(S), _ptr(o), B, H, dk, dv, _io(q.dtype)]
+        if fuse is not None:
+            args += fuse(q, (B, H, dv))
+        st = getattr(lib(), fn_name)(*args, _stream(stream))
     if st != 0:
-        raise Gdn2Error(st, "gdn2_decode_step")
+        raise Gdn2Error(st, fn_name)
     return o
+
+
+def decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
+    """One token per sequence: S [B,H,d_k,d_v] fp32 is updated in place; returns o [B,H,d_v]."""
+    return _decode("gdn2_decode_step", q, k, v, log_alpha, b, w, S, o, stream)
+
+
+def decode_step_ex(q, k, v, log_alpha, b, w, S, *, prep: bool = False, allow_neg_eigval: bool = False,
+                   l2_eps: float = 1e-6, gate=None, norm_weight=None, norm_eps: float = 1e-5,
+                   o=None, stream=None):
+    """Decode step with the fused input prep and (gate [B,H,d_v], norm_weight [d_v])
+    the gated RMS-norm output epilogue."""
+    fuse = lambda q_, shape: _fuse_args(q_, prep, allow_neg_eigval, l2_eps, gate, norm_weight,
+                                        norm_eps, shape)
+    return _decode("gdn2_decode_step_ex", q, k, v, log_alpha, b, w, S, o, stream, fuse)
 
 
 def device_status(stream=None) -> int:

@@ -44,12 +44,17 @@ struct FfmaCfg {
     static constexpr size_t BYTES = sizeof(float) * FLOATS;
 };
 
-template <typename IO, int DK>
+// FUSED with fz.prep reads raw q, k, b, w: rows of q and k are L2-normalised
+// over d_k (x / sqrt(sum x^2 + l2_eps)), b = sigmoid(b) (x2 with neg_eigval),
+// w = sigmoid(w).  The output epilogue of this path runs as a separate pass.
+template <typename IO, int DK, bool FUSED = false>
 __global__ void __launch_bounds__(256, 1)
 chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                       const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ wg,
                       const float *__restrict__ S0, IO *__restrict__ o, float *__restrict__ S_T,
-                      int T, int H, int d_v) {
+                      int T, int H, int d_v, const FuseArgs fz = {}) {
+    const bool prep = FUSED && fz.prep;
+    const float bscale = (FUSED && fz.neg_eigval) ? 2.f : 1.f;
     using Cfg = FfmaCfg<DK>;
     constexpr int C = Cfg::C, NV = Cfg::NV, LK = Cfg::LK, LC = Cfg::LC;
     extern __shared__ float sm[];
@@ -81,15 +86,37 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
             const bool in = r < rows;
             sQ[r * LK + c] = in ? ld_io(q + g) : 0.f;
             sK[r * LK + c] = in ? ld_io(k + g) : 0.f;
-            sE[r * LK + c] = in ? ld_io(bg + g) : 0.f;
+            sE[r * LK + c] = in ? (prep ? bscale * sigmoid_f32(ld_io(bg + g)) : ld_io(bg + g)) : 0.f;
             sG[r * LK + c] = in ? ld_io(la + g) : 0.f;
         }
         for (int idx = tid; idx < C * NV; idx += 256) {
             const int r = idx / NV, j = idx % NV;
             const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
-            sWV[r * LC + j] = (r < rows) ? ld_io(wg + g) * ld_io(v + g) : 0.f;
+            const float wv = (r < rows) ? ld_io(wg + g) : 0.f;
+            sWV[r * LC + j] = (r < rows) ? (prep ? sigmoid_f32(wv) : wv) * ld_io(v + g) : 0.f;
         }
         __syncthreads();
+        if (prep) {   // L2-normalise each row of q and k: warp w takes rows w, w + 8, ...
+            const int wp = tid >> 5, l = tid & 31;
+            for (int r = wp; r < C; r += 8) {
+                float sq = 0.f, sk = 0.f;
+                for (int c = l; c < DK; c += 32) {
+                    sq = fmaf(sQ[r * LK + c], sQ[r * LK + c], sq);
+                    sk = fmaf(sK[r * LK + c], sK[r * LK + c], sk);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                }
+                const float iq = l2_inv(sq, fz.l2_eps), ik = l2_inv(sk, fz.l2_eps);
+                for (int c = l; c < DK; c += 32) {
+                    sQ[r * LK + c] *= iq;
+                    sK[r * LK + c] *= ik;
+                }
+            }
+            __syncthreads();
+        }
         // ---- cumulative log-decay per key channel and the scaled operands
         if (tid < DK) {
             const int c = tid;

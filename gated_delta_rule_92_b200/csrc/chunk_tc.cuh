@@ -36,6 +36,7 @@
 // tcgen05.commit; hand-offs go through mbarriers.  Every wait is bounded; a
 // timeout records an error, drains this CTA's MMAs and returns.
 #pragma once
+#include "decode.cuh"
 #include "gdn2_device.cuh"
 
 namespace gdn2 {
@@ -239,9 +240,12 @@ struct PrepLA {
 // it (exchanged through `carry` and named barrier `bar` over the 128
 // threads).  A half-warp covers 16 consecutive quads = one 128-byte swizzled
 // row, so the 8-byte shared accesses are conflict-free.
-template <int DK>
+// With fz.prep (FUSED only) q, k, b arrive raw: each row of q and k is scaled
+// by 1 / sqrt(sum^2 + l2_eps) (the sums over d_k reduced across the NP lanes
+// that share the row) and b becomes sigmoid(b) (x2 with neg_eigval).
+template <int DK, bool FUSED = false>
 __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLA<DK> &law,
-                                           float *gc, float *carry, int g, int bar) {
+                                           float *gc, float *carry, int g, int bar, const FuseArgs &fz = {}) {
     constexpr int NP = PrepLA<DK>::NP, NB = PrepLA<DK>::NB, R = PrepLA<DK>::R;
     static_assert(NB * R == 64 && NB <= 8, "prep split");
     const int p = g % NP, hb = g / NP;
@@ -288,6 +292,26 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
         }
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
+            float rq = 1.f, rk = 1.f, bs = 1.f;
+            if constexpr (FUSED) {
+                if (fz.prep) {
+                    float sq = 0.f, sk = 0.f;
+                    const uint32_t qa[2] = {qw[j].x, qw[j].y}, ka[2] = {kw[j].x, kw[j].y};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        sq += bf16_lo(qa[h]) * bf16_lo(qa[h]) + bf16_hi(qa[h]) * bf16_hi(qa[h]);
+                        sk += bf16_lo(ka[h]) * bf16_lo(ka[h]) + bf16_hi(ka[h]) * bf16_hi(ka[h]);
+                    }
+#pragma unroll
+                    for (int off = NP / 2; off > 0; off >>= 1) {
+                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    }
+                    rq = l2_inv(sq, fz.l2_eps);
+                    rk = l2_inv(sk, fz.l2_eps);
+                    bs = fz.neg_eigval ? 2.f : 1.f;
+                }
+            }
             const uint2 la2 = law.v[i0 + j];
             sum[0] = fmaf(bf16_lo(la2.x), kLog2e, sum[0]);
             sum[1] = fmaf(bf16_hi(la2.x), kLog2e, sum[1]);
@@ -299,9 +323,21 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
             for (int h = 0; h < 2; ++h) {
                 const float ga0 = ex2(sum[2 * h]), ga1 = ex2(sum[2 * h + 1]);
                 const float iv0 = ex2(-sum[2 * h]), iv1 = ex2(-sum[2 * h + 1]);
-                const float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
-                oq[h] = pack_bf16x2(bf16_lo(qv[h]) * ga0, bf16_hi(qv[h]) * ga1);
-                oe[h] = pack_bf16x2(bf16_lo(bv[h]) * k0 * ga0, bf16_hi(bv[h]) * k1 * ga1);
+                float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
+                float b0 = bf16_lo(bv[h]), b1 = bf16_hi(bv[h]);
+                float q0 = bf16_lo(qv[h]), q1 = bf16_hi(qv[h]);
+                if constexpr (FUSED) {
+                    if (fz.prep) {
+                        k0 *= rk;
+                        k1 *= rk;
+                        q0 *= rq;
+                        q1 *= rq;
+                        b0 = bs * sigmoid_tanh(b0);
+                        b1 = bs * sigmoid_tanh(b1);
+                    }
+                }
+                oq[h] = pack_bf16x2(q0 * ga0, q1 * ga1);
+                oe[h] = pack_bf16x2(b0 * k0 * ga0, b1 * k1 * ga1);
                 ok[h] = pack_bf16x2(k0 * iv0, k1 * iv1);
             }
             *reinterpret_cast<uint2 *>(q_t + o[j]) = make_uint2(oq[0], oq[1]);
@@ -316,13 +352,16 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
     fence_proxy_async_smem();
 }
 
-template <int DK, int NV>
+// FUSED adds the input prep (fz.prep: raw q, k, b, w) and, when fz.gate is
+// set, the gated RMS norm of each output row before it is stored; the
+// launcher sets fz.gate only when d_v == NV, so one CTA holds the whole row.
+template <int DK, int NV, bool FUSED = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16 *__restrict__ la,
                     const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T,
-                    int T, int H, int d_v, unsigned long long wait_ns) {
+                    int T, int H, int d_v, unsigned long long wait_ns, const FuseArgs fz = {}) {
     using Cfg = TcCfg<DK, NV>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -456,7 +495,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4);
+            else if (grp_b) prep_chunk<DK, FUSED>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, fz);
         }
         for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
@@ -490,7 +529,18 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
                     ld_shared_v4(sb + Cfg::OFF_V + off, a0, a1, a2, a3);
                     ld_shared_v4(sb + Cfg::OFF_W + off, b0, b1, b2, b3);
-                    const uint4 r4 = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));
+                    uint4 r4;
+                    if (FUSED && fz.prep) {   // w arrives raw: sigmoid(w) . v, rounded once
+                        const uint32_t vv[4] = {a0, a1, a2, a3}, ww[4] = {b0, b1, b2, b3};
+                        uint32_t rr[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            rr[e] = pack_bf16x2(sigmoid_tanh(bf16_lo(ww[e])) * bf16_lo(vv[e]),
+                                                sigmoid_tanh(bf16_hi(ww[e])) * bf16_hi(vv[e]));
+                        r4 = make_uint4(rr[0], rr[1], rr[2], rr[3]);
+                    } else {
+                        r4 = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));
+                    }
                     st_shared_v4(sb + Cfg::OFF_V + off, r4.x, r4.y, r4.z, r4.w);
                 }
             }
@@ -548,8 +598,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = ok_b && mbar_wait(&k_full[s3n], static_cast<uint32_t>(((m + 1) / 3) & 1), wait_ns);
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
-                    prep_chunk<DK>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
-                                   gC + ((m + 1) % 3) * 128, carry, t - 128, 4);
+                    prep_chunk<DK, FUSED>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
+                                          gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz);
             }
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
@@ -774,9 +824,52 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if ((warp & 3) < 2) {
                 const int r = t;   // output row r (TMEM lanes 0-63); rows past T are padding
                 const bool valid = n * 64 + r < T;
-                __nv_bfloat16 *orow = o + (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0;
+                const long orow_off = (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0;
+                __nv_bfloat16 *orow = o + orow_off;
+                bool plain = true;
+                if constexpr (FUSED) {
+                    if (fz.gate != nullptr) {   // y = o / rms(o) . weight . silu(g)  (d_v == NV)
+                        plain = false;
+                        float ss = 0.f;
 #pragma unroll 1
-                for (int jc = 0; jc < NV / 32; ++jc) {
+                        for (int jc = 0; jc < NV / 32; ++jc) {
+                            float x[32];
+                            tmem_ld32(t_X + lane_q + jc * 32, x);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
+                        }
+                        const float inv = rsqrtf(ss / (float)NV + fz.norm_eps);
+                        const __nv_bfloat16 *grow = static_cast<const __nv_bfloat16 *>(fz.gate) + orow_off;
+#pragma unroll 1
+                        for (int jc = 0; jc < NV / 32; ++jc) {
+                            float x[32];
+                            tmem_ld32(t_X + lane_q + jc * 32, x);
+                            if (valid) {
+                                const uint4 *gsrc = reinterpret_cast<const uint4 *>(grow + jc * 32);
+                                const float4 *wsrc = reinterpret_cast<const float4 *>(fz.norm_weight + j0 + jc * 32);
+                                uint4 *dst = reinterpret_cast<uint4 *>(orow + jc * 32);
+#pragma unroll
+                                for (int q4 = 0; q4 < 4; ++q4) {
+                                    const uint4 gv = __ldg(gsrc + q4);
+                                    const float4 w0 = __ldg(wsrc + 2 * q4), w1 = __ldg(wsrc + 2 * q4 + 1);
+                                    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                                    const float wt[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                                    uint32_t pk[4];
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const float g0 = bf16_lo(gw[e]), g1 = bf16_hi(gw[e]);
+                                        pk[e] = pack_bf16x2(x[8 * q4 + 2 * e] * inv * wt[2 * e] * g0 * sigmoid_tanh(g0),
+                                                            x[8 * q4 + 2 * e + 1] * inv * wt[2 * e + 1] * g1 *
+                                                                sigmoid_tanh(g1));
+                                    }
+                                    dst[q4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                                }
+                            }
+                        }
+                    }
+                }
+#pragma unroll 1
+                for (int jc = 0; jc < NV / 32 && plain; ++jc) {
                     float x[32];
                     tmem_ld32(t_X + lane_q + jc * 32, x);
                     if (valid) {

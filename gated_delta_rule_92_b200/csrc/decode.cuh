@@ -17,6 +17,8 @@
 // block keeps 32-64 KB of HBM reads in flight.  Column sums over d_k are
 // reduced through shared memory.
 #pragma once
+#include <cooperative_groups.h>
+
 #include "gdn2_device.cuh"
 
 namespace gdn2 {
@@ -44,11 +46,32 @@ __device__ __forceinline__ void st_io4<__nv_bfloat16>(__nv_bfloat16 *p, float a,
     *reinterpret_cast<uint2 *>(p) = u;
 }
 
-template <typename IO, int DK, int NVD>
+// Optional fusion around the step (burn-gdn2 README, "Architecture": the
+// L2-Norm before the mixer and the SiLU-gated RMS norm after it;
+// "Configuration": allow_neg_eigval, norm_eps).
+struct FuseArgs {
+    int prep;                  // q, k, b, w raw: L2-normalise q, k; b, w = sigmoid
+    int neg_eigval;            // with prep: b = 2 sigmoid(b_raw)
+    float l2_eps;
+    const void *gate;          // non-null: y = o / sqrt(mean(o^2) + eps) * weight * silu(gate)
+    const float *norm_weight;  // [d_v]
+    float norm_eps;
+};
+
+template <typename IO>
+__device__ __forceinline__ float sigmoid_io(float x) {
+    if constexpr (sizeof(IO) == 4) return sigmoid_f32(x);
+    else return sigmoid_tanh(x);
+}
+
+// With FUSED, the d_v / NVD blocks of one (b, h) form a thread-block cluster
+// along y when the epilogue is on and d_v > NVD, so the RMS over d_v can add
+// the blocks' partial sums through distributed shared memory.
+template <typename IO, int DK, int NVD, bool FUSED = false>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                    const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ wg,
-                   float *__restrict__ S, IO *__restrict__ o, int d_v) {
+                   float *__restrict__ S, IO *__restrict__ o, int d_v, FuseArgs fz = {}) {
     constexpr int TPR = NVD / 4;   // threads across one row of the slice
     constexpr int RG = 256 / TPR;  // thread rows
     constexpr int RPT = DK / RG;   // state rows per thread
@@ -59,6 +82,8 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     __shared__ __align__(16) float s_red_r[RG][NVD];
     __shared__ __align__(16) float s_red_p[RG][NVD];
     __shared__ float s_qk[8];
+    __shared__ float s_nrm[2][8];      // fused prep: per-warp sums of q^2, k^2
+    __shared__ float s_ss[8];          // fused epilogue: sum of o^2 per block of the cluster
 
     const int tid = threadIdx.x;
     const int cg = tid % TPR;        // float4 column group
@@ -77,19 +102,46 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     // per-row and per-column coefficients
     const IO *qh = q + bh * DK, *kh = k + bh * DK, *lah = la + bh * DK, *bh_ = bg + bh * DK;
     float qk = 0.f;
+    float kv = 0.f, qv = 0.f, bv = 0.f;
+    if (tid < DK) {
+        kv = ld_io(kh + tid);
+        qv = ld_io(qh + tid);
+        bv = ld_io(bh_ + tid);
+    }
+    if constexpr (FUSED) {
+        if (fz.prep) {   // q / |q|, k / |k| over d_k (block reduction), sigmoid gates
+            float sq = qv * qv, sk = kv * kv;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            }
+            if ((tid & 31) == 0 && tid < DK) { s_nrm[0][tid >> 5] = sq; s_nrm[1][tid >> 5] = sk; }
+            __syncthreads();
+            sq = 0.f;
+            sk = 0.f;
+#pragma unroll
+            for (int wi = 0; wi < DK / 32; ++wi) { sq += s_nrm[0][wi]; sk += s_nrm[1][wi]; }
+            qv *= l2_inv(sq, fz.l2_eps);
+            kv *= l2_inv(sk, fz.l2_eps);
+            bv = (fz.neg_eigval ? 2.f : 1.f) * sigmoid_io<IO>(bv);
+        }
+    }
     if (tid < DK) {
         const float a = __expf(ld_io(lah + tid));
-        const float kv = ld_io(kh + tid);
-        const float qv = ld_io(qh + tid);
         s_alpha[tid] = a;
-        s_erase[tid] = ld_io(bh_ + tid) * kv * a;
+        s_erase[tid] = bv * kv * a;
         s_qa[tid] = qv * a;
         s_k[tid] = kv;
         qk = qv * kv;
     }
     if (tid < NVD) {
         const long vo = bh * (long)d_v + j0 + tid;
-        s_wv[tid] = ld_io(wg + vo) * ld_io(v + vo);
+        float wv = ld_io(wg + vo);
+        if constexpr (FUSED) {
+            if (fz.prep) wv = sigmoid_io<IO>(wv);
+        }
+        s_wv[tid] = wv * ld_io(v + vo);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
@@ -118,6 +170,7 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     const float4 wv = *reinterpret_cast<const float4 *>(&s_wv[cg * 4]);
     const float4 u = make_float4(wv.x - rt.x, wv.y - rt.y, wv.z - rt.z, wv.w - rt.w);
 
+    float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
     if (rg == 0) {
 #pragma unroll
         for (int g = 0; g < RG; ++g) {
@@ -127,9 +180,43 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         float qkt = 0.f;
 #pragma unroll
         for (int wi = 0; wi < (DK + 31) / 32; ++wi) qkt += s_qk[wi];
-        st_io4<IO>(o + bh * (long)d_v + j0 + cg * 4, pt.x + qkt * u.x, pt.y + qkt * u.y, pt.z + qkt * u.z,
-                   pt.w + qkt * u.w);
+        ov = make_float4(pt.x + qkt * u.x, pt.y + qkt * u.y, pt.z + qkt * u.z, pt.w + qkt * u.w);
     }
+    bool plain_store = true;
+    if constexpr (FUSED) {
+        if (fz.gate != nullptr) {   // gated RMS norm over the whole d_v row
+            plain_store = false;
+            float ss = ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w;   // zero for rg != 0
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            const int nblk = d_v / NVD;   // cluster size along y (1: no cluster)
+            if (nblk == 1) {
+                if (tid == 0) s_ss[0] = ss;
+                __syncthreads();
+            } else {
+                // every block of the cluster has started before any writes into a
+                // peer's shared memory; the second sync publishes the sums
+                cooperative_groups::cluster_group cl = cooperative_groups::this_cluster();
+                cl.sync();
+                if (tid == 0)
+                    for (int r = 0; r < nblk; ++r) cl.map_shared_rank(s_ss, r)[blockIdx.y] = ss;
+                cl.sync();
+            }
+            if (rg == 0) {
+                float tot = 0.f;
+                for (int r = 0; r < nblk; ++r) tot += s_ss[r];
+                const float inv = rsqrtf(tot / (float)d_v + fz.norm_eps);
+                const long go = bh * (long)d_v + j0 + cg * 4;
+                const IO *gp = static_cast<const IO *>(fz.gate) + go;
+                const float4 wt = __ldg(reinterpret_cast<const float4 *>(fz.norm_weight + j0 + cg * 4));
+                const float g0 = ld_io(gp), g1 = ld_io(gp + 1), g2 = ld_io(gp + 2), g3 = ld_io(gp + 3);
+                st_io4<IO>(o + go, ov.x * inv * wt.x * g0 * sigmoid_io<IO>(g0),
+                           ov.y * inv * wt.y * g1 * sigmoid_io<IO>(g1), ov.z * inv * wt.z * g2 * sigmoid_io<IO>(g2),
+                           ov.w * inv * wt.w * g3 * sigmoid_io<IO>(g3));
+            }
+        }
+    }
+    if (plain_store && rg == 0) st_io4<IO>(o + bh * (long)d_v + j0 + cg * 4, ov.x, ov.y, ov.z, ov.w);
 
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {

@@ -262,6 +262,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&p);
 }
+// 1 / sqrt(s + eps) for an L2 norm; a zero vector with eps = 0 gives 0 (the
+// vector stays zero instead of becoming 0 / 0).
+__device__ __forceinline__ float l2_inv(float s, float eps) {
+    const float d = s + eps;
+    return d > 0.f ? rsqrtf(d) : 0.f;
+}
+// Logistic function 1 / (1 + e^-x) with an IEEE division (fp32-I/O paths).
+__device__ __forceinline__ float sigmoid_f32(float x) { return 1.f / (1.f + __expf(-x)); }
+// Logistic function as 0.5 + 0.5 tanh(x / 2) with the one-instruction tanh
+// approximation (relative error about 2^-11; for paths whose result is bf16).
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 

@@ -14,6 +14,7 @@
 #include "chunk_ffma.cuh"
 #include "chunk_tc.cuh"
 #include "decode.cuh"
+#include "epilogue.cuh"
 #include "gdn2_device.cuh"
 
 namespace gdn2 {
@@ -71,49 +72,120 @@ bool make_token_map(CUtensorMap *m, const void *base, int B, int T, int H, int d
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <typename IO>
+gdn2_status_t launch_rmsnorm(void *o, const void *g, const float *weight, long rows, int d_v, float eps,
+                             cudaStream_t st) {
+    if (rows == 0) return GDN2_OK;
+    gated_rmsnorm_kernel<IO><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        static_cast<IO *>(o), static_cast<const IO *>(g), weight, rows, d_v, eps);
+    return from_cuda(cudaGetLastError());
+}
+
 template <int DK, int NV>
 gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void *la, const void *b, const void *w,
-                        const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st) {
+                        const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st,
+                        const FuseArgs *fz = nullptr) {
     using Cfg = TcCfg<DK, NV>;
     CUtensorMap tq, tk, tb, tv, tw;
     if (!make_token_map(&tq, q, B, T, H, DK) || !make_token_map(&tk, k, B, T, H, DK) ||
         !make_token_map(&tb, b, B, T, H, DK) || !make_token_map(&tv, v, B, T, H, d_v) ||
         !make_token_map(&tw, w, B, T, H, d_v))
         return GDN2_ERR_CUDA;
-    auto kern = chunk_fwd_tc_kernel<DK, NV>;
+    dim3 grid(d_v / NV, H, B);
+    const __nv_bfloat16 *lap = static_cast<const __nv_bfloat16 *>(la);
+    __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(o);
+    if (fz == nullptr) {
+        auto kern = chunk_fwd_tc_kernel<DK, NV>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
+        if (e != cudaSuccess) return GDN2_ERR_CUDA;
+        kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, lap, S0, op, S_T, T, H, d_v, kWaitNs,
+                                                        FuseArgs{});
+        return from_cuda(cudaGetLastError());
+    }
+    // the in-kernel epilogue needs the whole d_v row in one CTA; otherwise one
+    // more pass normalises o in place
+    FuseArgs kf = *fz;
+    if (d_v != NV) kf.gate = nullptr;
+    auto kern = chunk_fwd_tc_kernel<DK, NV, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    dim3 grid(d_v / NV, H, B);
-    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, static_cast<const __nv_bfloat16 *>(la), S0,
-                                                    static_cast<__nv_bfloat16 *>(o), S_T, T, H, d_v, kWaitNs);
-    return from_cuda(cudaGetLastError());
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, lap, S0, op, S_T, T, H, d_v, kWaitNs, kf);
+    gdn2_status_t s = from_cuda(cudaGetLastError());
+    if (s != GDN2_OK || fz->gate == nullptr || kf.gate != nullptr) return s;
+    return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, (long)B * T * H, d_v, fz->norm_eps, st);
 }
 
 template <typename IO, int DK>
 gdn2_status_t launch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
                           const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_v,
-                          cudaStream_t st) {
+                          cudaStream_t st, const FuseArgs *fz = nullptr) {
     using Cfg = FfmaCfg<DK>;
-    auto kern = chunk_fwd_ffma_kernel<IO, DK>;
+    dim3 grid(d_v / Cfg::NV, H, B);
+    const IO *qp = static_cast<const IO *>(q), *kp = static_cast<const IO *>(k), *vp = static_cast<const IO *>(v);
+    const IO *lp = static_cast<const IO *>(la), *bp = static_cast<const IO *>(b), *wp = static_cast<const IO *>(w);
+    IO *op = static_cast<IO *>(o);
+    if (fz == nullptr) {
+        auto kern = chunk_fwd_ffma_kernel<IO, DK>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
+        if (e != cudaSuccess) return GDN2_ERR_CUDA;
+        kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, T, H, d_v, FuseArgs{});
+        return from_cuda(cudaGetLastError());
+    }
+    auto kern = chunk_fwd_ffma_kernel<IO, DK, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    dim3 grid(d_v / Cfg::NV, H, B);
-    kern<<<grid, 256, Cfg::BYTES, st>>>(static_cast<const IO *>(q), static_cast<const IO *>(k),
-                                        static_cast<const IO *>(v), static_cast<const IO *>(la),
-                                        static_cast<const IO *>(b), static_cast<const IO *>(w), S0,
-                                        static_cast<IO *>(o), S_T, T, H, d_v);
-    return from_cuda(cudaGetLastError());
+    kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, T, H, d_v, *fz);
+    gdn2_status_t s = from_cuda(cudaGetLastError());
+    if (s != GDN2_OK || fz->gate == nullptr) return s;
+    return launch_rmsnorm<IO>(o, fz->gate, fz->norm_weight, (long)B * T * H, d_v, fz->norm_eps, st);
 }
 
 template <typename IO, int DK, int NVD>
 gdn2_status_t launch_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
-                            const void *w, float *S, void *o, int B, int H, int d_v, cudaStream_t st) {
+                            const void *w, float *S, void *o, int B, int H, int d_v, cudaStream_t st,
+                            const FuseArgs *fz) {
     dim3 grid((unsigned)((long)B * H), d_v / NVD);
-    decode_step_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
-        static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
-        static_cast<const IO *>(la), static_cast<const IO *>(b), static_cast<const IO *>(w), S,
-        static_cast<IO *>(o), d_v);
-    return from_cuda(cudaGetLastError());
+    if (fz == nullptr) {
+        decode_step_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
+            static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
+            static_cast<const IO *>(la), static_cast<const IO *>(b), static_cast<const IO *>(w), S,
+            static_cast<IO *>(o), d_v, FuseArgs{});
+        return from_cuda(cudaGetLastError());
+    }
+    // fused: the d_v / NVD blocks of one head form a cluster along y when the
+    // epilogue needs the whole row
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = (fz->gate != nullptr) ? (unsigned)(d_v / NVD) : 1u;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return from_cuda(cudaLaunchKernelEx(&cfg, decode_step_kernel<IO, DK, NVD, true>, static_cast<const IO *>(q),
+                                        static_cast<const IO *>(k), static_cast<const IO *>(v),
+                                        static_cast<const IO *>(la), static_cast<const IO *>(b),
+                                        static_cast<const IO *>(w), S, static_cast<IO *>(o), d_v, *fz));
+}
+
+// Checks the fusion arguments of the _ex entry points and fills `fz`.
+gdn2_status_t check_fuse(int flags, float l2_eps, const void *gate, const float *norm_weight, float norm_eps,
+                         FuseArgs *fz) {
+    if (flags & ~(GDN2_FUSE_INPUT_PREP | GDN2_FUSE_NEG_EIGVAL)) return GDN2_ERR_INVALID_ARG;
+    if ((flags & GDN2_FUSE_NEG_EIGVAL) && !(flags & GDN2_FUSE_INPUT_PREP)) return GDN2_ERR_INVALID_ARG;
+    if ((flags & GDN2_FUSE_INPUT_PREP) && !(l2_eps >= 0.f)) return GDN2_ERR_INVALID_ARG;
+    if (gate != nullptr && (norm_weight == nullptr || !(norm_eps >= 0.f))) return GDN2_ERR_INVALID_ARG;
+    if ((gate && !aligned16(gate)) || (norm_weight && !aligned16(norm_weight))) return GDN2_ERR_MISALIGNED;
+    fz->prep = (flags & GDN2_FUSE_INPUT_PREP) ? 1 : 0;
+    fz->neg_eigval = (flags & GDN2_FUSE_NEG_EIGVAL) ? 1 : 0;
+    fz->l2_eps = l2_eps;
+    fz->gate = gate;
+    fz->norm_weight = gate ? norm_weight : nullptr;
+    fz->norm_eps = norm_eps;
+    return GDN2_OK;
 }
 
 // Shared validation of the chunk entry points.
@@ -145,13 +217,24 @@ gdn2_status_t empty_sequence(const float *S0, float *S_T, int B, int H, int d_k,
 
 gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
                             const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
-                            int d_v, gdn2_io_t io, cudaStream_t st) {
+                            int d_v, gdn2_io_t io, cudaStream_t st, const FuseArgs *fz = nullptr) {
     if (io == GDN2_IO_F32) {
-        if (d_k == 64) return launch_ffma<float, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
-        return launch_ffma<float, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
+        if (d_k == 64) return launch_ffma<float, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+        return launch_ffma<float, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
     }
-    if (d_k == 64) return launch_ffma<__nv_bfloat16, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
-    return launch_ffma<__nv_bfloat16, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st);
+    if (d_k == 64) return launch_ffma<__nv_bfloat16, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+    return launch_ffma<__nv_bfloat16, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+}
+
+gdn2_status_t dispatch_tc(const void *q, const void *k, const void *v, const void *la, const void *b,
+                          const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
+                          int d_v, cudaStream_t st, const FuseArgs *fz = nullptr) {
+    const bool wide = (d_v % 128 == 0);
+    if (d_k == 64)
+        return wide ? launch_tc<64, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz)
+                    : launch_tc<64, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+    return wide ? launch_tc<128, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz)
+                : launch_tc<128, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
 }
 
 }  // namespace
@@ -167,12 +250,25 @@ extern "C" gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
     if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st);
-    const bool wide = (d_v % 128 == 0);
-    if (d_k == 64)
-        return wide ? launch_tc<64, 128>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st)
-                    : launch_tc<64, 64>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st);
-    return wide ? launch_tc<128, 128>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st)
-                : launch_tc<128, 64>(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_v, st);
+    return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, st);
+}
+
+extern "C" gdn2_status_t gdn2_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *log_alpha,
+                                           const void *b, const void *w, const float *S0, void *o, float *S_T,
+                                           int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io_t io,
+                                           int flags, float l2_eps, const void *gate, const float *norm_weight,
+                                           float norm_eps, void *stream) {
+    FuseArgs fz;
+    gdn2_status_t s = check_fuse(flags, l2_eps, gate, norm_weight, norm_eps, &fz);
+    if (s != GDN2_OK) return s;
+    s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, io);
+    if (s != GDN2_OK) return s;
+    if (T > 0 && gate == nullptr && norm_weight != nullptr) return GDN2_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
+    if (io == GDN2_IO_F32)
+        return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st, &fz);
+    return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, st, &fz);
 }
 
 extern "C" gdn2_status_t gdn2_chunk_fwd_cuda_core(const void *q, const void *k, const void *v,
@@ -186,9 +282,11 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_cuda_core(const void *q, const void *k, 
     return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st);
 }
 
-extern "C" gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
-                                          const void *b, const void *w, float *S, void *o, int B, int H, int d_k,
-                                          int d_v, gdn2_io_t io, void *stream) {
+namespace gdn2 {
+namespace {
+gdn2_status_t decode_impl(const void *q, const void *k, const void *v, const void *log_alpha, const void *b,
+                          const void *w, float *S, void *o, int B, int H, int d_k, int d_v, gdn2_io_t io,
+                          void *stream, const FuseArgs *fz) {
     if (!q || !k || !v || !log_alpha || !b || !w || !S || !o) return GDN2_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || d_k <= 0 || d_v <= 0) return GDN2_ERR_INVALID_ARG;
     if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
@@ -201,8 +299,8 @@ extern "C" gdn2_status_t gdn2_decode_step(const void *q, const void *k, const vo
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool wide = (d_v % 128 == 0);
 #define GDN2_DECODE(IO, DK)                                                                            \
-    return wide ? launch_decode<IO, DK, 128>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st)             \
-                : launch_decode<IO, DK, 64>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st)
+    return wide ? launch_decode<IO, DK, 128>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st, fz)         \
+                : launch_decode<IO, DK, 64>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st, fz)
     if (io == GDN2_IO_F32) {
         if (d_k == 64) GDN2_DECODE(float, 64);
         GDN2_DECODE(float, 128);
@@ -210,6 +308,25 @@ extern "C" gdn2_status_t gdn2_decode_step(const void *q, const void *k, const vo
     if (d_k == 64) GDN2_DECODE(__nv_bfloat16, 64);
     GDN2_DECODE(__nv_bfloat16, 128);
 #undef GDN2_DECODE
+}
+}  // namespace
+}  // namespace gdn2
+
+extern "C" gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
+                                          const void *b, const void *w, float *S, void *o, int B, int H, int d_k,
+                                          int d_v, gdn2_io_t io, void *stream) {
+    return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, d_k, d_v, io, stream, nullptr);
+}
+
+extern "C" gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *log_alpha,
+                                             const void *b, const void *w, float *S, void *o, int B, int H,
+                                             int d_k, int d_v, gdn2_io_t io, int flags, float l2_eps,
+                                             const void *gate, const float *norm_weight, float norm_eps,
+                                             void *stream) {
+    FuseArgs fz;
+    const gdn2_status_t s = check_fuse(flags, l2_eps, gate, norm_weight, norm_eps, &fz);
+    if (s != GDN2_OK) return s;
+    return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, d_k, d_v, io, stream, &fz);
 }
 
 extern "C" gdn2_status_t gdn2_device_status(void *stream) {

@@ -19,6 +19,8 @@
  * and "Fused Recurrent (infer)"):
  *   gdn2_chunk_fwd   -- a whole sequence, chunk-parallel (chunked WY form);
  *   gdn2_decode_step -- one token per sequence against a caller-held state.
+ * Their _ex forms also fuse the input prep (L2-norm of q and k, sigmoid
+ * gates) and the gated RMS-norm output epilogue around the mixer.
  *
  * Common conventions
  * ------------------
@@ -128,6 +130,59 @@ gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v,
                                const void *log_alpha, const void *b, const void *w,
                                float *S, void *o, int B, int H, int d_k, int d_v,
                                gdn2_io_t io, void *stream);
+
+/*
+ * Fusion flags of the _ex entry points (burn-gdn2 README, "Architecture":
+ * the L2-Norm drawn before the mixer; "Configuration": allow_neg_eigval).
+ */
+#define GDN2_FUSE_INPUT_PREP 1   /* q, k, b, w are raw projections:
+                                    q <- q / sqrt(sum_i q_i^2 + l2_eps) over d_k, k likewise,
+                                    b <- sigmoid(b), w <- sigmoid(w) */
+#define GDN2_FUSE_NEG_EIGVAL 2   /* with INPUT_PREP: b <- 2 sigmoid(b), in (0, 2) */
+
+/*
+ * gdn2_chunk_fwd_ex / gdn2_decode_step_ex -- gdn2_chunk_fwd and
+ * gdn2_decode_step with the steps the README's "Architecture" diagram draws
+ * around the mixer fused into the same pass:
+ *
+ *   flags        : 0 or GDN2_FUSE_INPUT_PREP [| GDN2_FUSE_NEG_EIGVAL].  With
+ *                  INPUT_PREP the kernels read raw q, k, b, w and apply the
+ *                  maps above while loading them; the recurrence is then the
+ *                  one documented for gdn2_chunk_fwd on the prepared values.
+ *                  l2_eps (>= 0) is only read with INPUT_PREP.
+ *   gate         : NULL, or the output gate g [B, T, H, d_v] (decode:
+ *                  [B, H, d_v]), dtype io.  Non-NULL switches the output
+ *                  epilogue ("Gated RMS Norm <- SiLU Gate") on: per (token,
+ *                  head) the stored output is
+ *                      y_j = o_j / sqrt(mean_j o_j^2 + norm_eps) * norm_weight_j * silu(g_j)
+ *                  with silu(x) = x sigmoid(x), instead of o.
+ *   norm_weight  : float32 [d_v], one weight vector shared by all heads;
+ *                  required with gate, 16-byte aligned.
+ *   norm_eps     : >= 0 (the README default is 1e-5).
+ *
+ * The epilogue is applied before o is stored whenever one CTA holds a whole
+ * d_v row (tensor-core chunk kernel: d_v = 64 or 128; decode: any d_v, the
+ * CTAs of one head forming a thread-block cluster); otherwise (tensor-core
+ * chunk kernel with d_v > 128, CUDA-core chunk kernel) o is normalised in
+ * place by one more pass in the same stream.  With flags = 0 and gate = NULL
+ * these calls are gdn2_chunk_fwd and gdn2_decode_step.  Other arguments,
+ * shapes and errors as there; bad flags, a gate without norm_weight or a
+ * negative epsilon return GDN2_ERR_INVALID_ARG.
+ */
+gdn2_status_t gdn2_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                                const void *log_alpha, const void *b, const void *w,
+                                const float *S0, void *o, float *S_T,
+                                int B, int T, int H, int d_k, int d_v, int chunk,
+                                gdn2_io_t io, int flags, float l2_eps,
+                                const void *gate, const float *norm_weight, float norm_eps,
+                                void *stream);
+
+gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v,
+                                  const void *log_alpha, const void *b, const void *w,
+                                  float *S, void *o, int B, int H, int d_k, int d_v,
+                                  gdn2_io_t io, int flags, float l2_eps,
+                                  const void *gate, const float *norm_weight, float norm_eps,
+                                  void *stream);
 
 /*
  * gdn2_device_status -- synchronise `stream`, then read and clear the

@@ -88,3 +88,28 @@ def test_product_path_does_not_touch_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 with open(os.path.join(dirpath, fn)) as f:
                     assert "oracle" not in f.read().lower(), fn
+
+
+def test_fused_argument_validation_on_host(L):
+    """The _ex calls check their fusion arguments before touching the device."""
+    P, F = ctypes.c_void_p, ctypes.c_float
+    p, w = P(16), P(32)
+
+    def chunk_ex(flags=0, l2=1e-6, gate=None, weight=None, eps=1e-5, T=64):
+        return L.gdn2_chunk_fwd_ex(p, p, p, p, p, p, None, p, None, 1, T, 1, 64, 64, 64, 1,
+                                   flags, F(l2), gate, weight, F(eps), None)
+
+    def decode_ex(flags=0, l2=1e-6, gate=None, weight=None, eps=1e-5):
+        return L.gdn2_decode_step_ex(p, p, p, p, p, p, p, p, 1, 1, 64, 64, 1,
+                                     flags, F(l2), gate, weight, F(eps), None)
+
+    for call in (chunk_ex, decode_ex):
+        assert call(flags=8) == 1                     # unknown flag
+        assert call(flags=2) == 1                     # negative eigenvalues without the prep
+        assert call(flags=1, l2=-1.0) == 1            # negative L2 epsilon
+        assert call(gate=p) == 1                      # gate without norm_weight
+        assert call(gate=p, weight=w, eps=-1.0) == 1  # negative norm epsilon
+        assert call(gate=P(18), weight=w) == 3        # misaligned gate
+        assert call(gate=p, weight=P(20)) == 3        # misaligned weight
+    assert chunk_ex(flags=3, T=0, gate=p, weight=w) == 0   # empty sequence: nothing to do
+    assert chunk_ex(weight=w) == 1                         # weight without gate

@@ -32,7 +32,7 @@ MUTANTS = {
 FUSED_MUTANTS = {
     "l2_without_sqrt": ("const double nq = sqrt(sq + f->l2_eps), nk = sqrt(sk + f->l2_eps);",
                         "const double nq = sq + f->l2_eps, nk = sk + f->l2_eps;"),
-    "l2_key_skipped": ("kd[i] /= nk;", "kd[i] /= 1.0;"),
+    "l2_key_skipped": ("kd[i] *= ik;", "kd[i] *= 1.0;"),
     "logistic_sign": ("static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }",
                       "static double sigmoid(double x) { return 1.0 / (1.0 + exp(x)); }"),
     "neg_eigval_ignored": ("(f->neg_eigval ? 2.0 : 1.0)", "(1.0)"),

@@ -112,6 +112,41 @@ def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
     return out
 
 
+def draw_raw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
+             dtype=torch.bfloat16, alpha_lo: float = 0.9, alpha_hi: float = 0.999,
+             qk_scale: float = 1.0, s0_std: Optional[float] = None, steps: Optional[int] = None,
+             generator: Optional[torch.Generator] = None, device="cpu") -> dict:
+    """Inputs for the fused input prep and output epilogue: the raw
+    projections the layer would hand the mixer.
+
+    q, k ~ qk_scale N(0,1) (not normalised); b, w ~ N(0,1) (gate logits);
+    v ~ N(0,1); alpha ~ U[alpha_lo, alpha_hi], log_alpha = ln alpha; the
+    output gate g ~ N(0,1); the RMS-norm weight ~ U[0.5, 1.5] (synthetic, one
+    [d_v] vector, fp32); S0 ~ N(0, s0_std) or None.  Token tensors are
+    [B, T, H, d], or [steps, B, H, d] for decode when ``steps`` is given.
+    """
+    g = generator if generator is not None else torch.Generator(device=device).manual_seed(seed)
+    f32 = torch.float32
+    kw = dict(generator=g, dtype=f32, device=device)
+    lead = (steps, B, H) if steps is not None else (B, T, H)
+    q = qk_scale * torch.randn(*lead, d_k, **kw)
+    k = qk_scale * torch.randn(*lead, d_k, **kw)
+    v = torch.randn(*lead, d_v, **kw)
+    alpha = torch.empty(*lead, d_k, dtype=f32, device=device).uniform_(alpha_lo, alpha_hi, generator=g)
+    b = torch.randn(*lead, d_k, **kw)
+    w = torch.randn(*lead, d_v, **kw)
+    gate = torch.randn(*lead, d_v, **kw)
+    weight = torch.empty(d_v, dtype=f32, device=device).uniform_(0.5, 1.5, generator=g)
+    S0 = None
+    if s0_std is not None:
+        S0 = s0_std * torch.randn(B, H, d_k, d_v, **kw)
+    out = dict(q=q, k=k, v=v, log_alpha=torch.log(alpha), b=b, w=w, gate=gate)
+    out = {n: t.to(dtype).contiguous() for n, t in out.items()}
+    out["S0"] = S0
+    out["norm_weight"] = weight
+    return out
+
+
 def make_chunk_inputs(wl: Workload, *, B: Optional[int] = None, T: Optional[int] = None,
                       H: Optional[int] = None, seed: Optional[int] = None, device="cpu") -> dict:
     """Inputs of a chunk workload (optionally resized, same recipe)."""
