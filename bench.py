@@ -229,6 +229,53 @@ def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None):
     return ms, d, o, S_T
 
 
+def bench_chunk_fused(g, wl, steps, warmup, rank, stream):
+    """The workload's shapes from raw projections: fused input prep (L2 norm of
+    q, k; sigmoid gates) and the gated RMS-norm epilogue in the same call."""
+    d = W.draw_raw(wl.B, wl.T, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 7, dtype=wl.torch_dtype,
+                   alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, qk_scale=2.0, s0_std=wl.s0_std, device="cuda")
+    o = torch.empty_like(d["v"])
+    S_T = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
+
+    def step():
+        g.chunk_fwd_ex(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], prep=True,
+                       gate=d["gate"], norm_weight=d["norm_weight"], o=o, S_T=S_T, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    torch.cuda.synchronize()
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("fused chunk kernel reported a device timeout")
+    return ms / steps
+
+
+def bench_decode_fused(g, wl, steps, rank, stream):
+    d = W.draw_raw(wl.B, None, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 7, dtype=wl.torch_dtype,
+                   alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, qk_scale=2.0, s0_std=wl.s0_std, steps=steps,
+                   device="cuda")
+    S = d["S0"].clone()
+    o = torch.empty(wl.B, wl.H, wl.d_v, dtype=wl.torch_dtype, device="cuda")
+    it = {"s": 0}
+
+    def step():
+        s = it["s"] % steps
+        it["s"] += 1
+        g.decode_step_ex(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["b"][s], d["w"][s], S,
+                         prep=True, gate=d["gate"][s], norm_weight=d["norm_weight"], o=o, stream=stream)
+
+    for _ in range(8):
+        step()
+    torch.cuda.synchronize()
+    S.copy_(d["S0"])
+    it["s"] = 0
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("fused decode kernel reported a device timeout")
+    return ms / steps
+
+
 def bench_chunk_e2e(g, wl, d, steps, stream):
     """Same call through the public API, with pinned host inputs copied in
     and o, S_T copied out inside the timed region, every step."""
@@ -449,6 +496,27 @@ def main():
                          "unit": "GB/s", "frac": b4 / (per / 1e3) / 1e9 / peaks["hbm_gbs"],
                          "bytes_per_step": b4, "traffic": measured_traffic("decode_step", wl4.B)},
             "clocks": s4.summary()}
+        torch.cuda.empty_cache()
+        # f1 + f2: the headline chunk workload and the decode workload from raw
+        # projections, input prep and gated RMS-norm epilogue fused in
+        io_b = 2 if wl.io == "bf16" else 4
+        lf = bench_chunk_fused(g, wl, max(10, args.steps // 4), 3, rank, stream)
+        bf = chunk_bytes(wl, with_s0=wl.s0_std is not None) + wl.B * wl.T * wl.H * wl.d_v * io_b + 4 * wl.d_v
+        extras["chunk_fused_prep_epilogue"] = {
+            "workload": wl.describe() + " + fused input prep + gated RMS-norm epilogue",
+            "value": wl.B * wl.T / (lf / 1e3), "unit": "tokens/s", "ms_per_call": lf,
+            "roofline": {"bound": "hbm", "achieved": bf / (lf / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": bf / (lf / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_launch": bf}}
+        torch.cuda.empty_cache()
+        nfs = 256
+        pf = bench_decode_fused(g, wl4, nfs, rank, stream)
+        bdf = decode_bytes(wl4) + wl4.B * wl4.H * wl4.d_v * 2 + 4 * wl4.d_v
+        extras["decode_fused_prep_epilogue"] = {
+            "workload": wl4.describe().replace(f"steps{wl4.decode_steps}", f"steps{nfs}")
+            + " + fused input prep + gated RMS-norm epilogue",
+            "value": wl4.B / (pf / 1e3), "unit": "tokens/s", "us_per_step": 1e3 * pf, "steps": nfs,
+            "roofline": {"bound": "hbm", "achieved": bdf / (pf / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": bdf / (pf / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_step": bdf}}
         torch.cuda.empty_cache()
 
     cpu = None

@@ -63,7 +63,9 @@ struct TcCfg {
     static constexpr uint32_t OFF_U = OFF_S + VB * 16384u; // U [jb][64 i][64 j]
     static constexpr uint32_t OFF_CARRY = OFF_U + VB * 8192u;   // cumsum carries [row block][128]
     static constexpr uint32_t OFF_GC = OFF_CARRY + 2048;         // exp(G_C) [3][128]
-    static constexpr uint32_t OFF_BAR = OFF_GC + 1536;
+    static constexpr uint32_t OFF_NRM = OFF_GC + 1536;           // fused prep: 1/|q_r|, 1/|k_r| [64][2]
+    static constexpr uint32_t OFF_NW = OFF_NRM + 512;            // fused epilogue: norm weight [NV]
+    static constexpr uint32_t OFF_BAR = OFF_NW + 512;
     static constexpr uint32_t OFF_TMEMP = OFF_BAR + 256;   // up to 32 mbarriers
     static constexpr uint32_t SMEM_BYTES = OFF_TMEMP + 16;
     static constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -240,18 +242,38 @@ struct PrepLA {
 // it (exchanged through `carry` and named barrier `bar` over the 128
 // threads).  A half-warp covers 16 consecutive quads = one 128-byte swizzled
 // row, so the 8-byte shared accesses are conflict-free.
-// With fz.prep (FUSED only) q, k, b arrive raw: each row of q and k is scaled
-// by 1 / sqrt(sum^2 + l2_eps) (the sums over d_k reduced across the NP lanes
-// that share the row) and b becomes sigmoid(b) (x2 with neg_eigval).
-template <int DK, bool FUSED = false>
+// With PREP, q, k, b arrive raw: each row of q and k is scaled by
+// 1 / sqrt(sum^2 + l2_eps) (a pre-pass: thread t sums row t % 64 of q (t < 64)
+// or of k, and leaves the factor in `nrm`) and b becomes sigmoid(b) (x2 with
+// neg_eigval).
+template <int DK, bool PREP = false>
 __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLA<DK> &law,
-                                           float *gc, float *carry, int g, int bar, const FuseArgs &fz = {}) {
+                                           float *gc, float *carry, int g, int bar, const FuseArgs &fz = {},
+                                           float2 *nrm = nullptr) {
     constexpr int NP = PrepLA<DK>::NP, NB = PrepLA<DK>::NB, R = PrepLA<DK>::R;
     static_assert(NB * R == 64 && NB <= 8, "prep split");
     const int p = g % NP, hb = g / NP;
     const int kb = p >> 4, cb = (p & 15) * 8;   // channel block, byte in the 128-byte row
     uint8_t *q_t = smem + oqe + kb * 16384, *e_t = q_t + 8192, *k_t = smem + okt + kb * 8192;
     auto off = [&](int r) { return r * 128 + ((((cb >> 4) ^ r) & 7) << 4) + (cb & 15); };
+    if constexpr (PREP) {   // 1 / |row| of q (threads 0-63) and k (64-127)
+        const int r = g & 63;
+        const uint8_t *base = (g < 64) ? smem + oqe : smem + okt;
+        const uint32_t kstride = (g < 64) ? 16384u : 8192u;
+        float ss = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < DK / 8; ++c8) {
+            uint32_t a0, a1, a2, a3;
+            ld_shared_v4(smem_u32(base + (c8 >> 3) * kstride) + sw128_chunk(r, c8 & 7), a0, a1, a2, a3);
+            const uint32_t aa[4] = {a0, a1, a2, a3};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                ss = fmaf(bf16_lo(aa[e]), bf16_lo(aa[e]), ss);
+                ss = fmaf(bf16_hi(aa[e]), bf16_hi(aa[e]), ss);
+            }
+        }
+        reinterpret_cast<float *>(nrm)[2 * r + (g >> 6)] = l2_inv(ss, fz.l2_eps);
+    }
     // running sums in log2 units (G log2(e)), so that exp(+-G) = 2^(+-sum)
     constexpr float kLog2e = 1.4426950408889634f;
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
@@ -293,24 +315,11 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
             float rq = 1.f, rk = 1.f, bs = 1.f;
-            if constexpr (FUSED) {
-                if (fz.prep) {
-                    float sq = 0.f, sk = 0.f;
-                    const uint32_t qa[2] = {qw[j].x, qw[j].y}, ka[2] = {kw[j].x, kw[j].y};
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        sq += bf16_lo(qa[h]) * bf16_lo(qa[h]) + bf16_hi(qa[h]) * bf16_hi(qa[h]);
-                        sk += bf16_lo(ka[h]) * bf16_lo(ka[h]) + bf16_hi(ka[h]) * bf16_hi(ka[h]);
-                    }
-#pragma unroll
-                    for (int off = NP / 2; off > 0; off >>= 1) {
-                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
-                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
-                    }
-                    rq = l2_inv(sq, fz.l2_eps);
-                    rk = l2_inv(sk, fz.l2_eps);
-                    bs = fz.neg_eigval ? 2.f : 1.f;
-                }
+            if constexpr (PREP) {
+                const float2 nr = nrm[hb * R + i0 + j];
+                rq = nr.x;
+                rk = nr.y;
+                bs = fz.neg_eigval ? 2.f : 1.f;
             }
             const uint2 la2 = law.v[i0 + j];
             sum[0] = fmaf(bf16_lo(la2.x), kLog2e, sum[0]);
@@ -326,15 +335,13 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
                 float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
                 float b0 = bf16_lo(bv[h]), b1 = bf16_hi(bv[h]);
                 float q0 = bf16_lo(qv[h]), q1 = bf16_hi(qv[h]);
-                if constexpr (FUSED) {
-                    if (fz.prep) {
-                        k0 *= rk;
-                        k1 *= rk;
-                        q0 *= rq;
-                        q1 *= rq;
-                        b0 = bs * sigmoid_tanh(b0);
-                        b1 = bs * sigmoid_tanh(b1);
-                    }
+                if constexpr (PREP) {
+                    k0 *= rk;
+                    k1 *= rk;
+                    q0 *= rq;
+                    q1 *= rq;
+                    b0 = bs * sigmoid_tanh(b0);
+                    b1 = bs * sigmoid_tanh(b1);
                 }
                 oq[h] = pack_bf16x2(q0 * ga0, q1 * ga1);
                 oe[h] = pack_bf16x2(b0 * k0 * ga0, b1 * k1 * ga1);
@@ -352,16 +359,17 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
     fence_proxy_async_smem();
 }
 
-// FUSED adds the input prep (fz.prep: raw q, k, b, w) and, when fz.gate is
-// set, the gated RMS norm of each output row before it is stored; the
-// launcher sets fz.gate only when d_v == NV, so one CTA holds the whole row.
-template <int DK, int NV, bool FUSED = false>
+// PREP fuses the input prep (raw q, k, b, w); EPI the gated RMS norm of each
+// output row before it is stored (d_v == NV: one CTA holds the whole row).
+template <int DK, int NV, bool PREP = false, bool EPI = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16 *__restrict__ la,
-                    const float *__restrict__ S0, __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T,
-                    int T, int H, int d_v, unsigned long long wait_ns, const FuseArgs fz = {}) {
+                    const float *__restrict__ S0,
+                    __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int T, int H, int d_v,
+                    unsigned long long wait_ns, const FuseArgs fz) {
+    static_assert(!EPI || NV <= 128, "epilogue weight slice");
     using Cfg = TcCfg<DK, NV>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -396,6 +404,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ---------------------------------------------------------------- setup
     for (uint32_t off = tid * 16u; off < Cfg::OFF_CARRY; off += kTcThreads * 16u) st_shared_v4(sb + off, 0u, 0u, 0u, 0u);
     for (int i = tid; i < 3 * 128; i += kTcThreads) gC[i] = 1.f;   // channels >= d_k keep exp(G_C) = 1
+    if constexpr (EPI) {
+        float *nw = reinterpret_cast<float *>(smem + Cfg::OFF_NW);
+        for (int i = tid; i < NV; i += kTcThreads) nw[i] = fz.norm_weight[j0 + i];
+    }
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
         fence_mbar_init();
@@ -488,6 +500,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool grp_b = t >= 128;
         uint32_t ph1 = 0, ph2 = 0;
         float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
+        float2 *nrm = reinterpret_cast<float2 *>(smem + Cfg::OFF_NRM);
         PrepLA<DK> lan;   // group B: log_alpha of the next chunk to prepare
         // prologue: prep of chunk 0 (group B)
         if (NC > 0) {
@@ -495,7 +508,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK, FUSED>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, fz);
+            else if (grp_b) prep_chunk<DK, PREP>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, fz, nrm);
         }
         for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
@@ -530,7 +543,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ld_shared_v4(sb + Cfg::OFF_V + off, a0, a1, a2, a3);
                     ld_shared_v4(sb + Cfg::OFF_W + off, b0, b1, b2, b3);
                     uint4 r4;
-                    if (FUSED && fz.prep) {   // w arrives raw: sigmoid(w) . v, rounded once
+                    if (PREP) {   // w arrives raw: sigmoid(w) . v, rounded once
                         const uint32_t vv[4] = {a0, a1, a2, a3}, ww[4] = {b0, b1, b2, b3};
                         uint32_t rr[4];
 #pragma unroll
@@ -598,8 +611,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = ok_b && mbar_wait(&k_full[s3n], static_cast<uint32_t>(((m + 1) / 3) & 1), wait_ns);
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
-                    prep_chunk<DK, FUSED>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
-                                          gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz);
+                    prep_chunk<DK, PREP>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
+                                         gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm);
             }
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
@@ -716,6 +729,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint32_t ph1 = 0, ph2 = 0, ph3 = 0;
         for (int n = 0; n < NC; ++n) {
             const int s = n & 1;
+            if constexpr (EPI) {   // the epilogue's gate tile, into L2 a whole chain pass ahead
+                const int r = t >> 1;   // two threads per row: 2 x 128-byte lines of the NV slice
+                if (n * 64 + r < T && (t & 1) * 64 < NV)
+                    prefetch_l2(static_cast<const __nv_bfloat16 *>(fz.gate) +
+                                (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0 + (t & 1) * 64);
+            }
             const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = Cfg::OFF_K + (n % 3) * 16384u;
             const uint32_t OP = s ? Cfg::OFF_P1 : Cfg::OFF_P0;
             {
@@ -827,44 +846,30 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const long orow_off = (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0;
                 __nv_bfloat16 *orow = o + orow_off;
                 bool plain = true;
-                if constexpr (FUSED) {
-                    if (fz.gate != nullptr) {   // y = o / rms(o) . weight . silu(g)  (d_v == NV)
-                        plain = false;
-                        float ss = 0.f;
+                if constexpr (EPI) {   // first half of the epilogue: o / rms(o) -> bf16 in the U tile
+                    plain = false;
+                    float ss = 0.f;
 #pragma unroll 1
-                        for (int jc = 0; jc < NV / 32; ++jc) {
-                            float x[32];
-                            tmem_ld32(t_X + lane_q + jc * 32, x);
+                    for (int jc = 0; jc < NV / 32; ++jc) {
+                        float x[32];
+                        tmem_ld32(t_X + lane_q + jc * 32, x);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
-                        }
-                        const float inv = rsqrtf(ss / (float)NV + fz.norm_eps);
-                        const __nv_bfloat16 *grow = static_cast<const __nv_bfloat16 *>(fz.gate) + orow_off;
+                        for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
+                    }
+                    const float inv = rsqrtf(ss / (float)NV + fz.norm_eps);
 #pragma unroll 1
-                        for (int jc = 0; jc < NV / 32; ++jc) {
-                            float x[32];
-                            tmem_ld32(t_X + lane_q + jc * 32, x);
-                            if (valid) {
-                                const uint4 *gsrc = reinterpret_cast<const uint4 *>(grow + jc * 32);
-                                const float4 *wsrc = reinterpret_cast<const float4 *>(fz.norm_weight + j0 + jc * 32);
-                                uint4 *dst = reinterpret_cast<uint4 *>(orow + jc * 32);
+                    for (int jc = 0; jc < NV / 32; ++jc) {
+                        float x[32];
+                        tmem_ld32(t_X + lane_q + jc * 32, x);
+                        const uint32_t tile = sb + Cfg::OFF_U + ((jc * 32) >> 6) * 8192u;
+                        const uint32_t ch0 = ((jc * 32) & 63) >> 3;
 #pragma unroll
-                                for (int q4 = 0; q4 < 4; ++q4) {
-                                    const uint4 gv = __ldg(gsrc + q4);
-                                    const float4 w0 = __ldg(wsrc + 2 * q4), w1 = __ldg(wsrc + 2 * q4 + 1);
-                                    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-                                    const float wt[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                                    uint32_t pk[4];
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const float g0 = bf16_lo(gw[e]), g1 = bf16_hi(gw[e]);
-                                        pk[e] = pack_bf16x2(x[8 * q4 + 2 * e] * inv * wt[2 * e] * g0 * sigmoid_tanh(g0),
-                                                            x[8 * q4 + 2 * e + 1] * inv * wt[2 * e + 1] * g1 *
-                                                                sigmoid_tanh(g1));
-                                    }
-                                    dst[q4] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                                }
-                            }
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int e = 8 * q4;
+                            st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(x[e] * inv, x[e + 1] * inv),
+                                         pack_bf16x2(x[e + 2] * inv, x[e + 3] * inv),
+                                         pack_bf16x2(x[e + 4] * inv, x[e + 5] * inv),
+                                         pack_bf16x2(x[e + 6] * inv, x[e + 7] * inv));
                         }
                     }
                 }
@@ -881,6 +886,44 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                                  pack_bf16x2(x[e + 4], x[e + 5]), pack_bf16x2(x[e + 6], x[e + 7]));
                         }
                     }
+                }
+            }
+            if constexpr (EPI) {   // second half: . weight . silu(g), coalesced, by all four warps
+                named_bar(2, kChainThreads);
+                const float *nw = reinterpret_cast<const float *>(smem + Cfg::OFF_NW);
+                constexpr int CPR = NV / 8;                 // 16-byte chunks per row
+                constexpr int RPP = kChainThreads / CPR;    // rows per pass
+                const int c16 = t % CPR, rr = t / CPR;
+                const float4 w0 = *reinterpret_cast<const float4 *>(nw + 8 * c16);
+                const float4 w1 = *reinterpret_cast<const float4 *>(nw + 8 * c16 + 4);
+                const float wt[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                const __nv_bfloat16 *gbase = static_cast<const __nv_bfloat16 *>(fz.gate);
+                uint4 gall[64 / RPP];   // every gate load of this thread issued up front
+#pragma unroll
+                for (int i = 0; i < 64 / RPP; ++i) {
+                    const int r = i * RPP + rr;
+                    gall[i] = (n * 64 + r < T)
+                                  ? __ldg(reinterpret_cast<const uint4 *>(
+                                        gbase + (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0 + 8 * c16))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int i = 0; i < 64 / RPP; ++i) {
+                    const int r = i * RPP + rr;
+                    if (n * 64 + r >= T) continue;   // padding rows
+                    const long off = (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0 + 8 * c16;
+                    const uint4 gv = gall[i];
+                    uint32_t a0, a1, a2, a3;
+                    ld_shared_v4(sb + Cfg::OFF_U + (c16 >> 3) * 8192u + sw128_chunk(r, c16 & 7), a0, a1, a2, a3);
+                    const uint32_t ov[4] = {a0, a1, a2, a3}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float g0 = bf16_lo(gw[e]), g1 = bf16_hi(gw[e]);
+                        pk[e] = pack_bf16x2(bf16_lo(ov[e]) * wt[2 * e] * g0 * sigmoid_tanh(g0),
+                                            bf16_hi(ov[e]) * wt[2 * e + 1] * g1 * sigmoid_tanh(g1));
+                    }
+                    *reinterpret_cast<uint4 *>(o + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
             tmem_st_wait();

@@ -268,6 +268,10 @@ __device__ __forceinline__ float l2_inv(float s, float eps) {
     const float d = s + eps;
     return d > 0.f ? rsqrtf(d) : 0.f;
 }
+// Hint: bring the 128-byte line holding `p` into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 // Logistic function 1 / (1 + e^-x) with an IEEE division (fp32-I/O paths).
 __device__ __forceinline__ float sigmoid_f32(float x) { return 1.f / (1.f + __expf(-x)); }
 // Logistic function as 0.5 + 0.5 tanh(x / 2) with the one-instruction tanh

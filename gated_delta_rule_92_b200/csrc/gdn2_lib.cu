@@ -81,37 +81,41 @@ gdn2_status_t launch_rmsnorm(void *o, const void *g, const float *weight, long r
     return from_cuda(cudaGetLastError());
 }
 
+template <int DK, int NV, bool PREP, bool EPI>
+gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
+                               const CUtensorMap &tv, const CUtensorMap &tw, const void *la, const float *S0, void *o, float *S_T, int B, int T, int H,
+                               int d_v, cudaStream_t st, const FuseArgs &fz) {
+    using Cfg = TcCfg<DK, NV>;
+    auto kern = chunk_fwd_tc_kernel<DK, NV, PREP, EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
+    if (e != cudaSuccess) return GDN2_ERR_CUDA;
+    dim3 grid(d_v / NV, H, B);
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, static_cast<const __nv_bfloat16 *>(la),
+                                                    S0, static_cast<__nv_bfloat16 *>(o), S_T, T, H, d_v, kWaitNs,
+                                                    fz);
+    return from_cuda(cudaGetLastError());
+}
+
 template <int DK, int NV>
 gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void *la, const void *b, const void *w,
                         const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st,
                         const FuseArgs *fz = nullptr) {
-    using Cfg = TcCfg<DK, NV>;
     CUtensorMap tq, tk, tb, tv, tw;
     if (!make_token_map(&tq, q, B, T, H, DK) || !make_token_map(&tk, k, B, T, H, DK) ||
         !make_token_map(&tb, b, B, T, H, DK) || !make_token_map(&tv, v, B, T, H, d_v) ||
         !make_token_map(&tw, w, B, T, H, d_v))
         return GDN2_ERR_CUDA;
-    dim3 grid(d_v / NV, H, B);
-    const __nv_bfloat16 *lap = static_cast<const __nv_bfloat16 *>(la);
-    __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(o);
-    if (fz == nullptr) {
-        auto kern = chunk_fwd_tc_kernel<DK, NV>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
-        if (e != cudaSuccess) return GDN2_ERR_CUDA;
-        kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, lap, S0, op, S_T, T, H, d_v, kWaitNs,
-                                                        FuseArgs{});
-        return from_cuda(cudaGetLastError());
-    }
+    const bool prep = fz != nullptr && fz->prep;
     // the in-kernel epilogue needs the whole d_v row in one CTA; otherwise one
     // more pass normalises o in place
-    FuseArgs kf = *fz;
-    if (d_v != NV) kf.gate = nullptr;
-    auto kern = chunk_fwd_tc_kernel<DK, NV, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
-    if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, lap, S0, op, S_T, T, H, d_v, kWaitNs, kf);
-    gdn2_status_t s = from_cuda(cudaGetLastError());
-    if (s != GDN2_OK || fz->gate == nullptr || kf.gate != nullptr) return s;
+    const bool epi = fz != nullptr && fz->gate != nullptr && d_v == NV;
+    const FuseArgs kf = fz ? *fz : FuseArgs{};
+    gdn2_status_t s;
+    if (prep && epi) s = launch_tc_kernel<DK, NV, true, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
+    else if (prep) s = launch_tc_kernel<DK, NV, true, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
+    else if (epi) s = launch_tc_kernel<DK, NV, false, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
+    else s = launch_tc_kernel<DK, NV, false, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
+    if (s != GDN2_OK || fz == nullptr || fz->gate == nullptr || epi) return s;
     return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, (long)B * T * H, d_v, fz->norm_eps, st);
 }
 
