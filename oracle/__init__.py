@@ -51,7 +51,7 @@ def open_library(path: str):
     lib.gdn2_oracle_forward.restype = I
     D = ctypes.c_double
     lib.gdn2_oracle_forward_ex.argtypes = [P, P, P, P, P, P, P, P, P, P,
-                                           I, I, I, I, I, P, I, I,
+                                           I, I, I, I, I, I, P, P, I, I,
                                            I, D, P, P, D]
     lib.gdn2_oracle_forward_ex.restype = I
     lib.gdn2_oracle_max_threads.restype = I
@@ -83,7 +83,7 @@ def _ptr(a):
 def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
             want_state: bool = True, want_smax: bool = False, lib=None, *,
             prep: bool = False, allow_neg_eigval: bool = False, l2_eps: float = 1e-6,
-            gate=None, norm_weight=None, norm_eps: float = 1e-5):
+            gate=None, norm_weight=None, norm_eps: float = 1e-5, cu_seqlens=None):
     """Run the recurrence in fp64.
 
     q, k, log_alpha, b : [B, T, H, d_k];  v, w : [B, T, H, d_v] (any float
@@ -100,34 +100,52 @@ def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
     [B, T, H, d_v] with norm_weight [d_v] returns the gated RMS norm
     o / sqrt(mean(o^2) + norm_eps) * norm_weight * silu(gate) per (token, head)
     instead of o (README "Architecture": Gated RMS Norm <- SiLU Gate).
+
+    Value heads: v, w (and gate) may have HV = G H heads (README
+    "Configuration", num_v_heads); value head hv then reads key head hv // G,
+    and heads / S0 / S_T index the B * HV value heads.  cu_seqlens ([N + 1],
+    cu[0] = 0, non-decreasing, cu[N] = T): N sequences packed along the token
+    axis of [1, T, H, d] inputs; o is then a list with one [len, d_v] array per
+    requested head, S0 / S_T are [N, HV, d_k, d_v].
     """
     q, k, v, la, b, w = (_f32(x) for x in (q, k, v, log_alpha, b, w))
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+    Bt, T, H, dk = q.shape
+    HV, dv = v.shape[-2], v.shape[-1]
     for x in (k, la, b):
-        assert x.shape == (B, T, H, dk), x.shape
+        assert x.shape == (Bt, T, H, dk), x.shape
     for x in (v, w):
-        assert x.shape == (B, T, H, dv), x.shape
+        assert x.shape == (Bt, T, HV, dv), x.shape
+    assert HV % H == 0, (H, HV)
+    cu = None
+    if cu_seqlens is not None:
+        assert Bt == 1, "packed sequences take [1, T, H, d] inputs"
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        B = int(cu.size) - 1
+    else:
+        B = Bt
     s0 = None
     if S0 is not None:
         if hasattr(S0, "detach"):
             S0 = S0.detach().double().cpu().numpy()
         s0 = np.ascontiguousarray(np.asarray(S0, dtype=np.float64))
-        assert s0.shape == (B, H, dk, dv), s0.shape
+        assert s0.shape == (B, HV, dk, dv), s0.shape
     if heads is None:
         hl = None
-        nh = B * H
+        nh = B * HV
     else:
         hl = np.ascontiguousarray(np.asarray(list(heads), dtype=np.int32))
         nh = int(hl.size)
-    o = np.empty((nh, T, dv), dtype=np.float64)
+    hidx = range(B * HV) if hl is None else [int(x) for x in hl]
+    lens = [(int(cu[x // HV + 1] - cu[x // HV]) if 0 <= x < B * HV else 0) if cu is not None else T
+            for x in hidx]
+    o = np.empty((max(1, sum(lens)), dv), dtype=np.float64)
     st = np.empty((nh, dk, dv), dtype=np.float64) if want_state else None
     sm = np.empty((nh,), dtype=np.float64) if want_smax else None
     g = None
     wt = None
     if gate is not None:
         g = _f32(gate)
-        assert g.shape == (B, T, H, dv), g.shape
+        assert g.shape == (Bt, T, HV, dv), g.shape
         assert norm_weight is not None, "the epilogue needs norm_weight"
         if hasattr(norm_weight, "detach"):
             norm_weight = norm_weight.detach().double().cpu().numpy()
@@ -136,10 +154,15 @@ def forward(q, k, v, log_alpha, b, w, S0=None, heads=None, n_threads: int = 0,
     pflag = (1 | (2 if allow_neg_eigval else 0)) if prep else 0
     rc = (lib or _load()).gdn2_oracle_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w),
                                         _ptr(s0), _ptr(o), _ptr(st), _ptr(sm),
-                                        B, T, H, dk, dv, _ptr(hl), nh, int(n_threads),
+                                        B, T, H, HV, dk, dv, _ptr(cu), _ptr(hl), nh, int(n_threads),
                                         pflag, float(l2_eps), _ptr(g), _ptr(wt), float(norm_eps))
     if rc != 0:
         raise ValueError("gdn2 oracle rejected its arguments")
+    if cu is not None:
+        offs = np.cumsum([0] + lens)
+        o = [o[offs[i]:offs[i + 1]] for i in range(nh)]
+    else:
+        o = o[:nh * T].reshape(nh, T, dv)
     if want_smax:
         return o, st, sm
     return o, st

@@ -42,7 +42,8 @@
  * README's "Architecture" diagram draws next to it, each optional:
  *   input prep  (the "L2-Norm" after the projections; "Configuration",
  *                allow_neg_eigval "b x 2"):
- *       q = q_raw / sqrt(sum_i q_raw_i^2 + l2_eps), k likewise (over d_k),
+ *       q = q_raw / sqrt(sum_i q_raw_i^2 + l2_eps), k likewise (over d_k;
+ *           a zero vector with l2_eps = 0 stays zero),
  *       b = sigmoid(b_raw) (times 2 with allow_neg_eigval), w = sigmoid(w_raw);
  *   output epilogue ("Gated RMS Norm <- SiLU Gate"; "Configuration",
  *                norm_eps):
@@ -80,9 +81,11 @@ static void token_inputs(const float *qt, const float *kt, const float *bt, cons
     double sq = 0.0, sk = 0.0;
     for (long i = 0; i < dk; ++i) { sq += qd[i] * qd[i]; sk += kd[i] * kd[i]; }
     const double nq = sqrt(sq + f->l2_eps), nk = sqrt(sk + f->l2_eps);
+    /* reading: a zero vector (with l2_eps = 0) normalises to the zero vector */
+    const double iq = nq > 0.0 ? 1.0 / nq : 0.0, ik = nk > 0.0 ? 1.0 / nk : 0.0;
     for (long i = 0; i < dk; ++i) {
-        qd[i] /= nq;
-        kd[i] /= nk;
+        qd[i] *= iq;
+        kd[i] *= ik;
         bd[i] = (f->neg_eigval ? 2.0 : 1.0) * sigmoid(bd[i]);
     }
     for (long j = 0; j < dv; ++j) wd[j] = sigmoid(wd[j]);
@@ -91,7 +94,7 @@ static void token_inputs(const float *qt, const float *kt, const float *bt, cons
 static int run_head(const float *q, const float *k, const float *v,
                     const float *la, const float *b, const float *w, const float *g,
                     const double *S0, double *o, double *S_T, double *smax,
-                    long T, long H, long dk, long dv, const fuse_t *f)
+                    long T, long H, long HV, long dk, long dv, const fuse_t *f)
 {
     double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
     double *r = (double *)malloc(sizeof(double) * (size_t)dv);
@@ -102,7 +105,7 @@ static int run_head(const float *q, const float *k, const float *v,
     if (S0) memcpy(S, S0, sizeof(double) * (size_t)(dk * dv));
     else    memset(S, 0, sizeof(double) * (size_t)(dk * dv));
     double big = 0.0;
-    const long sk = H * dk, sv = H * dv;   /* stride between tokens */
+    const long sk = H * dk, sv = HV * dv;   /* stride between tokens */
     for (long t = 0; t < T; ++t) {
         const float *lat = la + t * sk, *vt = v + t * sv;
         token_inputs(q + t * sk, k + t * sk, b + t * sk, w + t * sv, qd, kd, bd, wd, dk, dv, f);
@@ -156,18 +159,39 @@ static int run_head(const float *q, const float *k, const float *v,
     return 0;
 }
 
+/* One recurrence per (sequence, value head).  Sequence n covers tokens
+ * [cu[n], cu[n+1]) of the packed token axis when cu is given (token tensors
+ * are then [1, T, H or HV, d]); otherwise B sequences of T tokens.  Value head
+ * hv (of HV = G H) reads key head hv / G for q, k, log_alpha and b. */
 static int forward_impl(const float *q, const float *k, const float *v,
                         const float *log_alpha, const float *b, const float *w,
                         const double *S0, double *o, double *S_T, double *smax,
-                        int B, int T, int H, int d_k, int d_v,
+                        int B, int T, int H, int HV, int d_k, int d_v, const int *cu,
                         const int *heads, int n_heads, int n_threads, const fuse_t *f)
 {
     if (!q || !k || !v || !log_alpha || !b || !w || !o) return -1;
-    if (B <= 0 || T < 0 || H <= 0 || d_k <= 0 || d_v <= 0) return -1;
+    if (B <= 0 || T < 0 || H <= 0 || HV <= 0 || d_k <= 0 || d_v <= 0) return -1;
+    if (HV % H != 0) return -1;
     if (f->gate && !f->weight) return -1;
     if (f->prep && !(f->l2_eps >= 0.0)) return -1;
-    const long nh = heads ? n_heads : (long)B * H;
+    if (cu) {
+        if (cu[0] != 0 || cu[B] != T) return -1;
+        for (int n = 0; n < B; ++n)
+            if (cu[n + 1] < cu[n]) return -1;
+    }
+    const long G = HV / H;
+    const long nh = heads ? n_heads : (long)B * HV;
     if (nh < 0) return -1;
+    /* output row offset of each requested head: sequences are concatenated */
+    long *orow = (long *)malloc(sizeof(long) * (size_t)(nh > 0 ? nh : 1));
+    if (!orow) return -1;
+    long acc = 0;
+    for (long n = 0; n < nh; ++n) {
+        const long bh = heads ? heads[n] : n;
+        const long bi = (bh >= 0 && bh < (long)B * HV) ? bh / HV : 0;
+        orow[n] = acc;
+        acc += cu ? (long)(cu[bi + 1] - cu[bi]) : (long)T;
+    }
     int bad = 0;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);
@@ -175,17 +199,19 @@ static int forward_impl(const float *q, const float *k, const float *v,
 #endif
     for (long n = 0; n < nh; ++n) {
         const long bh = heads ? heads[n] : n;
-        if (bh < 0 || bh >= (long)B * H) { bad |= 1; continue; }
-        const long bi = bh / H, hi = bh % H;
-        const long tok0 = bi * (long)T * H + hi;      /* (b, t=0, h) row */
-        const long off_k = tok0 * d_k, off_v = tok0 * d_v;
+        if (bh < 0 || bh >= (long)B * HV) { bad |= 1; continue; }
+        const long bi = bh / HV, hv = bh % HV, hk = hv / G;
+        const long t0 = cu ? (long)cu[bi] : bi * (long)T;   /* first token of the sequence */
+        const long len = cu ? (long)(cu[bi + 1] - cu[bi]) : (long)T;
+        const long off_k = (t0 * H + hk) * d_k, off_v = (t0 * HV + hv) * d_v;
         bad |= run_head(q + off_k, k + off_k, v + off_v, log_alpha + off_k,
                         b + off_k, w + off_v, f->gate ? f->gate + off_v : NULL,
                         S0 ? S0 + bh * (long)d_k * d_v : NULL,
-                        o + n * (long)T * d_v,
+                        o + orow[n] * d_v,
                         S_T ? S_T + n * (long)d_k * d_v : NULL,
-                        smax ? smax + n : NULL, T, H, d_k, d_v, f) != 0;
+                        smax ? smax + n : NULL, len, H, HV, d_k, d_v, f) != 0;
     }
+    free(orow);
     return bad ? -1 : 0;
 }
 
@@ -196,7 +222,7 @@ int gdn2_oracle_forward(const float *q, const float *k, const float *v,
                         const int *heads, int n_heads, int n_threads)
 {
     const fuse_t f = {0, 0, 0.0, NULL, NULL, 0.0};
-    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, d_k, d_v,
+    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, H, d_k, d_v, NULL,
                         heads, n_heads, n_threads, &f);
 }
 
@@ -206,14 +232,14 @@ int gdn2_oracle_forward(const float *q, const float *k, const float *v,
 int gdn2_oracle_forward_ex(const float *q, const float *k, const float *v,
                            const float *log_alpha, const float *b, const float *w,
                            const double *S0, double *o, double *S_T, double *smax,
-                           int B, int T, int H, int d_k, int d_v,
+                           int B, int T, int H, int HV, int d_k, int d_v, const int *cu_seqlens,
                            const int *heads, int n_heads, int n_threads,
                            int prep, double l2_eps, const float *gate, const double *weight,
                            double norm_eps)
 {
     if (prep != 0 && prep != 1 && prep != 3) return -1;
     const fuse_t f = {prep & 1, (prep >> 1) & 1, l2_eps, gate, weight, norm_eps};
-    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, d_k, d_v,
+    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, HV, d_k, d_v, cu_seqlens,
                         heads, n_heads, n_threads, &f);
 }
 
