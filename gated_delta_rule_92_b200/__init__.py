@@ -7,9 +7,14 @@ library has not been built this module raises on first use.
 
     chunk_fwd(q, k, v, log_alpha, b, w, S0=None) -> (o, S_T)
     decode_step(q, k, v, log_alpha, b, w, S)     -> o      (S updated in place)
+    chunk_fwd_ex / decode_step_ex                 -- the same with value heads,
+        packed sequences (cu_seqlens, chunk only) and the fused input prep and
+        gated RMS-norm output epilogue
 
 Token tensors are [B, T, H, d] (decode: [B, H, d]) in bfloat16 or float32,
-contiguous, on one CUDA device; states are float32 [B, H, d_k, d_v].
+contiguous, on one CUDA device; states are float32 [B, HV, d_k, d_v].  q, k,
+log_alpha, b carry the H key heads, v, w, o, gate the HV value heads
+(HV = H unless the _ex calls are given more value heads).
 """
 from __future__ import annotations
 
@@ -58,9 +63,11 @@ def lib() -> ctypes.CDLL:
         L.gdn2_decode_step.restype = I
         F = ctypes.c_float
         fuse_args = [I, F, P, P, F]
-        L.gdn2_chunk_fwd_ex.argtypes = chunk_args[:-1] + fuse_args + [P]
+        # (..., B, T, H, HV, d_k, d_v, chunk, io, cu_seqlens, flags, l2_eps, gate, weight, eps, stream)
+        L.gdn2_chunk_fwd_ex.argtypes = [P] * 9 + [I] * 8 + [P] + fuse_args + [P]
         L.gdn2_chunk_fwd_ex.restype = I
-        L.gdn2_decode_step_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I] + fuse_args + [P]
+        # (..., B, H, HV, d_k, d_v, io, flags, l2_eps, gate, weight, eps, stream)
+        L.gdn2_decode_step_ex.argtypes = [P] * 8 + [I] * 6 + fuse_args + [P]
         L.gdn2_decode_step_ex.restype = I
         L.gdn2_device_status.argtypes = [P]
         L.gdn2_device_status.restype = I
@@ -132,28 +139,46 @@ def _fuse_args(q, prep, allow_neg_eigval, l2_eps, gate, norm_weight, norm_eps, g
             _ptr(norm_weight) if gate is not None else None, ctypes.c_float(float(norm_eps))]
 
 
-def _chunk(fn_name, q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state, fuse=None):
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
+def _chunk(fn_name, q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state, fuse=None,
+           cu_seqlens=None, ex=False):
+    Bt, T, H, dk = q.shape
+    HV, dv = v.shape[2], v.shape[3]
     dev = q.device
     _check_tokens((q, k, v, log_alpha, b, w), q.dtype, dev)
     for t in (k, log_alpha, b):
-        if tuple(t.shape) != (B, T, H, dk):
+        if tuple(t.shape) != (Bt, T, H, dk):
             raise ValueError("q, k, log_alpha, b must be [B, T, H, d_k]")
-    if tuple(w.shape) != (B, T, H, dv):
-        raise ValueError("v, w must be [B, T, H, d_v]")
-    _check_state(S0, (B, H, dk, dv), dev)
+    if tuple(v.shape[:2]) != (Bt, T) or tuple(w.shape) != (Bt, T, HV, dv):
+        raise ValueError("v, w must be [B, T, HV, d_v]")
+    if HV != H and not ex:
+        raise ValueError(f"{fn_name} takes H value heads; use chunk_fwd_ex for num_v_heads != H")
+    if HV % H != 0:
+        raise ValueError("the number of value heads must be a multiple of the key heads")
+    B = Bt
+    if cu_seqlens is not None:
+        if Bt != 1:
+            raise ValueError("with cu_seqlens the token tensors are [1, T_total, heads, d]")
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2 \
+                or cu_seqlens.device != dev or not cu_seqlens.is_contiguous():
+            raise ValueError("cu_seqlens must be a contiguous int32 [B + 1] tensor on the device")
+        B = cu_seqlens.numel() - 1
+    _check_state(S0, (B, HV, dk, dv), dev)
     if o is None:
-        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+        o = torch.empty((Bt, T, HV, dv), dtype=q.dtype, device=dev)
     if S_T is None and want_state:
-        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+        S_T = torch.empty((B, HV, dk, dv), dtype=torch.float32, device=dev)
     _check_tokens((o,), q.dtype, dev)
-    _check_state(S_T, (B, H, dk, dv), dev)
+    if tuple(o.shape) != (Bt, T, HV, dv):
+        raise ValueError(f"o must be {(Bt, T, HV, dv)}")
+    _check_state(S_T, (B, HV, dk, dv), dev)
     with torch.cuda.device(dev):
-        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
-                _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk), _io(q.dtype)]
-        if fuse is not None:
-            args += fuse(q, (B, T, H, dv))
+        if ex:
+            args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0), _ptr(o),
+                    _ptr(S_T), B, T, H, HV, dk, dv, int(chunk), _io(q.dtype), _ptr(cu_seqlens)]
+            args += fuse(q, (Bt, T, HV, dv))
+        else:
+            args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                    _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk), _io(q.dtype)]
         st = getattr(lib(), fn_name)(*args, _stream(stream))
     if st != 0:
         raise Gdn2Error(st, fn_name)
@@ -166,16 +191,26 @@ def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int
     return _chunk("gdn2_chunk_fwd", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state)
 
 
-def chunk_fwd_ex(q, k, v, log_alpha, b, w, S0=None, *, prep: bool = False, allow_neg_eigval: bool = False,
-                 l2_eps: float = 1e-6, gate=None, norm_weight=None, norm_eps: float = 1e-5,
-                 o=None, S_T=None, chunk: int = 64, stream=None, want_state: bool = True):
-    """Chunk forward with the fused input prep (prep=True: raw q, k, b, w) and,
-    with gate [B,T,H,d_v] and norm_weight [d_v] fp32, the gated RMS-norm output
-    epilogue.  Returns (o or y, S_T)."""
+def chunk_fwd_ex(q, k, v, log_alpha, b, w, S0=None, *, cu_seqlens=None, prep: bool = False,
+                 allow_neg_eigval: bool = False, l2_eps: float = 1e-6, gate=None, norm_weight=None,
+                 norm_eps: float = 1e-5, o=None, S_T=None, chunk: int = 64, stream=None,
+                 want_state: bool = True):
+    """Chunk forward, generalised and fused:
+
+    * value heads: v, w (and gate, o) may carry HV = G * H heads; value head hv
+      reads key head hv // G.  States are [B, HV, d_k, d_v].
+    * cu_seqlens: int32 [B + 1] device offsets of B sequences packed along T;
+      token tensors are then [1, T_total, heads, d].
+    * prep=True: q, k, b, w are raw (L2-normalised / sigmoid in the kernel);
+      allow_neg_eigval doubles b.
+    * gate [.., HV, d_v] with norm_weight [d_v] fp32: the gated RMS-norm output
+      epilogue.
+
+    Returns (o or y, S_T)."""
     fuse = lambda q_, shape: _fuse_args(q_, prep, allow_neg_eigval, l2_eps, gate, norm_weight,
                                         norm_eps, shape)
     return _chunk("gdn2_chunk_fwd_ex", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream,
-                  want_state, fuse)
+                  want_state, fuse, cu_seqlens=cu_seqlens, ex=True)
 
 
 def chunk_fwd_cuda_core(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int = 64,
@@ -185,19 +220,33 @@ def chunk_fwd_cuda_core(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, 
                   want_state)
 
 
-def _decode(fn_name, q, k, v, log_alpha, b, w, S, o, stream, fuse=None):
+def _decode(fn_name, q, k, v, log_alpha, b, w, S, o, stream, fuse=None, ex=False):
     B, H, dk = q.shape
-    dv = v.shape[-1]
+    HV, dv = v.shape[1], v.shape[2]
     dev = q.device
     _check_tokens((q, k, v, log_alpha, b, w), q.dtype, dev)
-    _check_state(S, (B, H, dk, dv), dev)
+    for t in (k, log_alpha, b):
+        if tuple(t.shape) != (B, H, dk):
+            raise ValueError("q, k, log_alpha, b must be [B, H, d_k]")
+    if v.shape[0] != B or tuple(w.shape) != (B, HV, dv):
+        raise ValueError("v, w must be [B, HV, d_v]")
+    if HV != H and not ex:
+        raise ValueError(f"{fn_name} takes H value heads; use decode_step_ex for num_v_heads != H")
+    if HV % H != 0:
+        raise ValueError("the number of value heads must be a multiple of the key heads")
+    _check_state(S, (B, HV, dk, dv), dev)
     if o is None:
-        o = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
+        o = torch.empty((B, HV, dv), dtype=q.dtype, device=dev)
+    _check_tokens((o,), q.dtype, dev)
+    if tuple(o.shape) != (B, HV, dv):
+        raise ValueError(f"o must be {(B, HV, dv)}")
     with torch.cuda.device(dev):
-        args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
-                _ptr(S), _ptr(o), B, H, dk, dv, _io(q.dtype)]
-        if fuse is not None:
-            args += fuse(q, (B, H, dv))
+        if ex:
+            args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                    _ptr(S), _ptr(o), B, H, HV, dk, dv, _io(q.dtype)] + fuse(q, (B, HV, dv))
+        else:
+            args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                    _ptr(S), _ptr(o), B, H, dk, dv, _io(q.dtype)]
         st = getattr(lib(), fn_name)(*args, _stream(stream))
     if st != 0:
         raise Gdn2Error(st, fn_name)
@@ -212,11 +261,12 @@ def decode_step(q, k, v, log_alpha, b, w, S, *, o=None, stream=None):
 def decode_step_ex(q, k, v, log_alpha, b, w, S, *, prep: bool = False, allow_neg_eigval: bool = False,
                    l2_eps: float = 1e-6, gate=None, norm_weight=None, norm_eps: float = 1e-5,
                    o=None, stream=None):
-    """Decode step with the fused input prep and (gate [B,H,d_v], norm_weight [d_v])
-    the gated RMS-norm output epilogue."""
+    """Decode step with value heads (v, w, gate [B,HV,d_v], S [B,HV,d_k,d_v]), the
+    fused input prep and (gate, norm_weight [d_v]) the gated RMS-norm output
+    epilogue."""
     fuse = lambda q_, shape: _fuse_args(q_, prep, allow_neg_eigval, l2_eps, gate, norm_weight,
                                         norm_eps, shape)
-    return _decode("gdn2_decode_step_ex", q, k, v, log_alpha, b, w, S, o, stream, fuse)
+    return _decode("gdn2_decode_step_ex", q, k, v, log_alpha, b, w, S, o, stream, fuse, ex=True)
 
 
 def device_status(stream=None) -> int:

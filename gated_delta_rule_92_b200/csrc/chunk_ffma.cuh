@@ -52,7 +52,8 @@ __global__ void __launch_bounds__(256, 1)
 chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                       const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ wg,
                       const float *__restrict__ S0, IO *__restrict__ o, float *__restrict__ S_T,
-                      int T, int H, int d_v, const FuseArgs fz = {}) {
+                      int T, int H, int HV, int d_v, const int *__restrict__ cu_seqlens,
+                      const FuseArgs fz = {}) {
     const bool prep = FUSED && fz.prep;
     const float bscale = (FUSED && fz.neg_eigval) ? 2.f : 1.f;
     using Cfg = FfmaCfg<DK>;
@@ -64,9 +65,23 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     float *sGC = sm + Cfg::O_GC;
 
     const int tid = threadIdx.x;
-    const int j0 = blockIdx.x * NV, h = blockIdx.y, bb = blockIdx.z;
-    const long head = (long)bb * H + h;
-    const int NC = (T + C - 1) / C;   // the last chunk may be partial (padded rows are zeros)
+    // value head hv (of HV) reads key head h = hv / (HV / H); sequence bb is
+    // tokens [tok_base, tok_base + len): bb * T + [0, T), or [cu[bb], cu[bb+1])
+    const int j0 = blockIdx.x * NV, hv = blockIdx.y, bb = blockIdx.z;
+    const int h = hv / (HV / H);
+    long tok_base = (long)bb * T;
+    int len = T;
+    if (cu_seqlens != nullptr) {
+        const int a = cu_seqlens[bb], e = cu_seqlens[bb + 1];
+        if (a < 0 || e < a || e > T) {   // malformed packing: this sequence is skipped
+            if (threadIdx.x == 0) record_status(kStatusBadArgs);
+            return;
+        }
+        tok_base = a;
+        len = e - a;
+    }
+    const long head = (long)bb * HV + hv;
+    const int NC = (len + C - 1) / C;   // the last chunk may be partial (padded rows are zeros)
 
     // initial state slice
     for (int idx = tid; idx < DK * NV; idx += 256) {
@@ -75,8 +90,8 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     }
 
     for (int n = 0; n < NC; ++n) {
-        const long tok0 = (long)bb * T + (long)n * C;   // token row of local r = 0
-        const int rows = min(C, T - n * C);              // valid rows of this chunk
+        const long tok0 = tok_base + (long)n * C;   // token row of local r = 0
+        const int rows = min(C, len - n * C);        // valid rows of this chunk
         __syncthreads();
         // ---- load the chunk (fp32 in shared memory); rows past T are zeros,
         // which leaves the recurrence unchanged (k = q = b = w = 0, no decay)
@@ -91,7 +106,7 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
         }
         for (int idx = tid; idx < C * NV; idx += 256) {
             const int r = idx / NV, j = idx % NV;
-            const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
+            const long g = ((tok0 + r) * HV + hv) * d_v + j0 + j;
             const float wv = (r < rows) ? ld_io(wg + g) : 0.f;
             sWV[r * LC + j] = (r < rows) ? (prep ? sigmoid_f32(wv) : wv) * ld_io(v + g) : 0.f;
         }
@@ -193,7 +208,7 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
             float x = 0.f;
             for (int c = 0; c < DK; ++c) x = fmaf(sQ[r * LK + c], sS[c * LC + j], x);
             for (int i = 0; i <= r; ++i) x = fmaf(sP[r * LC + i], sU[i * LC + j], x);
-            const long g = ((tok0 + r) * H + h) * d_v + j0 + j;
+            const long g = ((tok0 + r) * HV + hv) * d_v + j0 + j;
             if (r < rows) {
                 if constexpr (sizeof(IO) == 4) o[g] = x;
                 else o[g] = __float2bfloat16_rn(x);

@@ -217,18 +217,19 @@ __device__ __forceinline__ float ex2(float x) {
 
 // log_alpha of one chunk for the prep thread g (channel quad p = g % (DK/4),
 // rows R hb .. R hb + R - 1 with hb = g / (DK/4)), straight from HBM into
-// registers; rows past T read as zero (no decay on padding).
+// registers; rows past the sequence end read as zero (no decay on padding).
 template <int DK>
 struct PrepLA {
     static constexpr int NP = DK / 4, NB = 128 / NP, R = 64 / NB;
     uint2 v[R];
-    __device__ __forceinline__ void load(const __nv_bfloat16 *la, int bb, int n, int h, int T, int H, int g) {
+    // chunk n of the sequence made of tokens [tok0, tok0 + len); key head h of H
+    __device__ __forceinline__ void load(const __nv_bfloat16 *la, long tok0, int n, int h, int len, int H, int g) {
         const int p = g % NP, hb = g / NP;
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int r = n * 64 + hb * R + i;
-            v[i] = r < T ? __ldg(reinterpret_cast<const uint2 *>(la + (((long)bb * T + r) * H + h) * DK + 4 * p))
-                         : make_uint2(0u, 0u);
+            v[i] = r < len ? __ldg(reinterpret_cast<const uint2 *>(la + ((tok0 + r) * H + h) * DK + 4 * p))
+                           : make_uint2(0u, 0u);
         }
     }
 };
@@ -246,16 +247,31 @@ struct PrepLA {
 // 1 / sqrt(sum^2 + l2_eps) (a pre-pass: thread t sums row t % 64 of q (t < 64)
 // or of k, and leaves the factor in `nrm`) and b becomes sigmoid(b) (x2 with
 // neg_eigval).
-template <int DK, bool PREP = false>
+// Rows at or past `rows_valid` (the end of a packed sequence inside the
+// chunk) hold the next sequence's tokens: they are cleared in the raw q, b, k
+// tiles first, which makes them the same exact no-ops as padding.  This runs
+// only on a sequence's partial last chunk and leaves the loop below as is.
+template <int DK, bool PREP = false, bool VARLEN = false>
 __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLA<DK> &law,
                                            float *gc, float *carry, int g, int bar, const FuseArgs &fz = {},
-                                           float2 *nrm = nullptr) {
+                                           float2 *nrm = nullptr, int rows_valid = 64) {
     constexpr int NP = PrepLA<DK>::NP, NB = PrepLA<DK>::NB, R = PrepLA<DK>::R;
     static_assert(NB * R == 64 && NB <= 8, "prep split");
     const int p = g % NP, hb = g / NP;
     const int kb = p >> 4, cb = (p & 15) * 8;   // channel block, byte in the 128-byte row
     uint8_t *q_t = smem + oqe + kb * 16384, *e_t = q_t + 8192, *k_t = smem + okt + kb * 8192;
     auto off = [&](int r) { return r * 128 + ((((cb >> 4) ^ r) & 7) << 4) + (cb & 15); };
+    if (VARLEN && rows_valid < 64) {   // uniform over the 128 threads
+        // a swizzled row keeps its own 128 bytes: clear bytes [128 rows_valid, 8192)
+        // of each 8 KB q, b and k sub-tile
+        const int n16 = (64 - rows_valid) * 8;
+        for (int idx = g; idx < 3 * (DK / 64) * n16; idx += 128) {
+            const int tile = idx / n16, piece = idx - tile * n16, kb2 = tile / 3, which = tile - kb2 * 3;
+            uint8_t *base = (which == 2) ? smem + okt + kb2 * 8192 : smem + oqe + kb2 * 16384 + which * 8192;
+            *reinterpret_cast<uint4 *>(base + rows_valid * 128 + piece * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        named_bar(bar, 128);
+    }
     if constexpr (PREP) {   // 1 / |row| of q (threads 0-63) and k (64-127)
         const int r = g & 63;
         const uint8_t *base = (g < 64) ? smem + oqe : smem + okt;
@@ -361,14 +377,14 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
 
 // PREP fuses the input prep (raw q, k, b, w); EPI the gated RMS norm of each
 // output row before it is stored (d_v == NV: one CTA holds the whole row).
-template <int DK, int NV, bool PREP = false, bool EPI = false>
+template <int DK, int NV, bool PREP = false, bool EPI = false, bool VARLEN = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16 *__restrict__ la,
                     const float *__restrict__ S0,
-                    __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int T, int H, int d_v,
-                    unsigned long long wait_ns, const FuseArgs fz) {
+                    __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int T, int H, int HV, int d_v,
+                    const int *__restrict__ cu_seqlens, unsigned long long wait_ns, const FuseArgs fz) {
     static_assert(!EPI || NV <= 128, "epilogue weight slice");
     using Cfg = TcCfg<DK, NV>;
     extern __shared__ uint8_t smem_raw[];
@@ -377,9 +393,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t sb = smem_u32(smem);
 
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int j0 = blockIdx.x * NV, h = blockIdx.y, bb = blockIdx.z;
-    const int NC = (T + Cfg::C - 1) / Cfg::C;   // the last chunk may be partial
-    const long head = (long)bb * H + h;
+    // CTA: value head hv (of HV) reading key head h = hv / (HV / H), sequence bb.
+    // A sequence is tokens [tok0, tok0 + len): bb * T + [0, T) for equal-length
+    // batches, [cu[bb], cu[bb + 1]) when packed (the TMA maps then have one
+    // "batch" of all tokens: coordinates (c, head, tok0 + 64 n, 0)).
+    const int j0 = blockIdx.x * NV, hv = blockIdx.y, bb = blockIdx.z;
+    const int h = hv / (HV / H);
+    long tok0 = (long)bb * T;
+    int len = T, tma_t0 = 0, tma_b = bb;
+    if constexpr (VARLEN) {
+        const int a = cu_seqlens[bb], e = cu_seqlens[bb + 1];
+        if (a < 0 || e < a || e > T) {   // malformed packing: this sequence is skipped
+            if (threadIdx.x == 0) record_status(kStatusBadArgs);
+            return;
+        }
+        tok0 = a;
+        len = e - a;
+        tma_t0 = a;
+        tma_b = 0;
+    }
+    const int NC = (len + Cfg::C - 1) / Cfg::C;   // the last chunk may be partial
+    const long head = (long)bb * HV + hv;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *qb_full = bars + 0;     // [2] TMA q, b of a chunk landed (stage m % 2)
@@ -434,15 +468,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // padded tokens exact no-ops of the recurrence (k = q = b = w = 0 and
             // log_alpha = 0).
             auto prefetch = [&](int n) {
-                const int r = n * 64;
+                const int r = tma_t0 + n * 64;
                 for (int kb = 0; kb < DK / 64; ++kb) {
-                    tma_prefetch_l2_4d(&tm_q, kb * 64, h, r, bb);
-                    tma_prefetch_l2_4d(&tm_k, kb * 64, h, r, bb);
-                    tma_prefetch_l2_4d(&tm_b, kb * 64, h, r, bb);
+                    tma_prefetch_l2_4d(&tm_q, kb * 64, h, r, tma_b);
+                    tma_prefetch_l2_4d(&tm_k, kb * 64, h, r, tma_b);
+                    tma_prefetch_l2_4d(&tm_b, kb * 64, h, r, tma_b);
                 }
                 for (int vb = 0; vb < Cfg::VB; ++vb) {
-                    tma_prefetch_l2_4d(&tm_v, j0 + vb * 64, h, r, bb);
-                    tma_prefetch_l2_4d(&tm_w, j0 + vb * 64, h, r, bb);
+                    tma_prefetch_l2_4d(&tm_v, j0 + vb * 64, hv, r, tma_b);
+                    tma_prefetch_l2_4d(&tm_w, j0 + vb * 64, hv, r, tma_b);
                 }
             };
             for (int p = 0; p < Cfg::PREFETCH && p < NC; ++p) prefetch(p);
@@ -451,38 +485,38 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             while (nq < NC || nk < NC || nw < NC || nv < NC) {
                 bool progress = false;
                 if (nq < NC && (nq < 2 || mbar_test_wait(&empty_qe[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
-                    const int s = nq & 1, r = nq * 64;
+                    const int s = nq & 1, r = tma_t0 + nq * 64;
                     const uint32_t oqe = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0;
                     mbar_arrive_expect_tx(&qb_full[s], 2u * Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb) {
-                        tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qb_full[s], kb * 64, h, r, bb);
-                        tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qb_full[s], kb * 64, h, r, bb);
+                        tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qb_full[s], kb * 64, h, r, tma_b);
+                        tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qb_full[s], kb * 64, h, r, tma_b);
                     }
                     if (nq + Cfg::PREFETCH < NC) prefetch(nq + Cfg::PREFETCH);
                     ++nq;
                     progress = true;
                 }
                 if (nk < NC && (nk < 3 || mbar_test_wait(&empty_k[nk % 3], static_cast<uint32_t>((nk / 3 - 1) & 1)))) {
-                    const int s3 = nk % 3, r = nk * 64;
+                    const int s3 = nk % 3, r = tma_t0 + nk * 64;
                     mbar_arrive_expect_tx(&k_full[s3], Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_4d(smem + Cfg::OFF_K + s3 * 16384 + kb * 8192, &tm_k, &k_full[s3], kb * 64, h, r, bb);
+                        tma_load_4d(smem + Cfg::OFF_K + s3 * 16384 + kb * 8192, &tm_k, &k_full[s3], kb * 64, h, r, tma_b);
                     ++nk;
                     progress = true;
                 }
                 if (nw < NC && (nw < 1 || mbar_test_wait(w_free, static_cast<uint32_t>((nw - 1) & 1)))) {
-                    const int r = nw * 64;
+                    const int r = tma_t0 + nw * 64;
                     mbar_arrive_expect_tx(w_full, Cfg::VAL_TILE);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_load_4d(smem + Cfg::OFF_W + vb * 8192, &tm_w, w_full, j0 + vb * 64, h, r, bb);
+                        tma_load_4d(smem + Cfg::OFF_W + vb * 8192, &tm_w, w_full, j0 + vb * 64, hv, r, tma_b);
                     ++nw;
                     progress = true;
                 }
                 if (nv < NC && (nv < 1 || mbar_test_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
-                    const int r = nv * 64;
+                    const int r = tma_t0 + nv * 64;
                     mbar_arrive_expect_tx(v_full, Cfg::VAL_TILE);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_load_4d(smem + Cfg::OFF_V + vb * 8192, &tm_v, v_full, j0 + vb * 64, h, r, bb);
+                        tma_load_4d(smem + Cfg::OFF_V + vb * 8192, &tm_v, v_full, j0 + vb * 64, hv, r, tma_b);
                     ++nv;
                     progress = true;
                 }
@@ -504,11 +538,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         PrepLA<DK> lan;   // group B: log_alpha of the next chunk to prepare
         // prologue: prep of chunk 0 (group B)
         if (NC > 0) {
-            if (grp_b) lan.load(la, bb, 0, h, T, H, t - 128);
+            if (grp_b) lan.load(la, tok0, 0, h, len, H, t - 128);
             bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK, PREP>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, fz, nrm);
+            else if (grp_b) prep_chunk<DK, PREP, VARLEN>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, fz, nrm,
+                                                 min(64, len));
         }
         for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
@@ -518,7 +553,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // barriers that close the previous iteration
             if (m == 0) named_bar(1, kKeyThreads);
             // log_alpha of chunk m+1, a whole iteration ahead of its use
-            if (grp_b && m + 1 < NC) lan.load(la, bb, m + 1, h, T, H, t - 128);
+            if (grp_b && m + 1 < NC) lan.load(la, tok0, m + 1, h, len, H, t - 128);
             // ---------------------------------------------------------- MMA1
             if (t == 0) {
                 tc_fence_after();
@@ -554,6 +589,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     } else {
                         r4 = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));
                     }
+                    // packed: the rows after the sequence end hold the next sequence's tokens
+                    if (VARLEN && ((off & 8191u) >> 7) >= static_cast<uint32_t>(len - m * 64))
+                        r4 = make_uint4(0u, 0u, 0u, 0u);
                     st_shared_v4(sb + Cfg::OFF_V + off, r4.x, r4.y, r4.z, r4.w);
                 }
             }
@@ -611,8 +649,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = ok_b && mbar_wait(&k_full[s3n], static_cast<uint32_t>(((m + 1) / 3) & 1), wait_ns);
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
-                    prep_chunk<DK, PREP>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
-                                         gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm);
+                    prep_chunk<DK, PREP, VARLEN>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
+                                         gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm,
+                                         min(64, len - (m + 1) * 64));
             }
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
@@ -713,6 +752,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
                 tmem_st32(t_S + lane_q + jc * 32, sv);
+                if (NC == 0 && S_T != nullptr && c < DK) {   // empty sequence: S_T = S0
+                    float4 *dst = reinterpret_cast<float4 *>(S_T + (head * DK + c) * d_v + j0 + jc * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(sv[4 * e], sv[4 * e + 1], sv[4 * e + 2], sv[4 * e + 3]);
+                }
                 const uint32_t tile = sb + Cfg::OFF_S + ((jc * 32) >> 6) * 16384u;
                 const uint32_t ch0 = ((jc * 32) & 63) >> 3;
 #pragma unroll
@@ -731,9 +776,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int s = n & 1;
             if constexpr (EPI) {   // the epilogue's gate tile, into L2 a whole chain pass ahead
                 const int r = t >> 1;   // two threads per row: 2 x 128-byte lines of the NV slice
-                if (n * 64 + r < T && (t & 1) * 64 < NV)
+                if (n * 64 + r < len && (t & 1) * 64 < NV)
                     prefetch_l2(static_cast<const __nv_bfloat16 *>(fz.gate) +
-                                (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0 + (t & 1) * 64);
+                                ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + (t & 1) * 64);
             }
             const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = Cfg::OFF_K + (n % 3) * 16384u;
             const uint32_t OP = s ? Cfg::OFF_P1 : Cfg::OFF_P0;
@@ -842,8 +887,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_after();
             if ((warp & 3) < 2) {
                 const int r = t;   // output row r (TMEM lanes 0-63); rows past T are padding
-                const bool valid = n * 64 + r < T;
-                const long orow_off = (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0;
+                const bool valid = n * 64 + r < len;
+                const long orow_off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0;
                 __nv_bfloat16 *orow = o + orow_off;
                 bool plain = true;
                 if constexpr (EPI) {   // first half of the epilogue: o / rms(o) -> bf16 in the U tile
@@ -902,16 +947,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int i = 0; i < 64 / RPP; ++i) {
                     const int r = i * RPP + rr;
-                    gall[i] = (n * 64 + r < T)
+                    gall[i] = (n * 64 + r < len)
                                   ? __ldg(reinterpret_cast<const uint4 *>(
-                                        gbase + (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0 + 8 * c16))
+                                        gbase + ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * c16))
                                   : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
                 for (int i = 0; i < 64 / RPP; ++i) {
                     const int r = i * RPP + rr;
-                    if (n * 64 + r >= T) continue;   // padding rows
-                    const long off = (((long)bb * T + (long)n * 64 + r) * H + h) * (long)d_v + j0 + 8 * c16;
+                    if (n * 64 + r >= len) continue;   // padding rows
+                    const long off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * c16;
                     const uint4 gv = gall[i];
                     uint32_t a0, a1, a2, a3;
                     ld_shared_v4(sb + Cfg::OFF_U + (c16 >> 3) * 8192u + sw128_chunk(r, c16 & 7), a0, a1, a2, a3);

@@ -10,8 +10,9 @@
 //     o_j  = p_j + (q . k) u_j                  = q^T S_t
 // so S is read once and written once; everything else is a few KB.
 //
-// Layout: one block of 256 threads per (head, 64- or 128-column slice of
-// d_v).  A row of the slice is NVD floats: NVD/4 threads each own a float4
+// Layout: one block of 256 threads per (value head, 64- or 128-column slice
+// of d_v); with HV = G H value heads (num_v_heads), value head hv reads key
+// head hv / G.  A row of the slice is NVD floats: NVD/4 threads each own a float4
 // column group, the remaining thread rows each own DK / (256 / (NVD/4)) rows.
 // Every thread issues all its 128-bit loads of S before any arithmetic, so a
 // block keeps 32-64 KB of HBM reads in flight.  Column sums over d_k are
@@ -71,7 +72,7 @@ template <typename IO, int DK, int NVD, bool FUSED = false>
 __global__ void __launch_bounds__(256, 2)
 decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                    const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ wg,
-                   float *__restrict__ S, IO *__restrict__ o, int d_v, FuseArgs fz = {}) {
+                   float *__restrict__ S, IO *__restrict__ o, int d_v, int H, int HV, FuseArgs fz = {}) {
     constexpr int TPR = NVD / 4;   // threads across one row of the slice
     constexpr int RG = 256 / TPR;  // thread rows
     constexpr int RPT = DK / RG;   // state rows per thread
@@ -88,7 +89,10 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     const int tid = threadIdx.x;
     const int cg = tid % TPR;        // float4 column group
     const int rg = tid / TPR;        // thread row
-    const long bh = blockIdx.x;      // flat b * H + h
+    const int bhi = blockIdx.x;      // flat b * HV + hv (value head; state, v, w, o); B HV <= INT_MAX
+    const long bh = bhi;
+    // its key head (q, k, log_alpha, b)
+    const long bk = (HV == H) ? bh : (long)((bhi / HV) * H + (bhi % HV) / (HV / H));
     const int j0 = blockIdx.y * NVD;
 
     float *Sh = S + bh * (long)DK * d_v + j0 + cg * 4;
@@ -100,7 +104,7 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     }
 
     // per-row and per-column coefficients
-    const IO *qh = q + bh * DK, *kh = k + bh * DK, *lah = la + bh * DK, *bh_ = bg + bh * DK;
+    const IO *qh = q + bk * DK, *kh = k + bk * DK, *lah = la + bk * DK, *bh_ = bg + bk * DK;
     float qk = 0.f;
     float kv = 0.f, qv = 0.f, bv = 0.f;
     if (tid < DK) {

@@ -12,12 +12,14 @@
 
 namespace gdn2 {
 
-// Status word written by kernels when a bounded wait gives up (one per
-// device; read and cleared by gdn2_device_status()).  The library is a
+// Status word written by kernels when a bounded wait gives up or device-side
+// arguments are malformed (one per device; read and cleared by
+// gdn2_device_status()).  The library is a
 // single translation unit, so the definition lives here.
 __device__ int g_device_status = 0;
 
 constexpr int kStatusTimeout = 5;   // == GDN2_ERR_DEVICE_TIMEOUT
+constexpr int kStatusBadArgs = 1;   // == GDN2_ERR_INVALID_ARG (e.g. malformed cu_seqlens)
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -29,9 +31,8 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-__device__ __forceinline__ void record_timeout() {
-    atomicExch(&g_device_status, kStatusTimeout);
-}
+__device__ __forceinline__ void record_status(int code) { atomicExch(&g_device_status, code); }
+__device__ __forceinline__ void record_timeout() { record_status(kStatusTimeout); }
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

@@ -72,6 +72,15 @@ bool make_token_map(CUtensorMap *m, const void *base, int B, int T, int H, int d
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Problem shape shared by the launchers: B sequences of T tokens, or, with
+// cu_seqlens, B sequences packed along T tokens; H key heads, HV value heads.
+struct Shape {
+    int B, T, H, HV, d_k, d_v;
+    const int *cu;      // device [B + 1] or null
+    int tensor_b() const { return cu ? 1 : B; }   // leading dim of the token tensors
+    long rows() const { return (long)tensor_b() * T * HV; }   // (token, value head) rows of o
+};
+
 template <typename IO>
 gdn2_status_t launch_rmsnorm(void *o, const void *g, const float *weight, long rows, int d_v, float eps,
                              cudaStream_t st) {
@@ -81,50 +90,61 @@ gdn2_status_t launch_rmsnorm(void *o, const void *g, const float *weight, long r
     return from_cuda(cudaGetLastError());
 }
 
-template <int DK, int NV, bool PREP, bool EPI>
+template <int DK, int NV, bool PREP, bool EPI, bool VARLEN>
 gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
-                               const CUtensorMap &tv, const CUtensorMap &tw, const void *la, const float *S0, void *o, float *S_T, int B, int T, int H,
-                               int d_v, cudaStream_t st, const FuseArgs &fz) {
+                               const CUtensorMap &tv, const CUtensorMap &tw, const void *la, const float *S0,
+                               void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz) {
     using Cfg = TcCfg<DK, NV>;
-    auto kern = chunk_fwd_tc_kernel<DK, NV, PREP, EPI>;
+    auto kern = chunk_fwd_tc_kernel<DK, NV, PREP, EPI, VARLEN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    dim3 grid(d_v / NV, H, B);
+    dim3 grid(sh.d_v / NV, sh.HV, sh.B);
     kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, static_cast<const __nv_bfloat16 *>(la),
-                                                    S0, static_cast<__nv_bfloat16 *>(o), S_T, T, H, d_v, kWaitNs,
-                                                    fz);
+                                                    S0, static_cast<__nv_bfloat16 *>(o), S_T, sh.T, sh.H, sh.HV,
+                                                    sh.d_v, sh.cu, kWaitNs, fz);
     return from_cuda(cudaGetLastError());
+}
+
+// Packed sequences take the kernel built with the per-sequence offsets; the
+// equal-length one has none of that code.
+template <int DK, int NV, bool PREP, bool EPI>
+gdn2_status_t launch_tc_seq(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
+                            const CUtensorMap &tv, const CUtensorMap &tw, const void *la, const float *S0,
+                            void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz) {
+    if (sh.cu) return launch_tc_kernel<DK, NV, PREP, EPI, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, fz);
+    return launch_tc_kernel<DK, NV, PREP, EPI, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, fz);
 }
 
 template <int DK, int NV>
 gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void *la, const void *b, const void *w,
-                        const float *S0, void *o, float *S_T, int B, int T, int H, int d_v, cudaStream_t st,
+                        const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
                         const FuseArgs *fz = nullptr) {
     CUtensorMap tq, tk, tb, tv, tw;
-    if (!make_token_map(&tq, q, B, T, H, DK) || !make_token_map(&tk, k, B, T, H, DK) ||
-        !make_token_map(&tb, b, B, T, H, DK) || !make_token_map(&tv, v, B, T, H, d_v) ||
-        !make_token_map(&tw, w, B, T, H, d_v))
+    const int Bt = sh.tensor_b();
+    if (!make_token_map(&tq, q, Bt, sh.T, sh.H, DK) || !make_token_map(&tk, k, Bt, sh.T, sh.H, DK) ||
+        !make_token_map(&tb, b, Bt, sh.T, sh.H, DK) || !make_token_map(&tv, v, Bt, sh.T, sh.HV, sh.d_v) ||
+        !make_token_map(&tw, w, Bt, sh.T, sh.HV, sh.d_v))
         return GDN2_ERR_CUDA;
     const bool prep = fz != nullptr && fz->prep;
     // the in-kernel epilogue needs the whole d_v row in one CTA; otherwise one
     // more pass normalises o in place
-    const bool epi = fz != nullptr && fz->gate != nullptr && d_v == NV;
+    const bool epi = fz != nullptr && fz->gate != nullptr && sh.d_v == NV;
     const FuseArgs kf = fz ? *fz : FuseArgs{};
     gdn2_status_t s;
-    if (prep && epi) s = launch_tc_kernel<DK, NV, true, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
-    else if (prep) s = launch_tc_kernel<DK, NV, true, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
-    else if (epi) s = launch_tc_kernel<DK, NV, false, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
-    else s = launch_tc_kernel<DK, NV, false, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, B, T, H, d_v, st, kf);
+    if (prep && epi) s = launch_tc_seq<DK, NV, true, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
+    else if (prep) s = launch_tc_seq<DK, NV, true, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
+    else if (epi) s = launch_tc_seq<DK, NV, false, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
+    else s = launch_tc_seq<DK, NV, false, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
     if (s != GDN2_OK || fz == nullptr || fz->gate == nullptr || epi) return s;
-    return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, (long)B * T * H, d_v, fz->norm_eps, st);
+    return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, sh.rows(), sh.d_v, fz->norm_eps, st);
 }
 
 template <typename IO, int DK>
 gdn2_status_t launch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
-                          const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_v,
-                          cudaStream_t st, const FuseArgs *fz = nullptr) {
+                          const void *w, const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
+                          const FuseArgs *fz = nullptr) {
     using Cfg = FfmaCfg<DK>;
-    dim3 grid(d_v / Cfg::NV, H, B);
+    dim3 grid(sh.d_v / Cfg::NV, sh.HV, sh.B);
     const IO *qp = static_cast<const IO *>(q), *kp = static_cast<const IO *>(k), *vp = static_cast<const IO *>(v);
     const IO *lp = static_cast<const IO *>(la), *bp = static_cast<const IO *>(b), *wp = static_cast<const IO *>(w);
     IO *op = static_cast<IO *>(o);
@@ -132,28 +152,29 @@ gdn2_status_t launch_ffma(const void *q, const void *k, const void *v, const voi
         auto kern = chunk_fwd_ffma_kernel<IO, DK>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
         if (e != cudaSuccess) return GDN2_ERR_CUDA;
-        kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, T, H, d_v, FuseArgs{});
+        kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, sh.T, sh.H, sh.HV, sh.d_v, sh.cu,
+                                            FuseArgs{});
         return from_cuda(cudaGetLastError());
     }
     auto kern = chunk_fwd_ffma_kernel<IO, DK, true>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
-    kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, T, H, d_v, *fz);
+    kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, sh.T, sh.H, sh.HV, sh.d_v, sh.cu, *fz);
     gdn2_status_t s = from_cuda(cudaGetLastError());
     if (s != GDN2_OK || fz->gate == nullptr) return s;
-    return launch_rmsnorm<IO>(o, fz->gate, fz->norm_weight, (long)B * T * H, d_v, fz->norm_eps, st);
+    return launch_rmsnorm<IO>(o, fz->gate, fz->norm_weight, sh.rows(), sh.d_v, fz->norm_eps, st);
 }
 
 template <typename IO, int DK, int NVD>
 gdn2_status_t launch_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
-                            const void *w, float *S, void *o, int B, int H, int d_v, cudaStream_t st,
+                            const void *w, float *S, void *o, int B, int H, int HV, int d_v, cudaStream_t st,
                             const FuseArgs *fz) {
-    dim3 grid((unsigned)((long)B * H), d_v / NVD);
+    dim3 grid((unsigned)((long)B * HV), d_v / NVD);
     if (fz == nullptr) {
         decode_step_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
             static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
             static_cast<const IO *>(la), static_cast<const IO *>(b), static_cast<const IO *>(w), S,
-            static_cast<IO *>(o), d_v, FuseArgs{});
+            static_cast<IO *>(o), d_v, H, HV, FuseArgs{});
         return from_cuda(cudaGetLastError());
     }
     // fused: the d_v / NVD blocks of one head form a cluster along y when the
@@ -172,7 +193,7 @@ gdn2_status_t launch_decode(const void *q, const void *k, const void *v, const v
     return from_cuda(cudaLaunchKernelEx(&cfg, decode_step_kernel<IO, DK, NVD, true>, static_cast<const IO *>(q),
                                         static_cast<const IO *>(k), static_cast<const IO *>(v),
                                         static_cast<const IO *>(la), static_cast<const IO *>(b),
-                                        static_cast<const IO *>(w), S, static_cast<IO *>(o), d_v, *fz));
+                                        static_cast<const IO *>(w), S, static_cast<IO *>(o), d_v, H, HV, *fz));
 }
 
 // Checks the fusion arguments of the _ex entry points and fills `fz`.
@@ -194,51 +215,54 @@ gdn2_status_t check_fuse(int flags, float l2_eps, const void *gate, const float 
 
 // Shared validation of the chunk entry points.
 gdn2_status_t check_chunk(const void *q, const void *k, const void *v, const void *la, const void *b,
-                          const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
-                          int d_v, int chunk, gdn2_io_t io) {
+                          const void *w, const float *S0, void *o, float *S_T, const Shape &sh, int chunk,
+                          gdn2_io_t io) {
+    const int B = sh.B, T = sh.T, H = sh.H, HV = sh.HV, d_k = sh.d_k, d_v = sh.d_v;
     // With T = 0 the token tensors are empty and may be null.
     if (T > 0 && (!q || !k || !v || !la || !b || !w || !o)) return GDN2_ERR_INVALID_ARG;
-    if (B <= 0 || H <= 0 || T < 0 || d_k <= 0 || d_v <= 0 || chunk <= 0) return GDN2_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || HV <= 0 || T < 0 || d_k <= 0 || d_v <= 0 || chunk <= 0) return GDN2_ERR_INVALID_ARG;
+    if (HV % H != 0) return GDN2_ERR_INVALID_ARG;
     if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
     const void *ptrs[9] = {q, k, v, la, b, w, S0, o, S_T};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN2_ERR_MISALIGNED;
+    if (sh.cu && (reinterpret_cast<uintptr_t>(sh.cu) & 3u)) return GDN2_ERR_MISALIGNED;
     if (chunk != 64) return GDN2_ERR_UNSUPPORTED;
     if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
     if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
-    if ((long)B * T > INT_MAX || B > 65535 || H > 65535) return GDN2_ERR_UNSUPPORTED;
+    if ((long)sh.tensor_b() * T > INT_MAX || B > 65535 || HV > 65535) return GDN2_ERR_UNSUPPORTED;
     return GDN2_OK;
 }
 
-// T = 0: no tokens; the final state is the initial state.
-gdn2_status_t empty_sequence(const float *S0, float *S_T, int B, int H, int d_k, int d_v, cudaStream_t st) {
+// No tokens at all: every final state is its initial state.
+gdn2_status_t empty_sequence(const float *S0, float *S_T, const Shape &sh, cudaStream_t st) {
     if (!S_T) return GDN2_OK;
-    const size_t bytes = sizeof(float) * (size_t)B * H * d_k * d_v;
+    const size_t bytes = sizeof(float) * (size_t)sh.B * sh.HV * sh.d_k * sh.d_v;
     if (!S0) return from_cuda(cudaMemsetAsync(S_T, 0, bytes, st));
     if (S0 == S_T) return GDN2_OK;
     return from_cuda(cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st));
 }
 
 gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
-                            const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
-                            int d_v, gdn2_io_t io, cudaStream_t st, const FuseArgs *fz = nullptr) {
+                            const void *w, const float *S0, void *o, float *S_T, const Shape &sh, gdn2_io_t io,
+                            cudaStream_t st, const FuseArgs *fz = nullptr) {
     if (io == GDN2_IO_F32) {
-        if (d_k == 64) return launch_ffma<float, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
-        return launch_ffma<float, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+        if (sh.d_k == 64) return launch_ffma<float, 64>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
+        return launch_ffma<float, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
     }
-    if (d_k == 64) return launch_ffma<__nv_bfloat16, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
-    return launch_ffma<__nv_bfloat16, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+    if (sh.d_k == 64) return launch_ffma<__nv_bfloat16, 64>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
+    return launch_ffma<__nv_bfloat16, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
 }
 
 gdn2_status_t dispatch_tc(const void *q, const void *k, const void *v, const void *la, const void *b,
-                          const void *w, const float *S0, void *o, float *S_T, int B, int T, int H, int d_k,
-                          int d_v, cudaStream_t st, const FuseArgs *fz = nullptr) {
-    const bool wide = (d_v % 128 == 0);
-    if (d_k == 64)
-        return wide ? launch_tc<64, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz)
-                    : launch_tc<64, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
-    return wide ? launch_tc<128, 128>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz)
-                : launch_tc<128, 64>(q, k, v, la, b, w, S0, o, S_T, B, T, H, d_v, st, fz);
+                          const void *w, const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
+                          const FuseArgs *fz = nullptr) {
+    const bool wide = (sh.d_v % 128 == 0);
+    if (sh.d_k == 64)
+        return wide ? launch_tc<64, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz)
+                    : launch_tc<64, 64>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
+    return wide ? launch_tc<128, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz)
+                : launch_tc<128, 64>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
 }
 
 }  // namespace
@@ -249,62 +273,65 @@ using namespace gdn2;
 extern "C" gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
                                         const void *b, const void *w, const float *S0, void *o, float *S_T, int B,
                                         int T, int H, int d_k, int d_v, int chunk, gdn2_io_t io, void *stream) {
-    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, io);
+    const Shape sh{B, T, H, H, d_k, d_v, nullptr};
+    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io);
     if (s != GDN2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
-    if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st);
-    return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, st);
+    if (T == 0) return empty_sequence(S0, S_T, sh, st);
+    if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, io, st);
+    return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, sh, st);
 }
 
 extern "C" gdn2_status_t gdn2_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *log_alpha,
                                            const void *b, const void *w, const float *S0, void *o, float *S_T,
-                                           int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io_t io,
-                                           int flags, float l2_eps, const void *gate, const float *norm_weight,
-                                           float norm_eps, void *stream) {
+                                           int B, int T, int H, int HV, int d_k, int d_v, int chunk, gdn2_io_t io,
+                                           const int *cu_seqlens, int flags, float l2_eps, const void *gate,
+                                           const float *norm_weight, float norm_eps, void *stream) {
     FuseArgs fz;
     gdn2_status_t s = check_fuse(flags, l2_eps, gate, norm_weight, norm_eps, &fz);
     if (s != GDN2_OK) return s;
-    s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, io);
+    const Shape sh{B, T, H, HV != 0 ? HV : H, d_k, d_v, cu_seqlens};
+    s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io);
     if (s != GDN2_OK) return s;
-    if (T > 0 && gate == nullptr && norm_weight != nullptr) return GDN2_ERR_INVALID_ARG;
+    if (gate == nullptr && norm_weight != nullptr) return GDN2_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
-    if (io == GDN2_IO_F32)
-        return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st, &fz);
-    return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, st, &fz);
+    if (T == 0) return empty_sequence(S0, S_T, sh, st);
+    if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, io, st, &fz);
+    return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, sh, st, &fz);
 }
 
 extern "C" gdn2_status_t gdn2_chunk_fwd_cuda_core(const void *q, const void *k, const void *v,
                                                   const void *log_alpha, const void *b, const void *w,
                                                   const float *S0, void *o, float *S_T, int B, int T, int H,
                                                   int d_k, int d_v, int chunk, gdn2_io_t io, void *stream) {
-    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, chunk, io);
+    const Shape sh{B, T, H, H, d_k, d_v, nullptr};
+    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io);
     if (s != GDN2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (T == 0) return empty_sequence(S0, S_T, B, H, d_k, d_v, st);
-    return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, d_k, d_v, io, st);
+    if (T == 0) return empty_sequence(S0, S_T, sh, st);
+    return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, io, st);
 }
 
 namespace gdn2 {
 namespace {
 gdn2_status_t decode_impl(const void *q, const void *k, const void *v, const void *log_alpha, const void *b,
-                          const void *w, float *S, void *o, int B, int H, int d_k, int d_v, gdn2_io_t io,
+                          const void *w, float *S, void *o, int B, int H, int HV, int d_k, int d_v, gdn2_io_t io,
                           void *stream, const FuseArgs *fz) {
     if (!q || !k || !v || !log_alpha || !b || !w || !S || !o) return GDN2_ERR_INVALID_ARG;
-    if (B <= 0 || H <= 0 || d_k <= 0 || d_v <= 0) return GDN2_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || HV <= 0 || d_k <= 0 || d_v <= 0) return GDN2_ERR_INVALID_ARG;
+    if (HV % H != 0) return GDN2_ERR_INVALID_ARG;
     if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
     const void *ptrs[8] = {q, k, v, log_alpha, b, w, S, o};
     for (const void *p : ptrs)
         if (!aligned16(p)) return GDN2_ERR_MISALIGNED;
     if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
     if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
-    if ((long)B * H > INT_MAX) return GDN2_ERR_UNSUPPORTED;
+    if ((long)B * HV > INT_MAX) return GDN2_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool wide = (d_v % 128 == 0);
 #define GDN2_DECODE(IO, DK)                                                                            \
-    return wide ? launch_decode<IO, DK, 128>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st, fz)         \
-                : launch_decode<IO, DK, 64>(q, k, v, log_alpha, b, w, S, o, B, H, d_v, st, fz)
+    return wide ? launch_decode<IO, DK, 128>(q, k, v, log_alpha, b, w, S, o, B, H, HV, d_v, st, fz)     \
+                : launch_decode<IO, DK, 64>(q, k, v, log_alpha, b, w, S, o, B, H, HV, d_v, st, fz)
     if (io == GDN2_IO_F32) {
         if (d_k == 64) GDN2_DECODE(float, 64);
         GDN2_DECODE(float, 128);
@@ -319,18 +346,19 @@ gdn2_status_t decode_impl(const void *q, const void *k, const void *v, const voi
 extern "C" gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v, const void *log_alpha,
                                           const void *b, const void *w, float *S, void *o, int B, int H, int d_k,
                                           int d_v, gdn2_io_t io, void *stream) {
-    return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, d_k, d_v, io, stream, nullptr);
+    return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, H, d_k, d_v, io, stream, nullptr);
 }
 
 extern "C" gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v, const void *log_alpha,
                                              const void *b, const void *w, float *S, void *o, int B, int H,
-                                             int d_k, int d_v, gdn2_io_t io, int flags, float l2_eps,
+                                             int HV, int d_k, int d_v, gdn2_io_t io, int flags, float l2_eps,
                                              const void *gate, const float *norm_weight, float norm_eps,
                                              void *stream) {
     FuseArgs fz;
     const gdn2_status_t s = check_fuse(flags, l2_eps, gate, norm_weight, norm_eps, &fz);
     if (s != GDN2_OK) return s;
-    return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, d_k, d_v, io, stream, &fz);
+    if (gate == nullptr && norm_weight != nullptr) return GDN2_ERR_INVALID_ARG;
+    return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, HV != 0 ? HV : H, d_k, d_v, io, stream, &fz);
 }
 
 extern "C" gdn2_status_t gdn2_device_status(void *stream) {

@@ -142,44 +142,75 @@ gdn2_status_t gdn2_decode_step(const void *q, const void *k, const void *v,
 
 /*
  * gdn2_chunk_fwd_ex / gdn2_decode_step_ex -- gdn2_chunk_fwd and
- * gdn2_decode_step with the steps the README's "Architecture" diagram draws
- * around the mixer fused into the same pass:
+ * gdn2_decode_step generalised in two directions, with the steps the
+ * README's "Architecture" diagram draws around the mixer fused into the same
+ * pass.
  *
+ * Value heads (README "Configuration": num_v_heads):
+ *   HV           : number of value heads; 0 means HV = H.  HV must be a
+ *                  multiple of H.  Value head hv reads key head
+ *                  hv / (HV / H): q, k, log_alpha and b keep H heads, while
+ *                  v, w, o, gate and the states carry HV heads:
+ *                      v, w, o, gate : [B, T, HV, d_v]
+ *                      S0, S_T, S    : [B, HV, d_k, d_v]
+ *
+ * Packed variable-length sequences (chunk only):
+ *   cu_seqlens   : NULL, or a DEVICE int32 array [B + 1] of token offsets,
+ *                  cu_seqlens[0] = 0 <= cu_seqlens[1] <= ... <= cu_seqlens[B]
+ *                  = T, 4-byte aligned.  The B sequences are then packed one
+ *                  after another along T (T = total tokens): every token
+ *                  tensor has a leading dimension of 1 ([1, T, H, d_k],
+ *                  [1, T, HV, d_v]) and sequence i is tokens
+ *                  [cu_seqlens[i], cu_seqlens[i+1]), with its own state
+ *                  S0[i] -> S_T[i].  Each sequence is processed exactly as
+ *                  a separate call would (its last chunk may be partial;
+ *                  an empty sequence has S_T[i] = S0[i]).  The offsets are
+ *                  read on the device: a sequence whose offsets are out of
+ *                  order or outside [0, T] is skipped (its o rows and S_T
+ *                  slice are not written) and GDN2_ERR_INVALID_ARG is
+ *                  recorded in the status word that gdn2_device_status()
+ *                  returns.
+ *
+ * Fusion:
  *   flags        : 0 or GDN2_FUSE_INPUT_PREP [| GDN2_FUSE_NEG_EIGVAL].  With
  *                  INPUT_PREP the kernels read raw q, k, b, w and apply the
  *                  maps above while loading them; the recurrence is then the
  *                  one documented for gdn2_chunk_fwd on the prepared values.
- *                  l2_eps (>= 0) is only read with INPUT_PREP.
- *   gate         : NULL, or the output gate g [B, T, H, d_v] (decode:
- *                  [B, H, d_v]), dtype io.  Non-NULL switches the output
- *                  epilogue ("Gated RMS Norm <- SiLU Gate") on: per (token,
- *                  head) the stored output is
+ *                  l2_eps (>= 0) is only read with INPUT_PREP.  A zero q or
+ *                  k row stays zero for any l2_eps.
+ *   gate         : NULL, or the output gate g, laid out as o, dtype io.
+ *                  Non-NULL switches the output epilogue ("Gated RMS Norm <-
+ *                  SiLU Gate") on: per (token, value head) the stored output
+ *                  is
  *                      y_j = o_j / sqrt(mean_j o_j^2 + norm_eps) * norm_weight_j * silu(g_j)
  *                  with silu(x) = x sigmoid(x), instead of o.
  *   norm_weight  : float32 [d_v], one weight vector shared by all heads;
- *                  required with gate, 16-byte aligned.
+ *                  required with gate (and only with it), 16-byte aligned.
  *   norm_eps     : >= 0 (the README default is 1e-5).
  *
  * The epilogue is applied before o is stored whenever one CTA holds a whole
  * d_v row (tensor-core chunk kernel: d_v = 64 or 128; decode: any d_v, the
  * CTAs of one head forming a thread-block cluster); otherwise (tensor-core
  * chunk kernel with d_v > 128, CUDA-core chunk kernel) o is normalised in
- * place by one more pass in the same stream.  With flags = 0 and gate = NULL
- * these calls are gdn2_chunk_fwd and gdn2_decode_step.  Other arguments,
- * shapes and errors as there; bad flags, a gate without norm_weight or a
- * negative epsilon return GDN2_ERR_INVALID_ARG.
+ * place by one more pass in the same stream.  With HV = H (or 0),
+ * cu_seqlens = NULL, flags = 0 and gate = NULL these calls are
+ * gdn2_chunk_fwd and gdn2_decode_step.  Other arguments, shapes and errors
+ * as there; bad flags, a gate without norm_weight (or a weight without a
+ * gate), a negative epsilon or HV not a multiple of H return
+ * GDN2_ERR_INVALID_ARG.
  */
 gdn2_status_t gdn2_chunk_fwd_ex(const void *q, const void *k, const void *v,
                                 const void *log_alpha, const void *b, const void *w,
                                 const float *S0, void *o, float *S_T,
-                                int B, int T, int H, int d_k, int d_v, int chunk,
-                                gdn2_io_t io, int flags, float l2_eps,
+                                int B, int T, int H, int HV, int d_k, int d_v, int chunk,
+                                gdn2_io_t io, const int *cu_seqlens,
+                                int flags, float l2_eps,
                                 const void *gate, const float *norm_weight, float norm_eps,
                                 void *stream);
 
 gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v,
                                   const void *log_alpha, const void *b, const void *w,
-                                  float *S, void *o, int B, int H, int d_k, int d_v,
+                                  float *S, void *o, int B, int H, int HV, int d_k, int d_v,
                                   gdn2_io_t io, int flags, float l2_eps,
                                   const void *gate, const float *norm_weight, float norm_eps,
                                   void *stream);
@@ -187,7 +218,9 @@ gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v,
 /*
  * gdn2_device_status -- synchronise `stream`, then read and clear the
  * current device's status word.  Returns GDN2_OK, GDN2_ERR_DEVICE_TIMEOUT if
- * a kernel gave up on a bounded wait since the last call, or GDN2_ERR_CUDA.
+ * a kernel gave up on a bounded wait since the last call,
+ * GDN2_ERR_INVALID_ARG if a kernel skipped a sequence with malformed
+ * cu_seqlens offsets, or GDN2_ERR_CUDA.
  */
 gdn2_status_t gdn2_device_status(void *stream);
 

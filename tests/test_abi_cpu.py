@@ -96,11 +96,11 @@ def test_fused_argument_validation_on_host(L):
     p, w = P(16), P(32)
 
     def chunk_ex(flags=0, l2=1e-6, gate=None, weight=None, eps=1e-5, T=64):
-        return L.gdn2_chunk_fwd_ex(p, p, p, p, p, p, None, p, None, 1, T, 1, 64, 64, 64, 1,
+        return L.gdn2_chunk_fwd_ex(p, p, p, p, p, p, None, p, None, 1, T, 1, 1, 64, 64, 64, 1, None,
                                    flags, F(l2), gate, weight, F(eps), None)
 
     def decode_ex(flags=0, l2=1e-6, gate=None, weight=None, eps=1e-5):
-        return L.gdn2_decode_step_ex(p, p, p, p, p, p, p, p, 1, 1, 64, 64, 1,
+        return L.gdn2_decode_step_ex(p, p, p, p, p, p, p, p, 1, 1, 1, 64, 64, 1,
                                      flags, F(l2), gate, weight, F(eps), None)
 
     for call in (chunk_ex, decode_ex):
@@ -113,3 +113,26 @@ def test_fused_argument_validation_on_host(L):
         assert call(gate=p, weight=P(20)) == 3        # misaligned weight
     assert chunk_ex(flags=3, T=0, gate=p, weight=w) == 0   # empty sequence: nothing to do
     assert chunk_ex(weight=w) == 1                         # weight without gate
+
+
+def test_value_heads_and_packing_validation_on_host(L):
+    """HV must be a multiple of H; cu_seqlens must be 4-byte aligned; HV = 0 means H."""
+    P, F = ctypes.c_void_p, ctypes.c_float
+    p = P(16)
+
+    def chunk_ex(H=2, HV=4, cu=None, T=64, B=1):
+        return L.gdn2_chunk_fwd_ex(p, p, p, p, p, p, None, p, None, B, T, H, HV, 64, 64, 64, 1, cu,
+                                   0, F(1e-6), None, None, F(1e-5), None)
+
+    def decode_ex(H=2, HV=4, B=1):
+        return L.gdn2_decode_step_ex(p, p, p, p, p, p, p, p, B, H, HV, 64, 64, 1,
+                                     0, F(1e-6), None, None, F(1e-5), None)
+
+    assert chunk_ex(HV=3) == 1            # not a multiple of H
+    assert chunk_ex(HV=-2) == 1
+    assert decode_ex(HV=3) == 1
+    assert decode_ex(HV=-1) == 1
+    assert chunk_ex(cu=P(18)) == 3        # misaligned offsets
+    assert chunk_ex(T=0, cu=P(16)) == 0   # no tokens at all, no state: nothing to do
+    assert chunk_ex(T=0, HV=0) == 0
+    assert chunk_ex(HV=70000, H=1) == 2   # beyond the grid's y extent

@@ -84,12 +84,13 @@ def _l2n(x: torch.Tensor) -> torch.Tensor:
 
 def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
          dtype=torch.bfloat16, alpha_lo: float = 0.9, alpha_hi: float = 0.999,
-         b_scale: float = 1.0, s0_std: Optional[float] = None,
+         b_scale: float = 1.0, s0_std: Optional[float] = None, HV: Optional[int] = None,
          generator: Optional[torch.Generator] = None, device="cpu") -> dict:
     """Draw one batch of token inputs [B, T, H, d].
 
-    Returns a dict with q, k, v, log_alpha, b, w in ``dtype`` and S0 (fp32
-    [B, H, d_k, d_v] or None).  With ``device="cuda"`` the draws are made by
+    Returns a dict with q, k, log_alpha, b [B, T, H, d_k] and v, w
+    [B, T, HV, d_v] in ``dtype`` (HV value heads, default H) and S0 (fp32
+    [B, HV, d_k, d_v] or None).  With ``device="cuda"`` the draws are made by
     a CUDA generator with the same seed and recipe (a different stream of
     numbers than the CPU generator; used where only the distribution matters,
     e.g. timing).
@@ -97,15 +98,16 @@ def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
     g = generator if generator is not None else torch.Generator(device=device).manual_seed(seed)
     f32 = torch.float32
     kw = dict(generator=g, dtype=f32, device=device)
+    HV = H if HV is None else HV
     q = _l2n(torch.randn(B, T, H, d_k, **kw))
     k = _l2n(torch.randn(B, T, H, d_k, **kw))
-    v = torch.randn(B, T, H, d_v, **kw)
+    v = torch.randn(B, T, HV, d_v, **kw)
     alpha = torch.empty(B, T, H, d_k, dtype=f32, device=device).uniform_(alpha_lo, alpha_hi, generator=g)
     b = b_scale * torch.sigmoid(torch.randn(B, T, H, d_k, **kw))
-    w = torch.sigmoid(torch.randn(B, T, H, d_v, **kw))
+    w = torch.sigmoid(torch.randn(B, T, HV, d_v, **kw))
     S0 = None
     if s0_std is not None:
-        S0 = s0_std * torch.randn(B, H, d_k, d_v, **kw)
+        S0 = s0_std * torch.randn(B, HV, d_k, d_v, **kw)
     out = dict(q=q, k=k, v=v, log_alpha=torch.log(alpha), b=b, w=w)
     out = {n: t.to(dtype).contiguous() for n, t in out.items()}
     out["S0"] = S0
@@ -115,7 +117,7 @@ def draw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
 def draw_raw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
              dtype=torch.bfloat16, alpha_lo: float = 0.9, alpha_hi: float = 0.999,
              qk_scale: float = 1.0, s0_std: Optional[float] = None, steps: Optional[int] = None,
-             generator: Optional[torch.Generator] = None, device="cpu") -> dict:
+             HV: Optional[int] = None, generator: Optional[torch.Generator] = None, device="cpu") -> dict:
     """Inputs for the fused input prep and output epilogue: the raw
     projections the layer would hand the mixer.
 
@@ -123,28 +125,48 @@ def draw_raw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
     v ~ N(0,1); alpha ~ U[alpha_lo, alpha_hi], log_alpha = ln alpha; the
     output gate g ~ N(0,1); the RMS-norm weight ~ U[0.5, 1.5] (synthetic, one
     [d_v] vector, fp32); S0 ~ N(0, s0_std) or None.  Token tensors are
-    [B, T, H, d], or [steps, B, H, d] for decode when ``steps`` is given.
+    [B, T, H, d], or [steps, B, H, d] for decode when ``steps`` is given;
+    v, w and g carry HV value heads (default H), S0 is [B, HV, d_k, d_v].
     """
     g = generator if generator is not None else torch.Generator(device=device).manual_seed(seed)
     f32 = torch.float32
     kw = dict(generator=g, dtype=f32, device=device)
+    HV = H if HV is None else HV
     lead = (steps, B, H) if steps is not None else (B, T, H)
+    vlead = lead[:-1] + (HV,)
     q = qk_scale * torch.randn(*lead, d_k, **kw)
     k = qk_scale * torch.randn(*lead, d_k, **kw)
-    v = torch.randn(*lead, d_v, **kw)
+    v = torch.randn(*vlead, d_v, **kw)
     alpha = torch.empty(*lead, d_k, dtype=f32, device=device).uniform_(alpha_lo, alpha_hi, generator=g)
     b = torch.randn(*lead, d_k, **kw)
-    w = torch.randn(*lead, d_v, **kw)
-    gate = torch.randn(*lead, d_v, **kw)
+    w = torch.randn(*vlead, d_v, **kw)
+    gate = torch.randn(*vlead, d_v, **kw)
     weight = torch.empty(d_v, dtype=f32, device=device).uniform_(0.5, 1.5, generator=g)
     S0 = None
     if s0_std is not None:
-        S0 = s0_std * torch.randn(B, H, d_k, d_v, **kw)
+        S0 = s0_std * torch.randn(B, HV, d_k, d_v, **kw)
     out = dict(q=q, k=k, v=v, log_alpha=torch.log(alpha), b=b, w=w, gate=gate)
     out = {n: t.to(dtype).contiguous() for n, t in out.items()}
     out["S0"] = S0
     out["norm_weight"] = weight
     return out
+
+
+def packed_lengths(n: int, mean: int, *, seed: int, min_len: int = 0) -> list:
+    """Lengths of ``n`` packed sequences: a geometric-like mix around ``mean``
+    tokens (exponential draw, rounded), at least ``min_len``.  Used for the
+    packed variable-length cases."""
+    g = torch.Generator().manual_seed(seed)
+    e = torch.empty(n, dtype=torch.float64).exponential_(1.0, generator=g)
+    return [max(min_len, int(round(float(x) * mean))) for x in e]
+
+
+def cu_seqlens_of(lengths) -> torch.Tensor:
+    """int32 [n + 1] offsets of sequences of the given lengths packed back to back."""
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    return torch.tensor(cu, dtype=torch.int32)
 
 
 def make_chunk_inputs(wl: Workload, *, B: Optional[int] = None, T: Optional[int] = None,
