@@ -1,7 +1,8 @@
 // chunk_ffma.cuh -- chunk-parallel GDN-2 forward on CUDA cores (fp32 products).
 //
 // The recurrence (burn-gdn2 README, "Architecture") regrouped over chunks of
-// C = 64 tokens ("Chunk WY (train)" mode of the README).  For one chunk with
+// C = 16, 32 or 64 tokens ("Chunk WY (train)" mode; "Configuration":
+// chunk_size, default 64).  For one chunk with
 // chunk-start state S (d_k x d_v), per key channel c and local row r:
 //     g_r   = sum_{s<=r} log_alpha_s           gamma_r = exp(g_r)
 //     Q~_r  = q_r . gamma_r     K~_i = k_i / gamma_i     E_r = b_r . k_r . gamma_r
@@ -16,19 +17,21 @@
 // kernel, which evaluates the same products on tcgen05 in a different order.
 //
 // One block of 256 threads per (b, h, 64-column slice of d_v); everything
-// for one chunk lives in shared memory (about 215 KB at d_k = 128).
+// for one chunk lives in shared memory (about 215 KB at d_k = 128, C = 64).
 #pragma once
 #include "decode.cuh"
 #include "gdn2_device.cuh"
 
 namespace gdn2 {
 
-template <int DK>
+template <int DK, int CH = 64>
 struct FfmaCfg {
-    static constexpr int C = 64;
+    static_assert(CH == 16 || CH == 32 || CH == 64, "chunk length");
+    static constexpr int C = CH;
     static constexpr int NV = 64;
-    static constexpr int LK = DK + 1;   // padded row stride for [64][DK] tiles
-    static constexpr int LC = C + 1;    // padded row stride for [.][64] tiles
+    static constexpr int LK = DK + 1;   // padded row stride for [C][DK] tiles
+    static constexpr int LC = C + 1;    // padded row stride for [C][C] tiles (A, P, T)
+    static constexpr int LV = NV + 1;   // padded row stride for [.][NV] tiles (W.V, U, S)
     // float offsets
     static constexpr int O_Q = 0;
     static constexpr int O_K = O_Q + C * LK;
@@ -37,9 +40,9 @@ struct FfmaCfg {
     static constexpr int G_SIZE = (C * LK > 2 * C * LC) ? C * LK : 2 * C * LC;
     static constexpr int O_T = O_G + G_SIZE;
     static constexpr int O_WV = O_T + C * LC;           // W.V, then E S
-    static constexpr int O_U = O_WV + C * LC;           // T (W.V), then U
-    static constexpr int O_S = O_U + C * LC;            // state slice [DK][NV]
-    static constexpr int O_GC = O_S + DK * LC;
+    static constexpr int O_U = O_WV + C * LV;           // T (W.V), then U
+    static constexpr int O_S = O_U + C * LV;            // state slice [DK][NV]
+    static constexpr int O_GC = O_S + DK * LV;
     static constexpr int FLOATS = O_GC + DK;
     static constexpr size_t BYTES = sizeof(float) * FLOATS;
 };
@@ -47,7 +50,7 @@ struct FfmaCfg {
 // FUSED with fz.prep reads raw q, k, b, w: rows of q and k are L2-normalised
 // over d_k (x / sqrt(sum x^2 + l2_eps)), b = sigmoid(b) (x2 with neg_eigval),
 // w = sigmoid(w).  The output epilogue of this path runs as a separate pass.
-template <typename IO, int DK, bool FUSED = false>
+template <typename IO, int DK, bool FUSED = false, int CH = 64>
 __global__ void __launch_bounds__(256, 1)
 chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                       const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ wg,
@@ -56,8 +59,8 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
                       const FuseArgs fz = {}) {
     const bool prep = FUSED && fz.prep;
     const float bscale = (FUSED && fz.neg_eigval) ? 2.f : 1.f;
-    using Cfg = FfmaCfg<DK>;
-    constexpr int C = Cfg::C, NV = Cfg::NV, LK = Cfg::LK, LC = Cfg::LC;
+    using Cfg = FfmaCfg<DK, CH>;
+    constexpr int C = Cfg::C, NV = Cfg::NV, LK = Cfg::LK, LC = Cfg::LC, LV = Cfg::LV;
     extern __shared__ float sm[];
     float *sQ = sm + Cfg::O_Q, *sK = sm + Cfg::O_K, *sE = sm + Cfg::O_E, *sG = sm + Cfg::O_G;
     float *sA = sG, *sP = sG + C * LC;
@@ -86,7 +89,7 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     // initial state slice
     for (int idx = tid; idx < DK * NV; idx += 256) {
         const int c = idx / NV, j = idx % NV;
-        sS[c * LC + j] = S0 ? S0[(head * DK + c) * d_v + j0 + j] : 0.f;
+        sS[c * LV + j] = S0 ? S0[(head * DK + c) * d_v + j0 + j] : 0.f;
     }
 
     for (int n = 0; n < NC; ++n) {
@@ -108,7 +111,7 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
             const int r = idx / NV, j = idx % NV;
             const long g = ((tok0 + r) * HV + hv) * d_v + j0 + j;
             const float wv = (r < rows) ? ld_io(wg + g) : 0.f;
-            sWV[r * LC + j] = (r < rows) ? (prep ? sigmoid_f32(wv) : wv) * ld_io(v + g) : 0.f;
+            sWV[r * LV + j] = (r < rows) ? (prep ? sigmoid_f32(wv) : wv) * ld_io(v + g) : 0.f;
         }
         __syncthreads();
         if (prep) {   // L2-normalise each row of q and k: warp w takes rows w, w + 8, ...
@@ -177,37 +180,37 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
         for (int m = 0; m < C * NV / 256; ++m) {
             const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
             float x = 0.f;
-            for (int i = 0; i <= r; ++i) x = fmaf(sT[r * LC + i], sWV[i * LC + j], x);
+            for (int i = 0; i <= r; ++i) x = fmaf(sT[r * LC + i], sWV[i * LV + j], x);
             acc[m] = x;
         }
         __syncthreads();
         for (int m = 0; m < C * NV / 256; ++m) {
             const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            sU[r * LC + j] = acc[m];
+            sU[r * LV + j] = acc[m];
             float x = 0.f;
-            for (int c = 0; c < DK; ++c) x = fmaf(sE[r * LK + c], sS[c * LC + j], x);
-            sWV[r * LC + j] = x;
+            for (int c = 0; c < DK; ++c) x = fmaf(sE[r * LK + c], sS[c * LV + j], x);
+            sWV[r * LV + j] = x;
         }
         __syncthreads();
         // ---- U = T (W.V) - T (E S)
         for (int m = 0; m < C * NV / 256; ++m) {
             const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            float x = sU[r * LC + j];
-            for (int i = 0; i <= r; ++i) x = fmaf(-sT[r * LC + i], sWV[i * LC + j], x);
+            float x = sU[r * LV + j];
+            for (int i = 0; i <= r; ++i) x = fmaf(-sT[r * LC + i], sWV[i * LV + j], x);
             acc[m] = x;
         }
         __syncthreads();
         for (int m = 0; m < C * NV / 256; ++m) {
             const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            sU[r * LC + j] = acc[m];
+            sU[r * LV + j] = acc[m];
         }
         __syncthreads();
         // ---- O = Q~ S + P U
         for (int m = 0; m < C * NV / 256; ++m) {
             const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
             float x = 0.f;
-            for (int c = 0; c < DK; ++c) x = fmaf(sQ[r * LK + c], sS[c * LC + j], x);
-            for (int i = 0; i <= r; ++i) x = fmaf(sP[r * LC + i], sU[i * LC + j], x);
+            for (int c = 0; c < DK; ++c) x = fmaf(sQ[r * LK + c], sS[c * LV + j], x);
+            for (int i = 0; i <= r; ++i) x = fmaf(sP[r * LC + i], sU[i * LV + j], x);
             const long g = ((tok0 + r) * HV + hv) * d_v + j0 + j;
             if (r < rows) {
                 if constexpr (sizeof(IO) == 4) o[g] = x;
@@ -218,16 +221,16 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
         // ---- S <- diag(gamma_C) (S + K~^T U)
         for (int idx = tid; idx < DK * NV; idx += 256) {
             const int c = idx / NV, j = idx % NV;
-            float x = sS[c * LC + j];
-            for (int i = 0; i < C; ++i) x = fmaf(sK[i * LK + c], sU[i * LC + j], x);
-            sS[c * LC + j] = sGC[c] * x;
+            float x = sS[c * LV + j];
+            for (int i = 0; i < C; ++i) x = fmaf(sK[i * LK + c], sU[i * LV + j], x);
+            sS[c * LV + j] = sGC[c] * x;
         }
     }
     __syncthreads();
     if (S_T) {
         for (int idx = tid; idx < DK * NV; idx += 256) {
             const int c = idx / NV, j = idx % NV;
-            S_T[(head * DK + c) * d_v + j0 + j] = sS[c * LC + j];
+            S_T[(head * DK + c) * d_v + j0 + j] = sS[c * LV + j];
         }
     }
 }

@@ -139,24 +139,24 @@ gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void 
     return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, sh.rows(), sh.d_v, fz->norm_eps, st);
 }
 
-template <typename IO, int DK>
+template <typename IO, int DK, int CH>
 gdn2_status_t launch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
                           const void *w, const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
                           const FuseArgs *fz = nullptr) {
-    using Cfg = FfmaCfg<DK>;
+    using Cfg = FfmaCfg<DK, CH>;
     dim3 grid(sh.d_v / Cfg::NV, sh.HV, sh.B);
     const IO *qp = static_cast<const IO *>(q), *kp = static_cast<const IO *>(k), *vp = static_cast<const IO *>(v);
     const IO *lp = static_cast<const IO *>(la), *bp = static_cast<const IO *>(b), *wp = static_cast<const IO *>(w);
     IO *op = static_cast<IO *>(o);
     if (fz == nullptr) {
-        auto kern = chunk_fwd_ffma_kernel<IO, DK>;
+        auto kern = chunk_fwd_ffma_kernel<IO, DK, false, CH>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
         if (e != cudaSuccess) return GDN2_ERR_CUDA;
         kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, sh.T, sh.H, sh.HV, sh.d_v, sh.cu,
                                             FuseArgs{});
         return from_cuda(cudaGetLastError());
     }
-    auto kern = chunk_fwd_ffma_kernel<IO, DK, true>;
+    auto kern = chunk_fwd_ffma_kernel<IO, DK, true, CH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
     kern<<<grid, 256, Cfg::BYTES, st>>>(qp, kp, vp, lp, bp, wp, S0, op, S_T, sh.T, sh.H, sh.HV, sh.d_v, sh.cu, *fz);
@@ -227,7 +227,7 @@ gdn2_status_t check_chunk(const void *q, const void *k, const void *v, const voi
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return GDN2_ERR_MISALIGNED;
     if (sh.cu && (reinterpret_cast<uintptr_t>(sh.cu) & 3u)) return GDN2_ERR_MISALIGNED;
-    if (chunk != 64) return GDN2_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return GDN2_ERR_UNSUPPORTED;
     if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
     if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
     if ((long)sh.tensor_b() * T > INT_MAX || B > 65535 || HV > 65535) return GDN2_ERR_UNSUPPORTED;
@@ -243,15 +243,27 @@ gdn2_status_t empty_sequence(const float *S0, float *S_T, const Shape &sh, cudaS
     return from_cuda(cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st));
 }
 
-gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
-                            const void *w, const float *S0, void *o, float *S_T, const Shape &sh, gdn2_io_t io,
-                            cudaStream_t st, const FuseArgs *fz = nullptr) {
-    if (io == GDN2_IO_F32) {
-        if (sh.d_k == 64) return launch_ffma<float, 64>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
-        return launch_ffma<float, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
+template <typename IO>
+gdn2_status_t dispatch_ffma_io(const void *q, const void *k, const void *v, const void *la, const void *b,
+                               const void *w, const float *S0, void *o, float *S_T, const Shape &sh, int chunk,
+                               cudaStream_t st, const FuseArgs *fz) {
+#define GDN2_FFMA(DK, CH) return launch_ffma<IO, DK, CH>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz)
+    if (sh.d_k == 64) {
+        if (chunk == 16) GDN2_FFMA(64, 16);
+        if (chunk == 32) GDN2_FFMA(64, 32);
+        GDN2_FFMA(64, 64);
     }
-    if (sh.d_k == 64) return launch_ffma<__nv_bfloat16, 64>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
-    return launch_ffma<__nv_bfloat16, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz);
+    if (chunk == 16) GDN2_FFMA(128, 16);
+    if (chunk == 32) GDN2_FFMA(128, 32);
+    GDN2_FFMA(128, 64);
+#undef GDN2_FFMA
+}
+
+gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
+                            const void *w, const float *S0, void *o, float *S_T, const Shape &sh, int chunk,
+                            gdn2_io_t io, cudaStream_t st, const FuseArgs *fz = nullptr) {
+    if (io == GDN2_IO_F32) return dispatch_ffma_io<float>(q, k, v, la, b, w, S0, o, S_T, sh, chunk, st, fz);
+    return dispatch_ffma_io<__nv_bfloat16>(q, k, v, la, b, w, S0, o, S_T, sh, chunk, st, fz);
 }
 
 gdn2_status_t dispatch_tc(const void *q, const void *k, const void *v, const void *la, const void *b,
@@ -278,7 +290,7 @@ extern "C" gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void
     if (s != GDN2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) return empty_sequence(S0, S_T, sh, st);
-    if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, io, st);
+    if (io == GDN2_IO_F32 || chunk != 64) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io, st);
     return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, sh, st);
 }
 
@@ -296,7 +308,8 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_ex(const void *q, const void *k, const v
     if (gate == nullptr && norm_weight != nullptr) return GDN2_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) return empty_sequence(S0, S_T, sh, st);
-    if (io == GDN2_IO_F32) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, io, st, &fz);
+    if (io == GDN2_IO_F32 || chunk != 64)
+        return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io, st, &fz);
     return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, sh, st, &fz);
 }
 
@@ -309,7 +322,7 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_cuda_core(const void *q, const void *k, 
     if (s != GDN2_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) return empty_sequence(S0, S_T, sh, st);
-    return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, io, st);
+    return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io, st);
 }
 
 namespace gdn2 {

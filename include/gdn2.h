@@ -80,7 +80,9 @@ typedef enum {
  *   S_T                : out, [B, H, d_k, d_v] float32, or NULL (not written).
  *                        May alias S0 (each block reads its slice of S0
  *                        before it writes that slice of S_T).
- *   chunk              : chunk length; must be 64 (the README default).
+ *   chunk              : chunk length: 16, 32 or 64 (README "Configuration",
+ *                        chunk_size, default 64).  The result does not
+ *                        depend on it beyond rounding.
  *
  * Built shapes: d_k in {64, 128}; d_v a multiple of 64 with d_v <= 512;
  * any T >= 0.  A last chunk shorter than `chunk` is processed as if padded
@@ -89,9 +91,10 @@ typedef enum {
  * allowed: o is empty, token pointers may be NULL, and S_T = S0.
  * Other shapes return GDN2_ERR_UNSUPPORTED.
  *
- * Precision: bf16 I/O runs the tensor-core kernel (bf16 operands, fp32
- * accumulation, fp32 state carried between chunks); fp32 I/O runs the
- * CUDA-core kernel with fp32 products throughout.  o is rounded to the I/O
+ * Precision: bf16 I/O with chunk 64 runs the tensor-core kernel (bf16
+ * operands, fp32 accumulation, fp32 state carried between chunks); fp32 I/O,
+ * and bf16 I/O with chunk 16 or 32, run the CUDA-core kernel with fp32
+ * products throughout.  o is rounded to the I/O
  * dtype (round to nearest even); S_T is fp32.
  */
 gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v,

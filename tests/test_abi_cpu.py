@@ -62,7 +62,8 @@ def test_chunk_argument_validation_on_host(L):
     assert _chunk_call(L, io=7) == 1
     assert _chunk_call(L, ptr=24) == 3                   # misaligned
     assert _chunk_call(L, o=40) == 3
-    assert _chunk_call(L, chunk=32) == 2                 # only chunk 64 is built
+    assert _chunk_call(L, chunk=48) == 2                 # chunk 16, 32 and 64 are built
+    assert _chunk_call(L, chunk=128) == 2
     assert _chunk_call(L, dk=96) == 2
     assert _chunk_call(L, dv=96) == 2
     assert _chunk_call(L, dv=1024) == 2

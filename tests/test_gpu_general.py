@@ -207,3 +207,61 @@ def test_malformed_offsets_are_reported_not_read(g):
                             cu_seqlens=cu)
     assert g.device_status() == 1   # GDN2_ERR_INVALID_ARG recorded by the skipped sequence
     assert g.device_status() == 0   # and cleared by the read
+
+
+CHUNKS = [  # B, T, H, d_k, d_v, dtype
+    (1, 150, 2, 64, 64, torch.float32),
+    (2, 97, 2, 128, 128, torch.float32),
+    (1, 150, 2, 128, 128, torch.bfloat16),
+    (1, 77, 2, 64, 192, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("case", CHUNKS, ids=lambda c: f"B{c[0]}T{c[1]}H{c[2]}dk{c[3]}dv{c[4]}{str(c[5])[6:]}")
+@pytest.mark.parametrize("chunk", [16, 32], ids=lambda c: f"chunk{c}")
+def test_chunk_lengths(g, case, chunk):
+    """chunk_size 16 and 32 (CUDA-core kernel) against the oracle, which has no chunks."""
+    B, T, H, dk, dv, dt = case
+    inp = W.draw(B, T, H, dk, dv, seed=7000 + T + dk, dtype=dt, s0_std=0.05)
+    d = to_dev(inp)
+    o, S_T = g.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], chunk=chunk)
+    torch.cuda.synchronize()
+    assert g.device_status() == 0
+    ro, rS = oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"], S0=inp["S0"])
+    got = np.stack([o[x // H, :, x % H].float().cpu().numpy() for x in range(B * H)])
+    tol = TOL[dt]
+    eo = rel_inf(got, ro)
+    es = rel_inf(S_T.double().cpu().numpy().reshape(B * H, dk, dv), rS)
+    assert eo <= tol and es <= tol, f"o err {eo:.3e}, S_T err {es:.3e} (tol {tol})"
+
+
+def test_chunk_length_invariance_fp32(g):
+    """The chunk form is an exact regrouping: chunk 16, 32 and 64 agree to fp32 rounding."""
+    inp = W.draw(2, 300, 2, 128, 128, seed=7100, dtype=torch.float32, s0_std=0.05)
+    d = to_dev(inp)
+    outs = [g.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], chunk=c)
+            for c in (16, 32, 64)]
+    torch.cuda.synchronize()
+    o64, S64 = outs[-1]
+    for o, S in outs[:-1]:
+        assert float((o - o64).abs().max()) <= 2e-5 * float(o64.abs().max())
+        assert float((S - S64).abs().max()) <= 2e-5 * float(S64.abs().max())
+
+
+def test_chunk32_packed_value_heads_fused(g):
+    """chunk 32 with packed sequences, value heads, prep and epilogue together."""
+    lens = [33, 0, 96, 5]
+    cu = W.cu_seqlens_of(lens)
+    T, H, HV, dk, dv = int(cu[-1]), 2, 4, 128, 128
+    inp = _inputs(T, H, HV, dk, dv, torch.bfloat16, 7200, True)
+    inp["S0"] = 0.05 * torch.randn(len(lens), HV, dk, dv, generator=torch.Generator().manual_seed(7201))
+    d = to_dev(inp)
+    o, S_T = _run_ex(g, d, cu.cuda(), chunk=32, **_gpu_kw(d, True, True))
+    ro, rS = oracle.forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"],
+                            S0=inp["S0"], cu_seqlens=cu.numpy(), **_oracle_kw(inp, True, True))
+    got = [o[0, int(cu[x // HV]):int(cu[x // HV + 1]), x % HV].float().cpu().numpy()
+           for x in range(len(lens) * HV)]
+    scale = max(float(np.max(np.abs(r))) for r in ro if r.size)
+    eo = max(float(np.max(np.abs(a - r))) for a, r in zip(got, ro) if r.size) / scale
+    es = rel_inf(S_T.double().cpu().numpy().reshape(len(lens) * HV, dk, dv), rS)
+    assert eo <= 2e-2 and es <= 2e-2, f"o err {eo:.3e}, S_T err {es:.3e}"

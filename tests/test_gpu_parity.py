@@ -285,5 +285,5 @@ def test_unsupported_shapes_rejected_on_device_pointers(g):
     assert e.value.status == 2
     inp = to_dev(W.draw(1, 64, 1, 64, 64, seed=4, dtype=torch.bfloat16))
     with pytest.raises(g.Gdn2Error) as e:
-        g.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"], None, chunk=32)
+        g.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"], None, chunk=48)
     assert e.value.status == 2
