@@ -251,6 +251,40 @@ def bench_chunk_fused(g, wl, steps, warmup, rank, stream):
     return ms / steps
 
 
+def bench_chunk_general(g, wl, steps, rank, stream, *, H=None, HV=None, lengths=None):
+    """chunk_fwd_ex on the workload's shapes with H key heads and HV value heads
+    (defaults: the workload's H), optionally as packed sequences of the given
+    lengths (their sum replaces B x T).  Returns (ms per call, bytes per call)."""
+    H = wl.H if H is None else H
+    HV = H if HV is None else HV
+    if lengths is None:
+        Bt, T, N = wl.B, wl.T, wl.B
+        cu = None
+    else:
+        cu_h = W.cu_seqlens_of(lengths)
+        Bt, T, N = 1, int(cu_h[-1]), len(lengths)
+        cu = cu_h.to("cuda")
+    d = W.draw(Bt, T, H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 11, dtype=wl.torch_dtype,
+               alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, b_scale=wl.b_scale, HV=HV, device="cuda")
+    o = torch.empty_like(d["v"])
+    S_T = torch.empty(N, HV, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
+
+    def step():
+        g.chunk_fwd_ex(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], None, cu_seqlens=cu,
+                       o=o, S_T=S_T, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    torch.cuda.synchronize()
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("chunk kernel reported a device error")
+    io = 2 if wl.io == "bf16" else 4
+    nbytes = Bt * T * (H * 4 * wl.d_k + HV * 3 * wl.d_v) * io + N * HV * wl.d_k * wl.d_v * 4
+    return ms / steps, nbytes, Bt * T
+
+
 def bench_decode_fused(g, wl, steps, rank, stream):
     d = W.draw_raw(wl.B, None, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 7, dtype=wl.torch_dtype,
                    alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, qk_scale=2.0, s0_std=wl.s0_std, steps=steps,
@@ -518,6 +552,25 @@ def main():
             "roofline": {"bound": "hbm", "achieved": bdf / (pf / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": bdf / (pf / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_step": bdf}}
         torch.cuda.empty_cache()
+
+        # f3: the headline's 32768 tokens as packed sequences of mixed length, and
+        # value heads (8 key heads shared by 16 value heads) at the headline shape
+        lens = W.packed_lengths(64, wl.T // 8, seed=rank_seed(wl, rank) + 13, min_len=1)
+        nst = max(10, args.steps // 4)
+        for name, kw, desc in (
+                ("packed_varlen", dict(lengths=lens),
+                 f"chunk_fwd {len(lens)} packed sequences, {sum(lens)} tokens (lengths ~ exponential, "
+                 f"mean {wl.T // 8}), H{wl.H} d_k{wl.d_k} d_v{wl.d_v} chunk64 bf16"),
+                ("value_heads", dict(H=wl.H // 2, HV=wl.H),
+                 f"chunk_fwd B{wl.B} T{wl.T} H{wl.H // 2} key heads, HV{wl.H} value heads, "
+                 f"d_k{wl.d_k} d_v{wl.d_v} chunk64 bf16")):
+            lg, bg, ntok = bench_chunk_general(g, wl, nst, rank, stream, **kw)
+            extras[name] = {
+                "workload": desc, "value": ntok / (lg / 1e3), "unit": "tokens/s", "ms_per_call": lg,
+                "roofline": {"bound": "hbm", "achieved": bg / (lg / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": bg / (lg / 1e3) / 1e9 / peaks["hbm_gbs"],
+                             "bytes_per_launch": bg}}
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
