@@ -655,11 +655,13 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
             {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
-                // the scratch's last rows overlap the T tile
+                // the scratch's last rows overlap the T tile.  A quarter-warp takes one
+                // 8-column chunk of 8 consecutive rows: distinct banks on both sides.
                 uint32_t tp[2][4];
 #pragma unroll
                 for (int it = 0; it < 2; ++it) {
-                    const int idx = t + it * kKeyThreads, r = idx >> 3, ch = idx & 7, c0 = 8 * ch;
+                    const int idx = t + it * kKeyThreads;
+                    const int r = (idx & 7) | ((idx >> 6) << 3), ch = (idx >> 3) & 7, c0 = 8 * ch;
                     // T is unit lower triangular: the scratch above the diagonal is zero
                     // except the upper-right 32x32 block, which holds the solve's products
                     if (r < 32 && c0 >= 32) {
@@ -676,7 +678,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 named_bar(1, kKeyThreads);
 #pragma unroll
                 for (int it = 0; it < 2; ++it) {
-                    const int idx = t + it * kKeyThreads, r = idx >> 3, ch = idx & 7;
+                    const int idx = t + it * kKeyThreads;
+                    const int r = (idx & 7) | ((idx >> 6) << 3), ch = (idx >> 3) & 7;
                     st_shared_v4(sb + Cfg::OFF_T + sw128_chunk(r, ch), tp[it][0], tp[it][1], tp[it][2], tp[it][3]);
                 }
             }
