@@ -375,6 +375,37 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
     fence_proxy_async_smem();
 }
 
+// Packed sequences: grid slot z runs the sequence of length rank z (longest
+// first, ties by index), so that blocks, which start in z order, begin with
+// the long sequences and the short ones fill in behind them (longest-
+// processing-time-first scheduling).  Every CTA ranks the lengths itself in
+// `scratch` (shared memory that the setup clears afterwards): warp w takes
+// candidates i = w, w + warps, ..., its lanes count the sequences ahead of i.
+// Up to kMaxRankedSeqs sequences; beyond that slot z runs sequence z.
+constexpr int kMaxRankedSeqs = 1024;
+__device__ __forceinline__ int longest_first_sequence(const int *__restrict__ cu, int nseq, int slot, int *scratch) {
+    if (nseq <= 1 || nseq > kMaxRankedSeqs) return slot;
+    int *lens = scratch, *pick = scratch + kMaxRankedSeqs;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    for (int i = tid; i < nseq; i += blockDim.x) lens[i] = cu[i + 1] - cu[i];
+    if (tid == 0) *pick = slot;   // a total order always has one sequence of rank `slot`
+    __syncthreads();
+    for (int i = warp; i < nseq; i += nwarps) {
+        const int li = lens[i];
+        int ahead = 0;
+        for (int j = lane; j < nseq; j += 32) {
+            const int lj = lens[j];
+            ahead += (lj > li || (lj == li && j < i)) ? 1 : 0;
+        }
+        ahead = __reduce_add_sync(0xffffffffu, ahead);
+        if (lane == 0 && ahead == slot) *pick = i;
+    }
+    __syncthreads();
+    const int r = *pick;
+    __syncthreads();   // everyone has read it before the scratch is reused
+    return r;
+}
+
 // PREP fuses the input prep (raw q, k, b, w); EPI the gated RMS norm of each
 // output row before it is stored (d_v == NV: one CTA holds the whole row).
 template <int DK, int NV, bool PREP = false, bool EPI = false, bool VARLEN = false>
@@ -397,7 +428,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // A sequence is tokens [tok0, tok0 + len): bb * T + [0, T) for equal-length
     // batches, [cu[bb], cu[bb + 1]) when packed (the TMA maps then have one
     // "batch" of all tokens: coordinates (c, head, tok0 + 64 n, 0)).
-    const int j0 = blockIdx.x * NV, hv = blockIdx.y, bb = blockIdx.z;
+    const int j0 = blockIdx.x * NV, hv = blockIdx.y;
+    int bb = blockIdx.z;
+    if constexpr (VARLEN) bb = longest_first_sequence(cu_seqlens, gridDim.z, bb, reinterpret_cast<int *>(smem));
     const int h = hv / (HV / H);
     long tok0 = (long)bb * T;
     int len = T, tma_t0 = 0, tma_b = bb;

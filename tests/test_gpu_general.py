@@ -265,3 +265,15 @@ def test_chunk32_packed_value_heads_fused(g):
     eo = max(float(np.max(np.abs(a - r))) for a, r in zip(got, ro) if r.size) / scale
     es = rel_inf(S_T.double().cpu().numpy().reshape(len(lens) * HV, dk, dv), rS)
     assert eo <= 2e-2 and es <= 2e-2, f"o err {eo:.3e}, S_T err {es:.3e}"
+
+
+def test_packed_equal_lengths_ties(g):
+    """Equal lengths (rank ties broken by index) and a mix around one chunk."""
+    _packed_check(g, [64, 64, 30, 64, 30, 0, 64, 30], 2, 2, 128, 128, torch.bfloat16, seed=7300)
+
+
+def test_packed_more_sequences_than_ranked(g):
+    """1100 short sequences: more than the kernel ranks, so slot z runs sequence z."""
+    rng = np.random.default_rng(7400)
+    lens = [int(x) for x in rng.integers(0, 6, size=1100)]
+    _packed_check(g, lens, 1, 1, 64, 64, torch.bfloat16, seed=7401)
