@@ -121,8 +121,13 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 }
 // One warp: C (16 x 16, row stride LDA) = sign * Am (16 x K) Bm (K x 16), all in
 // fp32 shared memory with row stride LDA, products in tf32 on the tensor cores.
+// With a tile `tt`, C also goes, rounded to bf16, to rows trow.., columns
+// tcol.. of that 128-byte-swizzled 64 x 64 tile; keep_fp32 = false leaves
+// the fp32 copy out.
 template <int LDA, int K>
-__device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, float *Cm, float sign, int lane) {
+__device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, float *Cm, float sign, int lane,
+                                            uint8_t *tt = nullptr, int trow = 0, int tcol = 0,
+                                            bool keep_fp32 = true) {
     const int g = lane >> 2, q = lane & 3;
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -137,8 +142,16 @@ __device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, fl
     }
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        *reinterpret_cast<float2 *>(Cm + g * LDA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
-        *reinterpret_cast<float2 *>(Cm + (g + 8) * LDA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][2], sign * acc[nt][3]);
+        if (keep_fp32) {
+            *reinterpret_cast<float2 *>(Cm + g * LDA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
+            *reinterpret_cast<float2 *>(Cm + (g + 8) * LDA + 8 * nt + 2 * q) =
+                make_float2(sign * acc[nt][2], sign * acc[nt][3]);
+        }
+        if (tt != nullptr) {
+            const uint32_t c = static_cast<uint32_t>(tcol + 8 * nt + 2 * q);
+            *reinterpret_cast<uint32_t *>(tt + sw128_off(trow + g, c)) = pack_bf16x2(sign * acc[nt][0], sign * acc[nt][1]);
+            *reinterpret_cast<uint32_t *>(tt + sw128_off(trow + g + 8, c)) = pack_bf16x2(sign * acc[nt][2], sign * acc[nt][3]);
+        }
     }
 }
 
@@ -151,13 +164,17 @@ __device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, fl
 //   3. 32 -> 64: T_ba = -T_b (A_ba T_a) with a = rows/cols 0-31, b = 32-63
 //      (warp w: rows 16 (w % 2), columns 16 (w / 2) of each product).
 // The block products run on the tensor cores (mma.sync, tf32 inputs, fp32
-// accumulation); T is rounded to bf16 afterwards, which dominates the tf32
-// input rounding.  The intermediate products go to the upper-right 32x32
-// block, which T leaves zero; everywhere else above the diagonal the scratch
-// is exactly zero (given an A that is), so readers of T only zero that
-// block.  `bar` is a named barrier over exactly these 128 threads.
+// accumulation); T is rounded to bf16, which dominates the tf32 input
+// rounding.  The intermediate products go to the upper-right 32x32 block of
+// the scratch.  T also goes, as bf16, to the 128-byte-swizzled MMA tile `tt`
+// as each block becomes final: the diagonal blocks while step 2 runs (warps
+// 2-3, idle there), T_{2p+1,2p} and T_ba from the products' fragments, and
+// rows 0-7 last, because the scratch's last rows overlap them.  Blocks above
+// the diagonal of `tt` are never written here: they keep the zeros the
+// kernel's setup wrote.  `bar` is a named barrier over exactly these 128
+// threads; they fence their tile writes for the tensor core before returning.
 template <int LDA>
-__device__ __forceinline__ void unit_lower_inverse64(float *sA, int t, int bar) {
+__device__ __forceinline__ void unit_lower_inverse64(float *sA, uint8_t *tt, int t, int bar) {
     const int w = t >> 5, lane = t & 31;
     {   // 1. diagonal blocks
         float x[16];
@@ -186,16 +203,36 @@ __device__ __forceinline__ void unit_lower_inverse64(float *sA, int t, int bar) 
         float *Y = sA + (16 * w) * LDA + 32;
         warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R, sA + R * LDA + R, Y, 1.f, lane);
         __syncwarp();
-        warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R + 16, Y, sA + (R + 16) * LDA + R, -1.f, lane);
+        warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R + 16, Y, sA + (R + 16) * LDA + R, -1.f, lane, tt, R + 16, R);
+    } else {       // the diagonal blocks to the tile, 8 columns a thread, rows 8.. (0-7 come last)
+        for (int c = t - 64; c < 128; c += 64) {
+            const int b = c >> 5, row = 16 * b + ((c >> 1) & 15), col0 = 16 * b + 8 * (c & 1);
+            if (row < 8) continue;
+            const float4 a = *reinterpret_cast<const float4 *>(sA + row * LDA + col0);
+            const float4 d = *reinterpret_cast<const float4 *>(sA + row * LDA + col0 + 4);
+            *reinterpret_cast<uint4 *>(tt + sw128_chunk(row, col0 >> 3)) =
+                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(d.x, d.y), pack_bf16x2(d.z, d.w));
+        }
     }
     named_bar(bar, 128);
-    {   // 3. 32 -> 64: Y = A_ba T_a into rows 0-31, cols 32-63; then T_ba = -T_b Y
+    {   // 3. 32 -> 64: Y = A_ba T_a into rows 0-31, cols 32-63; then T_ba = -T_b Y (to the tile only)
         const int rm = 16 * (w & 1), cn = 16 * (w >> 1);
         warp_gemm16<LDA, 32>(sA + (32 + rm) * LDA, sA + cn, sA + rm * LDA + 32 + cn, 1.f, lane);
         named_bar(bar, 128);
-        warp_gemm16<LDA, 32>(sA + (32 + rm) * LDA + 32, sA + 32 + cn, sA + (32 + rm) * LDA + cn, -1.f, lane);
+        warp_gemm16<LDA, 32>(sA + (32 + rm) * LDA + 32, sA + 32 + cn, nullptr, -1.f, lane, tt, 32 + rm, cn, false);
         named_bar(bar, 128);
     }
+    if (t < 64) {   // rows 0-7: D_0's first rows in columns 0-15, zeros elsewhere
+        const int row = t >> 3, ch = t & 7;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (ch < 2) {
+            const float4 a = *reinterpret_cast<const float4 *>(sA + row * LDA + 8 * ch);
+            const float4 d = *reinterpret_cast<const float4 *>(sA + row * LDA + 8 * ch + 4);
+            v = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(d.x, d.y), pack_bf16x2(d.z, d.w));
+        }
+        *reinterpret_cast<uint4 *>(tt + sw128_chunk(row, ch)) = v;
+    }
+    fence_proxy_async_smem();   // MMA2 and MMA3 read the tile
 }
 
 // 8 bf16 products of two 16-byte vectors, rounded back to bf16 (packed bf16x2
@@ -453,7 +490,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *k_full = bars + 2;      // [3] TMA k of a chunk landed (stage m % 3)
     uint64_t *v_full = bars + 5;      // TMA v landed
     uint64_t *w_full = bars + 6;      // TMA w landed
-    uint64_t *v_free = bars + 7;      // key done with W.V (MMA3 complete)
+    uint64_t *v_free = bars + 7;      // MMA3 complete: the v tile (W.V) is free (tcgen05.commit)
     uint64_t *w_free = bars + 8;      // key done with the w tile (W.V formed, solve scratch released)
     uint64_t *full = bars + 9;        // [2] key products of a chunk ready
     uint64_t *empty_qe = bars + 11;   // [2] chain's MMA_s done: Q~/(T E) tiles of the stage free
@@ -463,7 +500,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *bk1 = bars + 19, *bk2 = bars + 20;
     uint64_t *bc1 = bars + 21, *bc2 = bars + 22, *bc3 = bars + 23;
     uint64_t *drain = bars + 24;      // [2] teardown: key and chain MMA issuers
-    constexpr int kNumBars = 26;
+    uint64_t *ut_ready = bars + 26;   // MMA3 of a chunk complete: T(W.V) in TMEM
+    constexpr int kNumBars = 27;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_TMEMP);
     float *gC = reinterpret_cast<float *>(smem + Cfg::OFF_GC);
     float *sA = reinterpret_cast<float *>(smem + Cfg::OFF_SCR);
@@ -627,6 +665,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         r4 = make_uint4(0u, 0u, 0u, 0u);
                     st_shared_v4(sb + Cfg::OFF_V + off, r4.x, r4.y, r4.z, r4.w);
                 }
+                fence_proxy_async_smem();   // MMA3 reads W.V
             }
             {
                 bool ok = mbar_wait(bk1, ph1, wait_ns);
@@ -675,7 +714,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ------------- group A: T = (I + A)^{-1};  group B: prep of chunk m+1
             bool ok_b = true;
             if (!grp_b) {
-                unit_lower_inverse64<Cfg::LDA>(sA, t, 3);
+                unit_lower_inverse64<Cfg::LDA>(sA, smem + Cfg::OFF_T, t, 3);
             } else if (m + 1 < NC) {
                 const int sn = (m + 1) & 1, s3n = (m + 1) % 3;
                 ok_b = mbar_wait(&qb_full[sn], static_cast<uint32_t>(((m + 1) >> 1) & 1), wait_ns);
@@ -683,69 +722,44 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
                     prep_chunk<DK, PREP, VARLEN>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
-                                         gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm,
-                                         min(64, len - (m + 1) * 64));
+                                                 gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm,
+                                                 min(64, len - (m + 1) * 64));
             }
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
-            {   // T (fp32 scratch) -> bf16 T tile; read everything before writing, since
-                // the scratch's last rows overlap the T tile.  A quarter-warp takes one
-                // 8-column chunk of 8 consecutive rows: distinct banks on both sides.
-                uint32_t tp[2][4];
-#pragma unroll
-                for (int it = 0; it < 2; ++it) {
-                    const int idx = t + it * kKeyThreads;
-                    const int r = (idx & 7) | ((idx >> 6) << 3), ch = (idx >> 3) & 7, c0 = 8 * ch;
-                    // T is unit lower triangular: the scratch above the diagonal is zero
-                    // except the upper-right 32x32 block, which holds the solve's products
-                    if (r < 32 && c0 >= 32) {
-                        tp[it][0] = tp[it][1] = tp[it][2] = tp[it][3] = 0u;
-                    } else {
-                        const float4 a = *reinterpret_cast<const float4 *>(sA + r * Cfg::LDA + c0);
-                        const float4 b4 = *reinterpret_cast<const float4 *>(sA + r * Cfg::LDA + c0 + 4);
-                        tp[it][0] = pack_bf16x2(a.x, a.y);
-                        tp[it][1] = pack_bf16x2(a.z, a.w);
-                        tp[it][2] = pack_bf16x2(b4.x, b4.y);
-                        tp[it][3] = pack_bf16x2(b4.z, b4.w);
-                    }
-                }
-                named_bar(1, kKeyThreads);
-#pragma unroll
-                for (int it = 0; it < 2; ++it) {
-                    const int idx = t + it * kKeyThreads;
-                    const int r = (idx & 7) | ((idx >> 6) << 3), ch = (idx >> 3) & 7;
-                    st_shared_v4(sb + Cfg::OFF_T + sw128_chunk(r, ch), tp[it][0], tp[it][1], tp[it][2], tp[it][3]);
-                }
-            }
-            fence_proxy_async_smem();
-            named_bar(1, kKeyThreads);
             if (t == 0) mbar_arrive(w_free);   // w tile (solve scratch) is free
-            // the chain must have read T(W.V) and run MMA_s of the previous chunk
-            if (m >= 1) {
-                const bool ok = mbar_wait(utfree, static_cast<uint32_t>((m - 1) & 1), wait_ns);
-                if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
-            }
             // ------------------------------------------------ MMA2 + MMA3
+            // MMA2 (T E) is committed on its own: the read-out below needs only it.
+            // MMA3 (T(W.V)) completes behind it and frees the v tile and hands
+            // T(W.V) to the chain through its own commits.  Only the issuer waits
+            // for the chain to have read the previous T(W.V) and run its MMA_s.
+            bool ok_ut = true;
             if (t == 0) {
-                tc_fence_after();
-                const uint32_t id2 = idesc_bf16(128, DK, false, true);
+                if (m >= 1) ok_ut = mbar_wait(utfree, static_cast<uint32_t>((m - 1) & 1), wait_ns);
+                if (ok_ut) {
+                    tc_fence_after();
+                    const uint32_t id2 = idesc_bf16(128, DK, false, true);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(t_KT, sdesc_sw128(sb + Cfg::OFF_T - 8192 + ks * 32, 16, 1024),
-                              sdesc_sw128(sb + OQE + 8192 + ks * 2048, 16384, 1024), id2, ks > 0 ? 1u : 0u);
-                const uint32_t id3 = idesc_bf16(128, NV, false, true);
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(t_KT, sdesc_sw128(sb + Cfg::OFF_T - 8192 + ks * 32, 16, 1024),
+                                  sdesc_sw128(sb + OQE + 8192 + ks * 2048, 16384, 1024), id2, ks > 0 ? 1u : 0u);
+                    umma_commit(bk2);
+                    const uint32_t id3 = idesc_bf16(128, NV, false, true);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_bf16(t_UT, sdesc_sw128(sb + Cfg::OFF_T - 8192 + ks * 32, 16, 1024),
-                              sdesc_sw128(sb + Cfg::OFF_V + ks * 2048, 8192, 1024), id3, ks > 0 ? 1u : 0u);
-                umma_commit(bk2);
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(t_UT, sdesc_sw128(sb + Cfg::OFF_T - 8192 + ks * 32, 16, 1024),
+                                  sdesc_sw128(sb + Cfg::OFF_V + ks * 2048, 8192, 1024), id3, ks > 0 ? 1u : 0u);
+                    umma_commit(v_free);
+                    umma_commit(ut_ready);
+                } else {
+                    umma_commit(bk2);   // nothing issued: arrives at once, the group then stops below
+                }
             }
             {
                 const bool ok = mbar_wait(bk2, ph2, wait_ns);
                 ph2 ^= 1u;
-                if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
+                if (group_any(1, kKeyThreads, !(ok && ok_ut))) { failed = true; break; }
             }
             tc_fence_after();
-            if (t == 0) mbar_arrive(v_free);
             // T E rows (TMEM lanes 64-127) -> bf16 over E; channel block kb = kh
             if (kq >= 2 && kh < DK / 64) {
                 const int r = 32 * (kq - 2) + l;
@@ -833,8 +847,9 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 umma_commit(bc1);
             }
             {
-                const bool ok = mbar_wait(bc1, ph1, wait_ns);
+                bool ok = mbar_wait(bc1, ph1, wait_ns);
                 ph1 ^= 1u;
+                ok = ok && mbar_wait(ut_ready, static_cast<uint32_t>(n & 1), wait_ns);   // T(W.V) of this chunk
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
             if (t == 0) mbar_arrive(&empty_qe[s]);   // MMA_s has read Q~ and T E of this stage
