@@ -17,7 +17,9 @@ gated-linear-attention closed forms, separately written KDA and Gated DeltaNet
 recurrences, a hand-derived worked example, and invariants (delta-write,
 state split, linearity, w/v symmetry).  The optional input prep and output
 epilogue are pinned in ``tests/test_oracle_fused_pins.py`` (hand-worked
-values, closed forms of sigmoid and SiLU, scale and sign invariances).
+values, closed forms of sigmoid and SiLU, scale and sign invariances).  The
+second, query-derived erase (``forward_qed``) is pinned in
+``tests/test_oracle_qed_pins.py``.
 """
 from __future__ import annotations
 
@@ -54,6 +56,9 @@ def open_library(path: str):
                                            I, I, I, I, I, I, P, P, I, I,
                                            I, D, P, P, D]
     lib.gdn2_oracle_forward_ex.restype = I
+    lib.gdn2_oracle_forward_qed.argtypes = [P, P, P, P, P, P, P, P, P, P, P,
+                                            I, I, I, I, I, P, I, I, I, D, D]
+    lib.gdn2_oracle_forward_qed.restype = I
     lib.gdn2_oracle_max_threads.restype = I
     return lib
 
@@ -185,3 +190,51 @@ def decode_steps(q, k, v, log_alpha, b, w, S0, heads=None, n_threads: int = 0, *
                    heads=heads, n_threads=n_threads, prep=prep, allow_neg_eigval=allow_neg_eigval,
                    l2_eps=l2_eps, gate=None if gate is None else tb(gate), norm_weight=norm_weight,
                    norm_eps=norm_eps)
+
+
+def forward_qed(q, k, v, log_alpha, b, c, w, S0=None, heads=None, n_threads: int = 0, *,
+                prep: bool = False, allow_neg_eigval: bool = False, l2_eps: float = 1e-6,
+                qed_eps: float = 1e-6, want_smax: bool = False, lib=None):
+    """The recurrence with the second, query-derived erase direction.
+
+    u_t = r_t / sqrt(r_t . r_t + qed_eps) with r_t = q_t - (q_t.k_t / k_t.k_t) k_t,
+    S_t = (I - k_t (b_t . k_t)^T - u_t (c_t . u_t)^T) diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T,
+    o_t = S_t^T q_t.  c : [B, T, H, d_k] is the second erase gate (a logit under
+    prep).  Shapes, heads and returns as in ``forward`` (equal-length sequences,
+    value heads = key heads).
+    """
+    q, k, v, la, b, c, w = (_f32(x) for x in (q, k, v, log_alpha, b, c, w))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for x in (k, la, b, c):
+        assert x.shape == (B, T, H, dk), x.shape
+    for x in (v, w):
+        assert x.shape == (B, T, H, dv), x.shape
+    s0 = None
+    if S0 is not None:
+        if hasattr(S0, "detach"):
+            S0 = S0.detach().double().cpu().numpy()
+        s0 = np.ascontiguousarray(np.asarray(S0, dtype=np.float64))
+        assert s0.shape == (B, H, dk, dv), s0.shape
+    hl = None if heads is None else np.ascontiguousarray(np.asarray(list(heads), dtype=np.int32))
+    nh = B * H if hl is None else int(hl.size)
+    o = np.empty((max(1, nh * T), dv), dtype=np.float64)
+    st = np.empty((nh, dk, dv), dtype=np.float64)
+    sm = np.empty((nh,), dtype=np.float64) if want_smax else None
+    pflag = (1 | (2 if allow_neg_eigval else 0)) if prep else 0
+    rc = (lib or _load()).gdn2_oracle_forward_qed(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(c),
+                                                  _ptr(w), _ptr(s0), _ptr(o), _ptr(st), _ptr(sm),
+                                                  B, T, H, dk, dv, _ptr(hl), nh, int(n_threads),
+                                                  pflag, float(l2_eps), float(qed_eps))
+    if rc != 0:
+        raise ValueError("gdn2 oracle rejected its arguments")
+    o = o[:nh * T].reshape(nh, T, dv)
+    return (o, st, sm) if want_smax else (o, st)
+
+
+def decode_steps_qed(q, k, v, log_alpha, b, c, w, S0, heads=None, n_threads: int = 0, **kw):
+    """``forward_qed`` over a step axis: inputs [steps, B, H, d], S0 [B, H, d_k, d_v]."""
+    def tb(x):
+        return np.ascontiguousarray(np.swapaxes(_f32(x), 0, 1))
+    return forward_qed(tb(q), tb(k), tb(v), tb(log_alpha), tb(b), tb(c), tb(w), S0=S0, heads=heads,
+                       n_threads=n_threads, **kw)

@@ -51,6 +51,19 @@
  *       silu(x) = x / (1 + exp(-x)), per (token, head) over d_v.
  * Readings: the L2 epsilon (not on the pages) is an argument; the RMS norm
  * is taken per head over d_v with one weight vector [d_v] for all heads.
+ *
+ * gdn2_oracle_forward_qed adds the second erase direction of the "Query
+ * Knows What to Forget" page (mlsanity 2608.13668, abstract: a direction
+ * taken from the query, orthogonal to the key, that cancels what the old
+ * state holds along the query).  The page gives no formula; the reading
+ * taken here is the plainest one the abstract supports:
+ *     r_t = q_t - ((q_t . k_t) / (k_t . k_t)) k_t      (q_t itself when k_t = 0)
+ *     u_t = r_t / sqrt(r_t . r_t + qed_eps)           (u_t . k_t = 0)
+ *     S_t = (I - k_t (b_t . k_t)^T - u_t (c_t . u_t)^T) diag(alpha_t) S_{t-1}
+ *           + k_t (w_t . v_t)^T
+ * with c_t in [0, 1] a second erase gate on the key axis, an input like b
+ * (sigmoid of a logit under the input prep, never doubled).  The two erases
+ * act together on the decayed state, as one rank-2 edit.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -66,6 +79,8 @@ typedef struct {
     const float *gate;     /* NULL: no epilogue; else [B, T, H, d_v] */
     const double *weight;  /* [d_v] */
     double norm_eps;
+    const float *qed_c;    /* NULL: no second erase; else [B, T, H, d_k] */
+    double qed_eps;
 } fuse_t;
 
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
@@ -92,16 +107,17 @@ static void token_inputs(const float *qt, const float *kt, const float *bt, cons
 }
 
 static int run_head(const float *q, const float *k, const float *v,
-                    const float *la, const float *b, const float *w, const float *g,
+                    const float *la, const float *b, const float *w, const float *g, const float *c,
                     const double *S0, double *o, double *S_T, double *smax,
                     long T, long H, long HV, long dk, long dv, const fuse_t *f)
 {
     double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv));
     double *r = (double *)malloc(sizeof(double) * (size_t)dv);
     double *u = (double *)malloc(sizeof(double) * (size_t)dv);
-    double *tk = (double *)malloc(sizeof(double) * (size_t)(3 * dk + dv));
+    double *tk = (double *)malloc(sizeof(double) * (size_t)(5 * dk + 2 * dv));
     if (!S || !r || !u || !tk) { free(S); free(r); free(u); free(tk); return -1; }
     double *qd = tk, *kd = tk + dk, *bd = tk + 2 * dk, *wd = tk + 3 * dk;
+    double *ud = tk + 3 * dk + dv, *cd = tk + 4 * dk + dv, *r2 = tk + 5 * dk + dv;
     if (S0) memcpy(S, S0, sizeof(double) * (size_t)(dk * dv));
     else    memset(S, 0, sizeof(double) * (size_t)(dk * dv));
     double big = 0.0;
@@ -121,6 +137,31 @@ static int run_head(const float *q, const float *k, const float *v,
             const double bk = bd[i] * kd[i];
             const double *row = S + i * dv;
             for (long j = 0; j < dv; ++j) r[j] += bk * row[j];
+        }
+        /* second erase: u_t from q_t orthogonal to k_t; r2 = (c_t . u_t)^T (decayed S) */
+        if (c) {
+            const float *ct = c + t * sk;
+            double qk = 0.0, kk = 0.0, rr = 0.0;
+            for (long i = 0; i < dk; ++i) { qk += qd[i] * kd[i]; kk += kd[i] * kd[i]; }
+            const double coef = kk > 0.0 ? qk / kk : 0.0;
+            for (long i = 0; i < dk; ++i) { ud[i] = qd[i] - coef * kd[i]; rr += ud[i] * ud[i]; }
+            const double nr = sqrt(rr + f->qed_eps);
+            const double inr = nr > 0.0 ? 1.0 / nr : 0.0;
+            for (long i = 0; i < dk; ++i) {
+                ud[i] *= inr;
+                cd[i] = f->prep ? sigmoid((double)ct[i]) : (double)ct[i];
+            }
+            for (long j = 0; j < dv; ++j) r2[j] = 0.0;
+            for (long i = 0; i < dk; ++i) {
+                const double cu = cd[i] * ud[i];
+                const double *row = S + i * dv;
+                for (long j = 0; j < dv; ++j) r2[j] += cu * row[j];
+            }
+            for (long i = 0; i < dk; ++i) {   /* S -= u_t r2^T, before the key-directed edit */
+                const double ui = ud[i];
+                double *row = S + i * dv;
+                for (long j = 0; j < dv; ++j) row[j] -= ui * r2[j];
+            }
         }
         /* u = w_t . v_t - r ;  S += k_t u^T */
         for (long j = 0; j < dv; ++j) u[j] = wd[j] * (double)vt[j] - r[j];
@@ -206,6 +247,7 @@ static int forward_impl(const float *q, const float *k, const float *v,
         const long off_k = (t0 * H + hk) * d_k, off_v = (t0 * HV + hv) * d_v;
         bad |= run_head(q + off_k, k + off_k, v + off_v, log_alpha + off_k,
                         b + off_k, w + off_v, f->gate ? f->gate + off_v : NULL,
+                        f->qed_c ? f->qed_c + off_k : NULL,
                         S0 ? S0 + bh * (long)d_k * d_v : NULL,
                         o + orow[n] * d_v,
                         S_T ? S_T + n * (long)d_k * d_v : NULL,
@@ -221,7 +263,7 @@ int gdn2_oracle_forward(const float *q, const float *k, const float *v,
                         int B, int T, int H, int d_k, int d_v,
                         const int *heads, int n_heads, int n_threads)
 {
-    const fuse_t f = {0, 0, 0.0, NULL, NULL, 0.0};
+    const fuse_t f = {0, 0, 0.0, NULL, NULL, 0.0, NULL, 0.0};
     return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, H, d_k, d_v, NULL,
                         heads, n_heads, n_threads, &f);
 }
@@ -238,8 +280,25 @@ int gdn2_oracle_forward_ex(const float *q, const float *k, const float *v,
                            double norm_eps)
 {
     if (prep != 0 && prep != 1 && prep != 3) return -1;
-    const fuse_t f = {prep & 1, (prep >> 1) & 1, l2_eps, gate, weight, norm_eps};
+    const fuse_t f = {prep & 1, (prep >> 1) & 1, l2_eps, gate, weight, norm_eps, NULL, 0.0};
     return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, HV, d_k, d_v, cu_seqlens,
+                        heads, n_heads, n_threads, &f);
+}
+
+/* The recurrence with the second, query-derived erase (see the header);
+ * c is [B, T, H, d_k]; prep as for gdn2_oracle_forward_ex (c = sigmoid(c_raw)
+ * under it).  Equal-length sequences, value heads = key heads, no epilogue. */
+int gdn2_oracle_forward_qed(const float *q, const float *k, const float *v,
+                            const float *log_alpha, const float *b, const float *c, const float *w,
+                            const double *S0, double *o, double *S_T, double *smax,
+                            int B, int T, int H, int d_k, int d_v,
+                            const int *heads, int n_heads, int n_threads,
+                            int prep, double l2_eps, double qed_eps)
+{
+    if (!c || !(qed_eps >= 0.0)) return -1;
+    if (prep != 0 && prep != 1 && prep != 3) return -1;
+    const fuse_t f = {prep & 1, (prep >> 1) & 1, l2_eps, NULL, NULL, 0.0, c, qed_eps};
+    return forward_impl(q, k, v, log_alpha, b, w, S0, o, S_T, smax, B, T, H, H, d_k, d_v, NULL,
                         heads, n_heads, n_threads, &f);
 }
 

@@ -43,6 +43,16 @@ FUSED_MUTANTS = {
 }
 
 
+# mistakes in the second, query-derived erase (forward_qed)
+QED_MUTANTS = {
+    "qed_erase_sign": ("row[j] -= ui * r2[j];", "row[j] += ui * r2[j];"),
+    "qed_not_orthogonal": ("const double coef = kk > 0.0 ? qk / kk : 0.0;", "const double coef = 0.0;"),
+    "qed_not_normalised": ("const double inr = nr > 0.0 ? 1.0 / nr : 0.0;", "const double inr = 1.0;"),
+    "qed_gate_on_key": ("const double cu = cd[i] * ud[i];", "const double cu = cd[i] * kd[i];"),
+    "qed_gate_left_raw": ("cd[i] = f->prep ? sigmoid((double)ct[i]) : (double)ct[i];", "cd[i] = (double)ct[i];"),
+}
+
+
 def _pins_pass(lib) -> bool:
     rng = np.random.default_rng(101)
     q, k, v, la, b, w, S0 = rand_inputs(rng, 2, 17, 2, 5, 4)
@@ -84,6 +94,29 @@ def _fused_pins_pass(lib) -> bool:
     return True
 
 
+def _qed_pins_pass(lib) -> bool:
+    import test_oracle_qed_pins as qp
+
+    class _Mod:   # the oracle module's functions, bound to this library
+        @staticmethod
+        def forward(*a, **kw):
+            return oracle.forward(*a, lib=lib, **kw)
+
+        @staticmethod
+        def forward_qed(*a, **kw):
+            return oracle.forward_qed(*a, lib=lib, **kw)
+
+    checks = [lambda: qp.test_qed_brute_force_matrix_form(_Mod, 2, 21, 2, 6, 5, 1e-6),
+              lambda: qp.test_qed_full_erase_read_sees_only_the_key_part(_Mod),
+              lambda: qp.test_qed_prep_gates_c_with_the_logistic(_Mod)]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
 def _compile(src_text: str, tmp_path, name: str):
     c = tmp_path / f"{name}.c"
     so = tmp_path / f"{name}.so"
@@ -100,7 +133,7 @@ def oracle_source():
 
 def test_unmutated_copy_passes(oracle_source, tmp_path):
     lib = _compile(oracle_source, tmp_path, "clean")
-    assert _pins_pass(lib) and _fused_pins_pass(lib)
+    assert _pins_pass(lib) and _fused_pins_pass(lib) and _qed_pins_pass(lib)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -117,3 +150,11 @@ def test_fused_mutant_is_caught(oracle_source, tmp_path, name):
     assert oracle_source.count(old) == 1, f"mutation site for {name} not found"
     lib = _compile(oracle_source.replace(old, new), tmp_path, name)
     assert not _fused_pins_pass(lib), f"fused pins did not catch mutant {name}"
+
+
+@pytest.mark.parametrize("name", sorted(QED_MUTANTS))
+def test_qed_mutant_is_caught(oracle_source, tmp_path, name):
+    old, new = QED_MUTANTS[name]
+    assert oracle_source.count(old) == 1, f"mutation site for {name} not found"
+    lib = _compile(oracle_source.replace(old, new), tmp_path, name)
+    assert not _qed_pins_pass(lib), f"QED pins did not catch mutant {name}"
