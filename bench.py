@@ -285,6 +285,54 @@ def bench_chunk_general(g, wl, steps, rank, stream, *, H=None, HV=None, lengths=
     return ms / steps, nbytes, Bt * T
 
 
+def bench_chunk_qed(g, wl, steps, rank, stream):
+    """The workload's shapes through the second, query-derived erase (CUDA cores)."""
+    d = W.draw(wl.B, wl.T, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 17, dtype=wl.torch_dtype,
+               alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, s0_std=wl.s0_std, device="cuda")
+    c = W.draw_qed_gate((wl.B, wl.T, wl.H), wl.d_k, seed=rank_seed(wl, rank) + 18, dtype=wl.torch_dtype,
+                        device="cuda")
+    o = torch.empty_like(d["v"])
+    S_T = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
+
+    def step():
+        g.chunk_fwd_qed(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], c, d["w"], d["S0"], o=o, S_T=S_T,
+                        stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+    torch.cuda.synchronize()
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("QED chunk kernel reported a device error")
+    return ms / steps
+
+
+def bench_decode_qed(g, wl, steps, rank, stream):
+    d = W.draw(steps, wl.B, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 19, dtype=wl.torch_dtype,
+               device="cuda")
+    c = W.draw_qed_gate((steps, wl.B, wl.H), wl.d_k, seed=rank_seed(wl, rank) + 20, dtype=wl.torch_dtype,
+                        device="cuda")
+    S = (0.02 * torch.randn(wl.B, wl.H, wl.d_k, wl.d_v, device="cuda")).contiguous()
+    o = torch.empty(wl.B, wl.H, wl.d_v, dtype=wl.torch_dtype, device="cuda")
+    it = {"s": 0}
+
+    def step():
+        s = it["s"] % steps
+        it["s"] += 1
+        g.decode_step_qed(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["b"][s], c[s], d["w"][s], S, o=o,
+                          stream=stream)
+
+    for _ in range(8):
+        step()
+    torch.cuda.synchronize()
+    it["s"] = 0
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("QED decode kernel reported a device error")
+    return ms / steps
+
+
 def bench_decode_fused(g, wl, steps, rank, stream):
     d = W.draw_raw(wl.B, None, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 7, dtype=wl.torch_dtype,
                    alpha_lo=wl.alpha_lo, alpha_hi=wl.alpha_hi, qk_scale=2.0, s0_std=wl.s0_std, steps=steps,
@@ -571,6 +619,26 @@ def main():
                              "unit": "GB/s", "frac": bg / (lg / 1e3) / 1e9 / peaks["hbm_gbs"],
                              "bytes_per_launch": bg}}
             torch.cuda.empty_cache()
+
+        # f4: the second, query-derived erase direction (CUDA cores)
+        lq = bench_chunk_qed(g, wl, 3, rank, stream)
+        bq = chunk_bytes(wl, with_s0=wl.s0_std is not None) + wl.B * wl.T * wl.H * wl.d_k * io_b
+        extras["chunk_qed"] = {
+            "workload": wl.describe() + " + second erase direction (query-derived)",
+            "value": wl.B * wl.T / (lq / 1e3), "unit": "tokens/s", "ms_per_call": lq,
+            "roofline": {"bound": "hbm", "achieved": bq / (lq / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": bq / (lq / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_launch": bq}}
+        torch.cuda.empty_cache()
+        nq = 256
+        pq = bench_decode_qed(g, wl4, nq, rank, stream)
+        bdq = decode_bytes(wl4) + wl4.B * wl4.H * wl4.d_k * 2
+        extras["decode_qed"] = {
+            "workload": wl4.describe().replace(f"steps{wl4.decode_steps}", f"steps{nq}")
+            + " + second erase direction (query-derived)",
+            "value": wl4.B / (pq / 1e3), "unit": "tokens/s", "us_per_step": 1e3 * pq, "steps": nq,
+            "roofline": {"bound": "hbm", "achieved": bdq / (pq / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": bdq / (pq / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_step": bdq}}
+        torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:

@@ -7,6 +7,8 @@ library has not been built this module raises on first use.
 
     chunk_fwd(q, k, v, log_alpha, b, w, S0=None) -> (o, S_T)
     decode_step(q, k, v, log_alpha, b, w, S)     -> o      (S updated in place)
+    chunk_fwd_qed / decode_step_qed              -- with the second, query-derived
+        erase direction (gate c on the key axis)
     chunk_fwd_ex / decode_step_ex                 -- the same with value heads,
         packed sequences (cu_seqlens, chunk only) and the fused input prep and
         gated RMS-norm output epilogue
@@ -31,7 +33,7 @@ IO_BF16 = 1
 STATUS_NAMES = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
                 3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT"}
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_decode_step",
-            "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex",
+            "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex", "gdn2_chunk_fwd_qed", "gdn2_decode_step_qed",
             "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_status_string",
             "gdn2_version")
 FUSE_INPUT_PREP = 1    # q, k, b, w are raw: L2-normalise q, k over d_k; b, w = sigmoid
@@ -69,6 +71,12 @@ def lib() -> ctypes.CDLL:
         # (..., B, H, HV, d_k, d_v, io, flags, l2_eps, gate, weight, eps, stream)
         L.gdn2_decode_step_ex.argtypes = [P] * 8 + [I] * 6 + fuse_args + [P]
         L.gdn2_decode_step_ex.restype = I
+        # (q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_k, d_v, io, qed_eps, stream)
+        L.gdn2_chunk_fwd_qed.argtypes = [P] * 10 + [I] * 6 + [F, P]
+        L.gdn2_chunk_fwd_qed.restype = I
+        # (q, k, v, log_alpha, b, c, w, S, o, B, H, d_k, d_v, io, qed_eps, stream)
+        L.gdn2_decode_step_qed.argtypes = [P] * 9 + [I] * 5 + [F, P]
+        L.gdn2_decode_step_qed.restype = I
         L.gdn2_device_status.argtypes = [P]
         L.gdn2_device_status.restype = I
         L.gdn2_selftest_wait_timeout.argtypes = [I, P]
@@ -267,6 +275,57 @@ def decode_step_ex(q, k, v, log_alpha, b, w, S, *, prep: bool = False, allow_neg
     fuse = lambda q_, shape: _fuse_args(q_, prep, allow_neg_eigval, l2_eps, gate, norm_weight,
                                         norm_eps, shape)
     return _decode("gdn2_decode_step_ex", q, k, v, log_alpha, b, w, S, o, stream, fuse, ex=True)
+
+
+def chunk_fwd_qed(q, k, v, log_alpha, b, c, w, S0=None, *, qed_eps: float = 1e-6, o=None, S_T=None,
+                  stream=None, want_state: bool = True):
+    """Chunk forward with the second erase direction u_t (the part of q_t orthogonal to
+    k_t, normalised) gated by c [B,T,H,d_k]; returns (o [B,T,H,d_v], S_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check_tokens((q, k, v, log_alpha, b, c, w), q.dtype, dev)
+    for t in (k, log_alpha, b, c):
+        if tuple(t.shape) != (B, T, H, dk):
+            raise ValueError("q, k, log_alpha, b, c must be [B, T, H, d_k]")
+    if tuple(w.shape) != (B, T, H, dv) or tuple(v.shape) != (B, T, H, dv):
+        raise ValueError("v, w must be [B, T, H, d_v]")
+    _check_state(S0, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=dev)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check_tokens((o,), q.dtype, dev)
+    _check_state(S_T, (B, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        st = lib().gdn2_chunk_fwd_qed(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(c), _ptr(w),
+                                      _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, _io(q.dtype),
+                                      ctypes.c_float(float(qed_eps)), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_chunk_fwd_qed")
+    return o, S_T
+
+
+def decode_step_qed(q, k, v, log_alpha, b, c, w, S, *, qed_eps: float = 1e-6, o=None, stream=None):
+    """One token per sequence with the second erase direction; S [B,H,d_k,d_v] fp32
+    is updated in place; returns o [B,H,d_v]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check_tokens((q, k, v, log_alpha, b, c, w), q.dtype, dev)
+    for t in (k, log_alpha, b, c):
+        if tuple(t.shape) != (B, H, dk):
+            raise ValueError("q, k, log_alpha, b, c must be [B, H, d_k]")
+    _check_state(S, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
+    with torch.cuda.device(dev):
+        st = lib().gdn2_decode_step_qed(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(c), _ptr(w),
+                                        _ptr(S), _ptr(o), B, H, dk, dv, _io(q.dtype),
+                                        ctypes.c_float(float(qed_eps)), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_decode_step_qed")
+    return o
 
 
 def device_status(stream=None) -> int:

@@ -15,6 +15,7 @@
 #include "chunk_tc.cuh"
 #include "decode.cuh"
 #include "epilogue.cuh"
+#include "qed.cuh"
 #include "gdn2_device.cuh"
 
 namespace gdn2 {
@@ -372,6 +373,86 @@ extern "C" gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const
     if (s != GDN2_OK) return s;
     if (gate == nullptr && norm_weight != nullptr) return GDN2_ERR_INVALID_ARG;
     return decode_impl(q, k, v, log_alpha, b, w, S, o, B, H, HV != 0 ? HV : H, d_k, d_v, io, stream, &fz);
+}
+
+namespace gdn2 {
+namespace {
+template <typename IO, int DK>
+gdn2_status_t launch_qed_chunk(const void *q, const void *k, const void *v, const void *la, const void *b,
+                               const void *c, const void *w, const float *S0, void *o, float *S_T, int B,
+                               int T, int H, int d_v, float eps, cudaStream_t st) {
+    using Cfg = QedCfg<DK>;
+    auto kern = chunk_fwd_qed_kernel<IO, DK>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+    dim3 grid(d_v / Cfg::NV, H, B);
+    kern<<<grid, 256, Cfg::BYTES, st>>>(static_cast<const IO *>(q), static_cast<const IO *>(k),
+                                        static_cast<const IO *>(v), static_cast<const IO *>(la),
+                                        static_cast<const IO *>(b), static_cast<const IO *>(c),
+                                        static_cast<const IO *>(w), S0, static_cast<IO *>(o), S_T, T, H, d_v, eps);
+    return from_cuda(cudaGetLastError());
+}
+
+template <typename IO, int DK, int NVD>
+gdn2_status_t launch_qed_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
+                                const void *c, const void *w, float *S, void *o, int B, int H, int d_v, float eps,
+                                cudaStream_t st) {
+    dim3 grid((unsigned)((long)B * H), d_v / NVD);
+    decode_step_qed_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
+        static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
+        static_cast<const IO *>(la), static_cast<const IO *>(b), static_cast<const IO *>(c),
+        static_cast<const IO *>(w), S, static_cast<IO *>(o), d_v, eps);
+    return from_cuda(cudaGetLastError());
+}
+}  // namespace
+}  // namespace gdn2
+
+extern "C" gdn2_status_t gdn2_chunk_fwd_qed(const void *q, const void *k, const void *v, const void *log_alpha,
+                                            const void *b, const void *c, const void *w, const float *S0, void *o,
+                                            float *S_T, int B, int T, int H, int d_k, int d_v, gdn2_io_t io,
+                                            float qed_eps, void *stream) {
+    const Shape sh{B, T, H, H, d_k, d_v, nullptr};
+    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, sh, 64, io);
+    if (s != GDN2_OK) return s;
+    if (T > 0 && c == nullptr) return GDN2_ERR_INVALID_ARG;
+    if (!(qed_eps >= 0.f)) return GDN2_ERR_INVALID_ARG;
+    if (c && !aligned16(c)) return GDN2_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return empty_sequence(S0, S_T, sh, st);
+    if (io == GDN2_IO_F32) {
+        if (d_k == 64) return launch_qed_chunk<float, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
+        return launch_qed_chunk<float, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
+    }
+    if (d_k == 64)
+        return launch_qed_chunk<__nv_bfloat16, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
+    return launch_qed_chunk<__nv_bfloat16, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
+}
+
+extern "C" gdn2_status_t gdn2_decode_step_qed(const void *q, const void *k, const void *v, const void *log_alpha,
+                                              const void *b, const void *c, const void *w, float *S, void *o,
+                                              int B, int H, int d_k, int d_v, gdn2_io_t io, float qed_eps,
+                                              void *stream) {
+    if (!q || !k || !v || !log_alpha || !b || !c || !w || !S || !o) return GDN2_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || d_k <= 0 || d_v <= 0 || !(qed_eps >= 0.f)) return GDN2_ERR_INVALID_ARG;
+    if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    const void *ptrs[9] = {q, k, v, log_alpha, b, c, w, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDN2_ERR_MISALIGNED;
+    if (d_k != 64 && d_k != 128) return GDN2_ERR_UNSUPPORTED;
+    if (d_v % 64 != 0 || d_v > 512) return GDN2_ERR_UNSUPPORTED;
+    if ((long)B * H > INT_MAX) return GDN2_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool wide = (d_v % 128 == 0);
+#define GDN2_QED_DECODE(IO, DK)                                                                                  \
+    return wide ? launch_qed_decode<IO, DK, 128>(q, k, v, log_alpha, b, c, w, S, o, B, H, d_v, qed_eps, st)     \
+                : launch_qed_decode<IO, DK, 64>(q, k, v, log_alpha, b, c, w, S, o, B, H, d_v, qed_eps, st)
+    if (io == GDN2_IO_F32) {
+        if (d_k == 64) GDN2_QED_DECODE(float, 64);
+        GDN2_QED_DECODE(float, 128);
+    }
+    if (d_k == 64) GDN2_QED_DECODE(__nv_bfloat16, 64);
+    GDN2_QED_DECODE(__nv_bfloat16, 128);
+#undef GDN2_QED_DECODE
 }
 
 extern "C" gdn2_status_t gdn2_device_status(void *stream) {

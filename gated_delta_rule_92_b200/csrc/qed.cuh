@@ -1,0 +1,366 @@
+// qed.cuh -- GDN-2 with the second, query-derived erase direction.
+//
+// "The Query Knows What to Forget" (mlsanity 2608.13668, abstract): a second
+// erase direction, taken from the query and orthogonal to the key, cancels
+// what the old state holds along the query.  The page prints no formula; the
+// reading built here is
+//     r_t = q_t - ((q_t . k_t) / (k_t . k_t)) k_t,   u_t = r_t / sqrt(r_t . r_t + eps)
+//     S_t = (I - k_t (b_t . k_t)^T - u_t (c_t . u_t)^T) diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T
+//     o_t = S_t^T q_t
+// with c_t a second erase gate on the key axis.  Both erases act on the same
+// decayed state, one rank-2 edit per token.  CUDA cores, fp32 products.
+#pragma once
+#include "chunk_ffma.cuh"
+#include "decode.cuh"
+#include "gdn2_device.cuh"
+
+namespace gdn2 {
+
+// Sum of `x` over the DK threads 0..DK-1 of the block (the others pass 0):
+// warp shuffles, then the DK / 32 warp totals through `scratch` (DK / 32 floats).
+// Every thread of the block must call it.
+template <int DK>
+__device__ __forceinline__ float block_sum_dk(float x, float *scratch) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if ((threadIdx.x & 31) == 0 && threadIdx.x < DK) scratch[threadIdx.x >> 5] = x;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < DK / 32; ++w) t += scratch[w];
+    __syncthreads();
+    return t;
+}
+
+// One decode step per (b, h, NVD-column slice of d_v), 256 threads.  Per
+// value column j, with S = S_{t-1} and the decay alpha:
+//     r1_j = sum_i (b_i k_i alpha_i) S_ij,  r2_j = sum_i (c_i u_i alpha_i) S_ij,
+//     p_j  = sum_i (q_i alpha_i) S_ij,      x_j  = w_j v_j - r1_j
+//     S_ij <- alpha_i S_ij + k_i x_j - u_i r2_j
+//     o_j  = p_j + (q . k) x_j - (q . u) r2_j,   q . u = |r|^2 / sqrt(|r|^2 + eps)
+// S is read once and written once, as in the GDN-2 step.
+template <typename IO, int DK, int NVD>
+__global__ void __launch_bounds__(256, 2)
+decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
+                       const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ cg_,
+                       const IO *__restrict__ wg, float *__restrict__ S, IO *__restrict__ o, int d_v,
+                       float qed_eps) {
+    constexpr int TPR = NVD / 4;   // threads across one row of the slice
+    constexpr int RG = 256 / TPR;  // thread rows
+    constexpr int RPT = DK / RG;   // state rows per thread
+    static_assert(RPT >= 1 && RG * RPT == DK, "bad decode tiling");
+
+    __shared__ float s_alpha[DK], s_e1[DK], s_e2[DK], s_qa[DK], s_k[DK], s_u[DK];
+    __shared__ float s_wv[NVD];
+    __shared__ __align__(16) float s_red[3][RG][NVD];
+    __shared__ float s_scr[DK / 32];
+
+    const int tid = threadIdx.x;
+    const int cgr = tid % TPR;   // float4 column group
+    const int rg = tid / TPR;    // thread row
+    const long bh = blockIdx.x;
+    const int j0 = blockIdx.y * NVD;
+
+    float *Sh = S + bh * (long)DK * d_v + j0 + cgr * 4;
+    float4 s[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(reinterpret_cast<const float4 *>(Sh + (long)(i * RG + rg) * d_v));
+
+    float qv = 0.f, kv = 0.f, bv = 0.f, cv = 0.f, lv = 0.f;
+    if (tid < DK) {
+        const long off = bh * DK + tid;
+        qv = ld_io(q + off);
+        kv = ld_io(k + off);
+        bv = ld_io(bg + off);
+        cv = ld_io(cg_ + off);
+        lv = ld_io(la + off);
+    }
+    // the query's part orthogonal to the key, normalised
+    const float qk = block_sum_dk<DK>(qv * kv, s_scr);
+    const float kk = block_sum_dk<DK>(kv * kv, s_scr);
+    const float coef = kk > 0.f ? qk / kk : 0.f;
+    const float rv = qv - coef * kv;
+    const float rr = block_sum_dk<DK>(rv * rv, s_scr);
+    const float den = rr + qed_eps;
+    const float nu = den > 0.f ? rsqrtf(den) : 0.f;
+    const float qu = rr * nu;   // q . u = r . r / sqrt(r . r + eps)
+    if (tid < DK) {
+        const float a = __expf(lv), uv = rv * nu;
+        s_alpha[tid] = a;
+        s_e1[tid] = bv * kv * a;
+        s_e2[tid] = cv * uv * a;
+        s_qa[tid] = qv * a;
+        s_k[tid] = kv;
+        s_u[tid] = uv;
+    }
+    if (tid < NVD) {
+        const long vo = bh * (long)d_v + j0 + tid;
+        s_wv[tid] = ld_io(wg + vo) * ld_io(v + vo);
+    }
+    __syncthreads();
+
+    // partial column sums over this thread's rows
+    float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), a2 = a1, ap = a1;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int row = i * RG + rg;
+        const float e1 = s_e1[row], e2 = s_e2[row], qa = s_qa[row];
+        a1.x += e1 * s[i].x; a1.y += e1 * s[i].y; a1.z += e1 * s[i].z; a1.w += e1 * s[i].w;
+        a2.x += e2 * s[i].x; a2.y += e2 * s[i].y; a2.z += e2 * s[i].z; a2.w += e2 * s[i].w;
+        ap.x += qa * s[i].x; ap.y += qa * s[i].y; ap.z += qa * s[i].z; ap.w += qa * s[i].w;
+    }
+    *reinterpret_cast<float4 *>(&s_red[0][rg][cgr * 4]) = a1;
+    *reinterpret_cast<float4 *>(&s_red[1][rg][cgr * 4]) = a2;
+    *reinterpret_cast<float4 *>(&s_red[2][rg][cgr * 4]) = ap;
+    __syncthreads();
+    float4 r1 = make_float4(0.f, 0.f, 0.f, 0.f), r2 = r1;
+#pragma unroll
+    for (int g = 0; g < RG; ++g) {
+        const float4 x = *reinterpret_cast<const float4 *>(&s_red[0][g][cgr * 4]);
+        const float4 y = *reinterpret_cast<const float4 *>(&s_red[1][g][cgr * 4]);
+        r1.x += x.x; r1.y += x.y; r1.z += x.z; r1.w += x.w;
+        r2.x += y.x; r2.y += y.y; r2.z += y.z; r2.w += y.w;
+    }
+    const float4 wv = *reinterpret_cast<const float4 *>(&s_wv[cgr * 4]);
+    const float4 x = make_float4(wv.x - r1.x, wv.y - r1.y, wv.z - r1.z, wv.w - r1.w);
+    if (rg == 0) {
+        float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < RG; ++g) {
+            const float4 y = *reinterpret_cast<const float4 *>(&s_red[2][g][cgr * 4]);
+            p.x += y.x; p.y += y.y; p.z += y.z; p.w += y.w;
+        }
+        st_io4<IO>(o + bh * (long)d_v + j0 + cgr * 4, p.x + qk * x.x - qu * r2.x, p.y + qk * x.y - qu * r2.y,
+                   p.z + qk * x.z - qu * r2.z, p.w + qk * x.w - qu * r2.w);
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int row = i * RG + rg;
+        const float a = s_alpha[row], kr = s_k[row], ur = s_u[row];
+        float4 n;
+        n.x = a * s[i].x + kr * x.x - ur * r2.x;
+        n.y = a * s[i].y + kr * x.y - ur * r2.y;
+        n.z = a * s[i].z + kr * x.z - ur * r2.z;
+        n.w = a * s[i].w + kr * x.w - ur * r2.w;
+        __stcs(reinterpret_cast<float4 *>(Sh + (long)row * d_v), n);
+    }
+}
+
+// Chunk form.  Unrolling the rank-2 edit over a chunk gives the same WY
+// algebra as GDN-2 with two pseudo-rows per token, rho = 2 t (key k_t, erase
+// b_t.k_t, value w_t.v_t) and rho = 2 t + 1 (direction u_t, erase c_t.u_t,
+// value 0), where both rows of a token see the state before that token:
+//     A_{rho rho'} = E_rho . K~_rho'  for tok(rho') < tok(rho)     (strict, by token)
+//     P_{t rho'}   = Q~_t . K~_rho'   for tok(rho') <= t
+//     U = (I + A)^{-1} (V - E S),  O = Q~ S + P U,  S' = diag(Gamma_C)(S + K~^T U)
+// with Gamma_t the cumulative decay, Q~ = q.Gamma, K~ = kappa/Gamma, E = eps.Gamma.
+// C = 32 tokens make the 64 pseudo-rows of the CUDA-core solve; one block of
+// 256 threads per (b, h, 64-column slice of d_v), everything in shared memory.
+template <int DK>
+struct QedCfg {
+    static constexpr int C = 32;        // tokens per chunk
+    static constexpr int R = 2 * C;     // pseudo-rows
+    static constexpr int NV = 64;
+    static constexpr int LK = DK + 1;   // padded strides: [.][DK], [.][R], [.][NV] tiles
+    static constexpr int LR = R + 1;
+    static constexpr int LV = NV + 1;
+    static constexpr int O_Q = 0;                  // [C][LK]  q -> Q~
+    static constexpr int O_K = O_Q + C * LK;       // [R][LK]  kappa -> K~
+    static constexpr int O_E = O_K + R * LK;       // [R][LK]  erase vectors -> E
+    static constexpr int O_G = O_E + R * LK;       // [C][LK]  log-decay, then A [R][LR], P [C][LR]
+    static constexpr int G_SIZE = (C * LK > (R + C) * LR) ? C * LK : (R + C) * LR;
+    static constexpr int O_T = O_G + G_SIZE;       // [R][LR]
+    static constexpr int O_WV = O_T + R * LR;      // [R][LV]  values, then E S
+    static constexpr int O_U = O_WV + R * LV;      // [R][LV]
+    static constexpr int O_S = O_U + R * LV;       // [DK][LV] state slice
+    static constexpr int O_GC = O_S + DK * LV;     // [DK]
+    static constexpr int FLOATS = O_GC + DK;
+    static constexpr size_t BYTES = sizeof(float) * FLOATS;
+};
+
+template <typename IO, int DK>
+__global__ void __launch_bounds__(256, 1)
+chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
+                     const IO *__restrict__ la, const IO *__restrict__ bg, const IO *__restrict__ cg_,
+                     const IO *__restrict__ wg, const float *__restrict__ S0, IO *__restrict__ o,
+                     float *__restrict__ S_T, int T, int H, int d_v, float qed_eps) {
+    using Cfg = QedCfg<DK>;
+    constexpr int C = Cfg::C, R = Cfg::R, NV = Cfg::NV, LK = Cfg::LK, LR = Cfg::LR, LV = Cfg::LV;
+    extern __shared__ float sm[];
+    float *sQ = sm + Cfg::O_Q, *sK = sm + Cfg::O_K, *sE = sm + Cfg::O_E, *sG = sm + Cfg::O_G;
+    float *sA = sG, *sP = sG + R * LR;
+    float *sT = sm + Cfg::O_T, *sWV = sm + Cfg::O_WV, *sU = sm + Cfg::O_U, *sS = sm + Cfg::O_S;
+    float *sGC = sm + Cfg::O_GC;
+
+    const int tid = threadIdx.x;
+    const int j0 = blockIdx.x * NV, h = blockIdx.y, bb = blockIdx.z;
+    const long head = (long)bb * H + h;
+    const int NC = (T + C - 1) / C;   // the last chunk may be partial (padded rows are zeros)
+
+    for (int idx = tid; idx < DK * NV; idx += 256) {
+        const int c = idx / NV, j = idx % NV;
+        sS[c * LV + j] = S0 ? S0[(head * DK + c) * d_v + j0 + j] : 0.f;
+    }
+    for (int n = 0; n < NC; ++n) {
+        const long tok0 = (long)bb * T + (long)n * C;
+        const int rows = min(C, T - n * C);
+        __syncthreads();
+        // ---- load; pseudo-row 2t: key k_t, erase b_t.k_t; 2t+1: c_t for now
+        for (int idx = tid; idx < C * DK; idx += 256) {
+            const int t = idx / DK, c = idx % DK;
+            const long g = ((tok0 + t) * H + h) * DK + c;
+            const bool in = t < rows;
+            const float kv = in ? ld_io(k + g) : 0.f;
+            sQ[t * LK + c] = in ? ld_io(q + g) : 0.f;
+            sK[(2 * t) * LK + c] = kv;
+            sE[(2 * t) * LK + c] = in ? ld_io(bg + g) * kv : 0.f;
+            sE[(2 * t + 1) * LK + c] = in ? ld_io(cg_ + g) : 0.f;
+            sG[t * LK + c] = in ? ld_io(la + g) : 0.f;
+        }
+        for (int idx = tid; idx < C * NV; idx += 256) {
+            const int t = idx / NV, j = idx % NV;
+            const long g = ((tok0 + t) * H + h) * (long)d_v + j0 + j;
+            sWV[(2 * t) * LV + j] = (t < rows) ? ld_io(wg + g) * ld_io(v + g) : 0.f;
+            sWV[(2 * t + 1) * LV + j] = 0.f;
+        }
+        __syncthreads();
+        // ---- u_t: warp w takes tokens w, w + 8, ...; lanes stride over the channels
+        {
+            const int wp = tid >> 5, l = tid & 31;
+            for (int t = wp; t < C; t += 8) {
+                const float *qr = sQ + t * LK, *kr = sK + (2 * t) * LK;
+                float qk = 0.f, kk = 0.f;
+                for (int c = l; c < DK; c += 32) {
+                    qk = fmaf(qr[c], kr[c], qk);
+                    kk = fmaf(kr[c], kr[c], kk);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    qk += __shfl_xor_sync(0xffffffffu, qk, off);
+                    kk += __shfl_xor_sync(0xffffffffu, kk, off);
+                }
+                const float coef = kk > 0.f ? qk / kk : 0.f;
+                float rr = 0.f;
+                for (int c = l; c < DK; c += 32) {
+                    const float r = qr[c] - coef * kr[c];
+                    rr = fmaf(r, r, rr);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, off);
+                const float den = rr + qed_eps, nu = den > 0.f ? rsqrtf(den) : 0.f;
+                float *ur = sK + (2 * t + 1) * LK, *er = sE + (2 * t + 1) * LK;
+                for (int c = l; c < DK; c += 32) {
+                    const float u = (qr[c] - coef * kr[c]) * nu;
+                    ur[c] = u;
+                    er[c] *= u;   // c_t . u_t
+                }
+            }
+        }
+        __syncthreads();
+        // ---- cumulative log-decay per channel and the scaled operands
+        if (tid < DK) {
+            const int c = tid;
+            float g = 0.f;
+            for (int t = 0; t < C; ++t) {
+                g += sG[t * LK + c];
+                const float gam = expf(g), inv = expf(-g);
+                sQ[t * LK + c] *= gam;
+                sE[(2 * t) * LK + c] *= gam;
+                sE[(2 * t + 1) * LK + c] *= gam;
+                sK[(2 * t) * LK + c] *= inv;
+                sK[(2 * t + 1) * LK + c] *= inv;
+            }
+            sGC[c] = expf(g);
+        }
+        __syncthreads();
+        // ---- A (strict by token) and P (inclusive by token); overwrite the log-decay
+        for (int idx = tid; idx < R * R; idx += 256) {
+            const int r = idx / R, i = idx % R;
+            float a = 0.f;
+            if ((i >> 1) < (r >> 1))
+                for (int c = 0; c < DK; ++c) a = fmaf(sE[r * LK + c], sK[i * LK + c], a);
+            sA[r * LR + i] = a;
+        }
+        for (int idx = tid; idx < C * R; idx += 256) {
+            const int t = idx / R, i = idx % R;
+            float p = 0.f;
+            if ((i >> 1) <= t)
+                for (int c = 0; c < DK; ++c) p = fmaf(sQ[t * LK + c], sK[i * LK + c], p);
+            sP[t * LR + i] = p;
+        }
+        __syncthreads();
+        // ---- T = (I + A)^{-1}, one column per thread by forward substitution
+        if (tid < R) {
+            const int j = tid;
+            for (int r = 0; r < R; ++r) {
+                float x = (r == j) ? 1.f : 0.f;
+                for (int i = j; i < r; ++i) x = fmaf(-sA[r * LR + i], sT[i * LR + j], x);
+                sT[r * LR + j] = (r < j) ? 0.f : x;
+            }
+        }
+        __syncthreads();
+        // ---- U = T V - T (E S)
+        constexpr int PER = R * NV / 256;
+        float acc[PER];
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            float x = 0.f;
+            for (int i = 0; i <= r; ++i) x = fmaf(sT[r * LR + i], sWV[i * LV + j], x);
+            acc[m] = x;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            sU[r * LV + j] = acc[m];
+            float x = 0.f;
+            for (int c = 0; c < DK; ++c) x = fmaf(sE[r * LK + c], sS[c * LV + j], x);
+            sWV[r * LV + j] = x;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
+            float x = sU[r * LV + j];
+            for (int i = 0; i <= r; ++i) x = fmaf(-sT[r * LR + i], sWV[i * LV + j], x);
+            acc[m] = x;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < PER; ++m) {
+            const int idx = tid + 256 * m;
+            sU[(idx / NV) * LV + idx % NV] = acc[m];
+        }
+        __syncthreads();
+        // ---- O = Q~ S + P U on the token rows
+        for (int idx = tid; idx < C * NV; idx += 256) {
+            const int t = idx / NV, j = idx % NV;
+            float x = 0.f;
+            for (int c = 0; c < DK; ++c) x = fmaf(sQ[t * LK + c], sS[c * LV + j], x);
+            for (int i = 0; i < R; ++i) x = fmaf(sP[t * LR + i], sU[i * LV + j], x);
+            if (t < rows) {
+                const long g = ((tok0 + t) * H + h) * (long)d_v + j0 + j;
+                if constexpr (sizeof(IO) == 4) o[g] = x;
+                else o[g] = __float2bfloat16_rn(x);
+            }
+        }
+        __syncthreads();
+        // ---- S <- diag(Gamma_C) (S + K~^T U)
+        for (int idx = tid; idx < DK * NV; idx += 256) {
+            const int c = idx / NV, j = idx % NV;
+            float x = sS[c * LV + j];
+            for (int i = 0; i < R; ++i) x = fmaf(sK[i * LK + c], sU[i * LV + j], x);
+            sS[c * LV + j] = sGC[c] * x;
+        }
+    }
+    __syncthreads();
+    if (S_T) {
+        for (int idx = tid; idx < DK * NV; idx += 256) {
+            const int c = idx / NV, j = idx % NV;
+            S_T[(head * DK + c) * d_v + j0 + j] = sS[c * LV + j];
+        }
+    }
+}
+
+}  // namespace gdn2

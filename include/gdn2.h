@@ -219,6 +219,39 @@ gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v,
                                   void *stream);
 
 /*
+ * gdn2_chunk_fwd_qed / gdn2_decode_step_qed -- the recurrence with a second,
+ * query-derived erase direction ("The Query Knows What to Forget",
+ * mlsanity 2608.13668, abstract: a direction taken from the query and
+ * orthogonal to the key that cancels what the old state holds along the
+ * query).  The page gives no formula; the reading implemented is
+ *
+ *     r_t = q_t - ((q_t . k_t) / (k_t . k_t)) k_t     (q_t when k_t = 0)
+ *     u_t = r_t / sqrt(r_t . r_t + qed_eps)          (0 when that is 0)
+ *     S_t = (I - k_t (b_t . k_t)^T - u_t (c_t . u_t)^T) diag(alpha_t) S_{t-1}
+ *           + k_t (w_t . v_t)^T,          o_t = S_t^T q_t
+ *
+ *   c       : in, [B, T, H, d_k] (decode: [B, H, d_k]), dtype io, the second
+ *             erase gate (c = 0 gives gdn2_chunk_fwd / gdn2_decode_step up
+ *             to rounding)
+ *   qed_eps : >= 0
+ * Other arguments, layouts, shapes and errors as gdn2_chunk_fwd (value heads
+ * equal key heads, no packing, no fusion) and gdn2_decode_step.  Both run on
+ * CUDA cores with fp32 products; the chunk form takes 32 tokens per chunk
+ * (64 rows of the chunked solve: each token adds its key and its query
+ * direction), so its `chunk` is fixed.
+ */
+gdn2_status_t gdn2_chunk_fwd_qed(const void *q, const void *k, const void *v,
+                                 const void *log_alpha, const void *b, const void *c, const void *w,
+                                 const float *S0, void *o, float *S_T,
+                                 int B, int T, int H, int d_k, int d_v,
+                                 gdn2_io_t io, float qed_eps, void *stream);
+
+gdn2_status_t gdn2_decode_step_qed(const void *q, const void *k, const void *v,
+                                   const void *log_alpha, const void *b, const void *c, const void *w,
+                                   float *S, void *o, int B, int H, int d_k, int d_v,
+                                   gdn2_io_t io, float qed_eps, void *stream);
+
+/*
  * gdn2_device_status -- synchronise `stream`, then read and clear the
  * current device's status word.  Returns GDN2_OK, GDN2_ERR_DEVICE_TIMEOUT if
  * a kernel gave up on a bounded wait since the last call,

@@ -137,3 +137,23 @@ def test_value_heads_and_packing_validation_on_host(L):
     assert chunk_ex(T=0, cu=P(16)) == 0   # no tokens at all, no state: nothing to do
     assert chunk_ex(T=0, HV=0) == 0
     assert chunk_ex(HV=70000, H=1) == 2   # beyond the grid's y extent
+
+
+def test_qed_argument_validation_on_host(L):
+    """The second-erase entry points check their arguments before touching the device."""
+    P, F = ctypes.c_void_p, ctypes.c_float
+    p = P(16)
+
+    def chunk_qed(c=p, eps=1e-6, T=64, dk=64, dv=64, ptr=p):
+        return L.gdn2_chunk_fwd_qed(ptr, p, p, p, p, c, p, None, p, None, 1, T, 1, dk, dv, 1, F(eps), None)
+
+    def decode_qed(c=p, eps=1e-6, dk=64, dv=64):
+        return L.gdn2_decode_step_qed(p, p, p, p, p, c, p, p, p, 1, 1, dk, dv, 1, F(eps), None)
+
+    for call in (chunk_qed, decode_qed):
+        assert call(c=None) == 1            # no second gate
+        assert call(eps=-1.0) == 1          # negative epsilon
+        assert call(c=P(20)) == 3           # misaligned gate
+        assert call(dk=96) == 2
+        assert call(dv=96) == 2
+    assert chunk_qed(T=0, ptr=None, c=None) == 0   # empty sequence, no state: nothing to do

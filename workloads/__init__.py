@@ -152,6 +152,15 @@ def draw_raw(B: int, T: int, H: int, d_k: int, d_v: int, *, seed: int,
     return out
 
 
+def draw_qed_gate(lead, d_k: int, *, seed: int, dtype=torch.bfloat16, device="cpu") -> torch.Tensor:
+    """The second erase gate c of the query-derived erase direction: sigmoid(N(0,1))
+    per key channel, shape lead + (d_k,), from its own generator (the other inputs'
+    draws are unchanged)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    c = torch.sigmoid(torch.randn(*lead, d_k, generator=g, dtype=torch.float32, device=device))
+    return c.to(dtype).contiguous()
+
+
 def packed_lengths(n: int, mean: int, *, seed: int, min_len: int = 0) -> list:
     """Lengths of ``n`` packed sequences: a geometric-like mix around ``mean``
     tokens (exponential draw, rounded), at least ``min_len``.  Used for the
