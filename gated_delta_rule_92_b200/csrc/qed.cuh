@@ -273,85 +273,194 @@ chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
             sGC[c] = expf(g);
         }
         __syncthreads();
-        // ---- A (strict by token) and P (inclusive by token); overwrite the log-decay
-        for (int idx = tid; idx < R * R; idx += 256) {
-            const int r = idx / R, i = idx % R;
-            float a = 0.f;
-            if ((i >> 1) < (r >> 1))
-                for (int c = 0; c < DK; ++c) a = fmaf(sE[r * LK + c], sK[i * LK + c], a);
-            sA[r * LR + i] = a;
-        }
-        for (int idx = tid; idx < C * R; idx += 256) {
-            const int t = idx / R, i = idx % R;
-            float p = 0.f;
-            if ((i >> 1) <= t)
-                for (int c = 0; c < DK; ++c) p = fmaf(sQ[t * LK + c], sK[i * LK + c], p);
-            sP[t * LR + i] = p;
+        // ---- A (strict by token) and P (inclusive by token); overwrite the log-decay.
+        // Register tiles: A in 4 x 4 (thread: rows 4 (tid / 16).., columns 4 (tid % 16)..),
+        // P in 2 x 4; a tile wholly above the token diagonal is zero without work.
+        {
+            const int rt = tid >> 4, ct = tid & 15;
+            float acc[4][4] = {};
+            if (ct <= rt) {
+                for (int c = 0; c < DK; ++c) {
+                    float e[4], kk[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        e[x] = sE[(4 * rt + x) * LK + c];
+                        kk[x] = sK[(4 * ct + x) * LK + c];
+                    }
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(e[x], kk[y], acc[x][y]);
+                }
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const int r = 4 * rt + x, i = 4 * ct + y;
+                    sA[r * LR + i] = ((i >> 1) < (r >> 1)) ? acc[x][y] : 0.f;
+                }
+            float pc[2][4] = {};
+            if (2 * ct <= 2 * rt + 1) {   // some column token <= some row token
+                for (int c = 0; c < DK; ++c) {
+                    float qq[2], kk[4];
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) qq[x] = sQ[(2 * rt + x) * LK + c];
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) kk[y] = sK[(4 * ct + y) * LK + c];
+#pragma unroll
+                    for (int x = 0; x < 2; ++x)
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) pc[x][y] = fmaf(qq[x], kk[y], pc[x][y]);
+                }
+            }
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const int t = 2 * rt + x, i = 4 * ct + y;
+                    sP[t * LR + i] = ((i >> 1) <= t) ? pc[x][y] : 0.f;
+                }
         }
         __syncthreads();
-        // ---- T = (I + A)^{-1}, one column per thread by forward substitution
-        if (tid < R) {
-            const int j = tid;
-            for (int r = 0; r < R; ++r) {
-                float x = (r == j) ? 1.f : 0.f;
-                for (int i = j; i < r; ++i) x = fmaf(-sA[r * LR + i], sT[i * LR + j], x);
-                sT[r * LR + j] = (r < j) ? 0.f : x;
+        // ---- T = (I + A)^{-1}: column j by 4 threads (rows r = 4 m + qd), right-looking:
+        // once row i of the column is final it is broadcast and every later row takes
+        // its term; rows above j stay zero by themselves
+        {
+            const int j = tid >> 2, qd = tid & 3, lane = tid & 31;
+            float acc[R / 4];
+#pragma unroll
+            for (int m = 0; m < R / 4; ++m) acc[m] = (4 * m + qd == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float xi = __shfl_sync(0xffffffffu, acc[i >> 2], (lane & ~3) | (i & 3));
+#pragma unroll
+                for (int m = i >> 2; m < R / 4; ++m) {
+                    const int r = 4 * m + qd;
+                    if (r > i) acc[m] = fmaf(-sA[r * LR + i], xi, acc[m]);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < R / 4; ++m) sT[(4 * m + qd) * LR + j] = acc[m];
+        }
+        __syncthreads();
+        // ---- U = T V - T (E S), 4 x 4 register tiles of the R x NV result
+        {
+            const int rt = tid >> 4, ct = tid & 15;
+            float u1[4][4] = {}, es[4][4] = {};
+            for (int i = 0; i < 4 * rt + 4; ++i) {   // T is lower triangular
+                float tt[4], vv[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) tt[x] = sT[(4 * rt + x) * LR + i];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) vv[y] = sWV[i * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) u1[x][y] = fmaf(tt[x], vv[y], u1[x][y]);
+            }
+            for (int c = 0; c < DK; ++c) {
+                float e[4], ss[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) e[x] = sE[(4 * rt + x) * LK + c];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) ss[y] = sS[c * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) es[x][y] = fmaf(e[x], ss[y], es[x][y]);
+            }
+            __syncthreads();   // everyone has read the values before E S replaces them
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    sU[(4 * rt + x) * LV + 4 * ct + y] = u1[x][y];
+                    sWV[(4 * rt + x) * LV + 4 * ct + y] = es[x][y];
+                }
+            __syncthreads();
+            for (int i = 0; i < 4 * rt + 4; ++i) {
+                float tt[4], vv[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) tt[x] = sT[(4 * rt + x) * LR + i];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) vv[y] = sWV[i * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) u1[x][y] = fmaf(-tt[x], vv[y], u1[x][y]);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) sU[(4 * rt + x) * LV + 4 * ct + y] = u1[x][y];
+        }
+        __syncthreads();
+        // ---- O = Q~ S + P U on the token rows, 2 x 4 register tiles
+        {
+            const int rt = tid >> 4, ct = tid & 15;
+            float ov[2][4] = {};
+            for (int c = 0; c < DK; ++c) {
+                float qq[2], ss[4];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) qq[x] = sQ[(2 * rt + x) * LK + c];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) ss[y] = sS[c * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) ov[x][y] = fmaf(qq[x], ss[y], ov[x][y]);
+            }
+            for (int i = 0; i < 4 * rt + 4; ++i) {   // P is zero past the row's token
+                float pp[2], uu[4];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) pp[x] = sP[(2 * rt + x) * LR + i];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) uu[y] = sU[i * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) ov[x][y] = fmaf(pp[x], uu[y], ov[x][y]);
+            }
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int t = 2 * rt + x;
+                if (t < rows) {
+                    const long g = ((tok0 + t) * H + h) * (long)d_v + j0 + 4 * ct;
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        if constexpr (sizeof(IO) == 4) o[g + y] = ov[x][y];
+                        else o[g + y] = __float2bfloat16_rn(ov[x][y]);
+                    }
+                }
             }
         }
         __syncthreads();
-        // ---- U = T V - T (E S)
-        constexpr int PER = R * NV / 256;
-        float acc[PER];
+        // ---- S <- diag(Gamma_C) (S + K~^T U), 4 x 8 register tiles of the DK x NV state
+        for (int tile = tid; tile < (DK / 4) * (NV / 8); tile += 256) {
+            const int rt = tile / (NV / 8), ct = tile % (NV / 8);
+            float sv[4][8];
 #pragma unroll
-        for (int m = 0; m < PER; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            float x = 0.f;
-            for (int i = 0; i <= r; ++i) x = fmaf(sT[r * LR + i], sWV[i * LV + j], x);
-            acc[m] = x;
-        }
-        __syncthreads();
+            for (int x = 0; x < 4; ++x)
 #pragma unroll
-        for (int m = 0; m < PER; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            sU[r * LV + j] = acc[m];
-            float x = 0.f;
-            for (int c = 0; c < DK; ++c) x = fmaf(sE[r * LK + c], sS[c * LV + j], x);
-            sWV[r * LV + j] = x;
-        }
-        __syncthreads();
+                for (int y = 0; y < 8; ++y) sv[x][y] = sS[(4 * rt + x) * LV + 8 * ct + y];
+            for (int i = 0; i < R; ++i) {
+                float kk[4], uu[8];
 #pragma unroll
-        for (int m = 0; m < PER; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            float x = sU[r * LV + j];
-            for (int i = 0; i <= r; ++i) x = fmaf(-sT[r * LR + i], sWV[i * LV + j], x);
-            acc[m] = x;
-        }
-        __syncthreads();
+                for (int x = 0; x < 4; ++x) kk[x] = sK[i * LK + 4 * rt + x];
 #pragma unroll
-        for (int m = 0; m < PER; ++m) {
-            const int idx = tid + 256 * m;
-            sU[(idx / NV) * LV + idx % NV] = acc[m];
-        }
-        __syncthreads();
-        // ---- O = Q~ S + P U on the token rows
-        for (int idx = tid; idx < C * NV; idx += 256) {
-            const int t = idx / NV, j = idx % NV;
-            float x = 0.f;
-            for (int c = 0; c < DK; ++c) x = fmaf(sQ[t * LK + c], sS[c * LV + j], x);
-            for (int i = 0; i < R; ++i) x = fmaf(sP[t * LR + i], sU[i * LV + j], x);
-            if (t < rows) {
-                const long g = ((tok0 + t) * H + h) * (long)d_v + j0 + j;
-                if constexpr (sizeof(IO) == 4) o[g] = x;
-                else o[g] = __float2bfloat16_rn(x);
+                for (int y = 0; y < 8; ++y) uu[y] = sU[i * LV + 8 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 8; ++y) sv[x][y] = fmaf(kk[x], uu[y], sv[x][y]);
             }
-        }
-        __syncthreads();
-        // ---- S <- diag(Gamma_C) (S + K~^T U)
-        for (int idx = tid; idx < DK * NV; idx += 256) {
-            const int c = idx / NV, j = idx % NV;
-            float x = sS[c * LV + j];
-            for (int i = 0; i < R; ++i) x = fmaf(sK[i * LK + c], sU[i * LV + j], x);
-            sS[c * LV + j] = sGC[c] * x;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float gcx = sGC[4 * rt + x];
+#pragma unroll
+                for (int y = 0; y < 8; ++y) sS[(4 * rt + x) * LV + 8 * ct + y] = gcx * sv[x][y];
+            }
         }
     }
     __syncthreads();
