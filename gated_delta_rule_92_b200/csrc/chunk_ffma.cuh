@@ -150,80 +150,177 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
             sGC[c] = expf(g);
         }
         __syncthreads();
-        // ---- A (strictly lower) and P (lower, inclusive); overwrite the log-decay
-        for (int idx = tid; idx < C * C; idx += 256) {
-            const int r = idx / C, i = idx % C;
-            float a = 0.f, p = 0.f;
-            if (i <= r) {
+        // ---- A (strictly lower) and P (lower, inclusive); overwrite the log-decay.
+        // Register tiles of TC x TC (thread: rows TC (tid / 16).., columns TC (tid % 16)..);
+        // a tile wholly above the diagonal is zero without work.
+        constexpr int TC = C / 16;
+        {
+            const int rt = tid >> 4, ct = tid & 15;
+            float aa[TC][TC] = {}, pp[TC][TC] = {};
+            if (ct <= rt) {
                 for (int c = 0; c < DK; ++c) {
-                    const float kt = sK[i * LK + c];
-                    a = fmaf(sE[r * LK + c], kt, a);
-                    p = fmaf(sQ[r * LK + c], kt, p);
+                    float e[TC], qq[TC], kk[TC];
+#pragma unroll
+                    for (int x = 0; x < TC; ++x) {
+                        e[x] = sE[(TC * rt + x) * LK + c];
+                        qq[x] = sQ[(TC * rt + x) * LK + c];
+                        kk[x] = sK[(TC * ct + x) * LK + c];
+                    }
+#pragma unroll
+                    for (int x = 0; x < TC; ++x)
+#pragma unroll
+                        for (int y = 0; y < TC; ++y) {
+                            aa[x][y] = fmaf(e[x], kk[y], aa[x][y]);
+                            pp[x][y] = fmaf(qq[x], kk[y], pp[x][y]);
+                        }
                 }
             }
-            sA[r * LC + i] = (i < r) ? a : 0.f;
-            sP[r * LC + i] = p;
+#pragma unroll
+            for (int x = 0; x < TC; ++x)
+#pragma unroll
+                for (int y = 0; y < TC; ++y) {
+                    const int r = TC * rt + x, i = TC * ct + y;
+                    sA[r * LC + i] = (i < r) ? aa[x][y] : 0.f;
+                    sP[r * LC + i] = (i <= r) ? pp[x][y] : 0.f;
+                }
         }
         __syncthreads();
-        // ---- T = (I + A)^{-1}, one column per thread by forward substitution
-        if (tid < C) {
-            const int j = tid;
-            for (int r = 0; r < C; ++r) {
-                float x = (r == j) ? 1.f : 0.f;
-                for (int i = j; i < r; ++i) x = fmaf(-sA[r * LC + i], sT[i * LC + j], x);
-                sT[r * LC + j] = (r < j) ? 0.f : x;
+        // ---- T = (I + A)^{-1}: column j by 256 / C threads (rows r = TPC m + qd),
+        // right-looking: once row i of the column is final it is broadcast from its
+        // owner and every later row takes its term; rows above j stay zero
+        {
+            constexpr int TPC = 256 / C, RPC = C / TPC;
+            const int j = tid / TPC, qd = tid % TPC, lane = tid & 31;
+            float acc[RPC];
+#pragma unroll
+            for (int m = 0; m < RPC; ++m) acc[m] = (TPC * m + qd == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < C; ++i) {
+                const float xi = __shfl_sync(0xffffffffu, acc[i / TPC], (lane & ~(TPC - 1)) | (i % TPC));
+#pragma unroll
+                for (int m = i / TPC; m < RPC; ++m) {
+                    const int r = TPC * m + qd;
+                    if (r > i) acc[m] = fmaf(-sA[r * LC + i], xi, acc[m]);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < RPC; ++m) sT[(TPC * m + qd) * LC + j] = acc[m];
+        }
+        __syncthreads();
+        // ---- U = T (W.V) - T (E S), TC x 4 register tiles of the C x NV result
+        {
+            const int rt = tid >> 4, ct = tid & 15;
+            float u1[TC][4] = {}, es[TC][4] = {};
+            for (int i = 0; i < TC * rt + TC; ++i) {   // T is lower triangular
+                float tt[TC], vv[4];
+#pragma unroll
+                for (int x = 0; x < TC; ++x) tt[x] = sT[(TC * rt + x) * LC + i];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) vv[y] = sWV[i * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < TC; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) u1[x][y] = fmaf(tt[x], vv[y], u1[x][y]);
+            }
+            for (int c = 0; c < DK; ++c) {
+                float e[TC], ss[4];
+#pragma unroll
+                for (int x = 0; x < TC; ++x) e[x] = sE[(TC * rt + x) * LK + c];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) ss[y] = sS[c * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < TC; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) es[x][y] = fmaf(e[x], ss[y], es[x][y]);
+            }
+            __syncthreads();   // everyone has read W.V before E S replaces it
+#pragma unroll
+            for (int x = 0; x < TC; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) sWV[(TC * rt + x) * LV + 4 * ct + y] = es[x][y];
+            __syncthreads();
+            for (int i = 0; i < TC * rt + TC; ++i) {
+                float tt[TC], vv[4];
+#pragma unroll
+                for (int x = 0; x < TC; ++x) tt[x] = sT[(TC * rt + x) * LC + i];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) vv[y] = sWV[i * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < TC; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) u1[x][y] = fmaf(-tt[x], vv[y], u1[x][y]);
+            }
+#pragma unroll
+            for (int x = 0; x < TC; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) sU[(TC * rt + x) * LV + 4 * ct + y] = u1[x][y];
+        }
+        __syncthreads();
+        // ---- O = Q~ S + P U, TC x 4 register tiles
+        {
+            const int rt = tid >> 4, ct = tid & 15;
+            float ov[TC][4] = {};
+            for (int c = 0; c < DK; ++c) {
+                float qq[TC], ss[4];
+#pragma unroll
+                for (int x = 0; x < TC; ++x) qq[x] = sQ[(TC * rt + x) * LK + c];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) ss[y] = sS[c * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < TC; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) ov[x][y] = fmaf(qq[x], ss[y], ov[x][y]);
+            }
+            for (int i = 0; i < TC * rt + TC; ++i) {   // P is lower triangular
+                float pv[TC], uu[4];
+#pragma unroll
+                for (int x = 0; x < TC; ++x) pv[x] = sP[(TC * rt + x) * LC + i];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) uu[y] = sU[i * LV + 4 * ct + y];
+#pragma unroll
+                for (int x = 0; x < TC; ++x)
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) ov[x][y] = fmaf(pv[x], uu[y], ov[x][y]);
+            }
+#pragma unroll
+            for (int x = 0; x < TC; ++x) {
+                const int r = TC * rt + x;
+                if (r < rows) {
+                    const long g = ((tok0 + r) * HV + hv) * d_v + j0 + 4 * ct;
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        if constexpr (sizeof(IO) == 4) o[g + y] = ov[x][y];
+                        else o[g + y] = __float2bfloat16_rn(ov[x][y]);
+                    }
+                }
             }
         }
         __syncthreads();
-        // ---- T (W.V) -> sU ;  E S -> sWV (W.V is dead afterwards)
-        float acc[C * NV / 256];
-        for (int m = 0; m < C * NV / 256; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            float x = 0.f;
-            for (int i = 0; i <= r; ++i) x = fmaf(sT[r * LC + i], sWV[i * LV + j], x);
-            acc[m] = x;
-        }
-        __syncthreads();
-        for (int m = 0; m < C * NV / 256; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            sU[r * LV + j] = acc[m];
-            float x = 0.f;
-            for (int c = 0; c < DK; ++c) x = fmaf(sE[r * LK + c], sS[c * LV + j], x);
-            sWV[r * LV + j] = x;
-        }
-        __syncthreads();
-        // ---- U = T (W.V) - T (E S)
-        for (int m = 0; m < C * NV / 256; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            float x = sU[r * LV + j];
-            for (int i = 0; i <= r; ++i) x = fmaf(-sT[r * LC + i], sWV[i * LV + j], x);
-            acc[m] = x;
-        }
-        __syncthreads();
-        for (int m = 0; m < C * NV / 256; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            sU[r * LV + j] = acc[m];
-        }
-        __syncthreads();
-        // ---- O = Q~ S + P U
-        for (int m = 0; m < C * NV / 256; ++m) {
-            const int idx = tid + 256 * m, r = idx / NV, j = idx % NV;
-            float x = 0.f;
-            for (int c = 0; c < DK; ++c) x = fmaf(sQ[r * LK + c], sS[c * LV + j], x);
-            for (int i = 0; i <= r; ++i) x = fmaf(sP[r * LC + i], sU[i * LV + j], x);
-            const long g = ((tok0 + r) * HV + hv) * d_v + j0 + j;
-            if (r < rows) {
-                if constexpr (sizeof(IO) == 4) o[g] = x;
-                else o[g] = __float2bfloat16_rn(x);
+        // ---- S <- diag(gamma_C) (S + K~^T U), 4 x 8 register tiles of the DK x NV state
+        for (int tile = tid; tile < (DK / 4) * (NV / 8); tile += 256) {
+            const int rt = tile / (NV / 8), ct = tile % (NV / 8);
+            float sv[4][8];
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 8; ++y) sv[x][y] = sS[(4 * rt + x) * LV + 8 * ct + y];
+            for (int i = 0; i < C; ++i) {
+                float kk[4], uu[8];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) kk[x] = sK[i * LK + 4 * rt + x];
+#pragma unroll
+                for (int y = 0; y < 8; ++y) uu[y] = sU[i * LV + 8 * ct + y];
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+#pragma unroll
+                    for (int y = 0; y < 8; ++y) sv[x][y] = fmaf(kk[x], uu[y], sv[x][y]);
             }
-        }
-        __syncthreads();
-        // ---- S <- diag(gamma_C) (S + K~^T U)
-        for (int idx = tid; idx < DK * NV; idx += 256) {
-            const int c = idx / NV, j = idx % NV;
-            float x = sS[c * LV + j];
-            for (int i = 0; i < C; ++i) x = fmaf(sK[i * LK + c], sU[i * LV + j], x);
-            sS[c * LV + j] = sGC[c] * x;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float gcx = sGC[4 * rt + x];
+#pragma unroll
+                for (int y = 0; y < 8; ++y) sS[(4 * rt + x) * LV + 8 * ct + y] = gcx * sv[x][y];
+            }
         }
     }
     __syncthreads();
