@@ -19,10 +19,13 @@
 //              place in the TMA tiles and exp(G_C) for the state update
 //       W.V    in place in the v tile
 //       MMA1   [Q~; E] K~^T -> TMEM (rows 0-63 P', rows 64-127 A')
-//       solve  T = (I + A)^{-1} in fp32 on CUDA cores (16x16 diagonal blocks
-//              by forward substitution, off-diagonal blocks by block products)
+//       solve  T = (I + A)^{-1} in fp32 (16x16 diagonal blocks by forward
+//              substitution, off-diagonal blocks by tf32 mma.sync block
+//              products), each block of T written to its bf16 MMA tile as soon
+//              as it is final
 //       MMA2   [. ; T] E       -> rows 64-127 = T E, back to bf16 over E
-//       MMA3   [. ; T] (W.V)   -> rows 64-127 = T (W.V)
+//       MMA3   [. ; T] (W.V)   -> rows 64-127 = T (W.V); its commits free the
+//              v tile and hand T (W.V) to the chain
 //     as a two-stage pipeline: warps 0-3 solve chunk m while warps 4-7 run
 //     the prep of chunk m+1 (exp(G_C) is triple buffered for that)
 //   chain warps 8-11 chunk m-1, the sequential state pass:
