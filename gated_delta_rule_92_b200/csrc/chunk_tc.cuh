@@ -354,20 +354,34 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
             sum[3] += c4.w;
         }
     }
-    // rows in batches: the tiles are rewritten in place, so loads of a batch
-    // cannot be hoisted above the previous batch's stores by the compiler
+    // rows in batches of RB, software-pipelined: the tiles are rewritten in
+    // place, so the compiler keeps every load behind the earlier stores; the
+    // next batch's loads are therefore issued here before this batch is stored
+    // (they read other rows)
     constexpr int RB = 2;
+    uint2 qw[RB], kw[RB], bw[RB];
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+        const int oj = off(hb * R + j);
+        qw[j] = *reinterpret_cast<const uint2 *>(q_t + oj);
+        kw[j] = *reinterpret_cast<const uint2 *>(k_t + oj);
+        bw[j] = *reinterpret_cast<const uint2 *>(e_t + oj);
+    }
 #pragma unroll
     for (int i0 = 0; i0 < R; i0 += RB) {
-        uint2 qw[RB], kw[RB], bw[RB];
+        uint2 qn[RB], kn[RB], bn[RB];
+        if (i0 + RB < R) {
+#pragma unroll
+            for (int j = 0; j < RB; ++j) {
+                const int oj = off(hb * R + i0 + RB + j);
+                qn[j] = *reinterpret_cast<const uint2 *>(q_t + oj);
+                kn[j] = *reinterpret_cast<const uint2 *>(k_t + oj);
+                bn[j] = *reinterpret_cast<const uint2 *>(e_t + oj);
+            }
+        }
         int o[RB];
 #pragma unroll
-        for (int j = 0; j < RB; ++j) {
-            o[j] = off(hb * R + i0 + j);
-            qw[j] = *reinterpret_cast<const uint2 *>(q_t + o[j]);
-            kw[j] = *reinterpret_cast<const uint2 *>(k_t + o[j]);
-            bw[j] = *reinterpret_cast<const uint2 *>(e_t + o[j]);
-        }
+        for (int j = 0; j < RB; ++j) o[j] = off(hb * R + i0 + j);
 #pragma unroll
         for (int j = 0; j < RB; ++j) {
             float rq = 1.f, rk = 1.f, bs = 1.f;
@@ -406,6 +420,14 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
             *reinterpret_cast<uint2 *>(q_t + o[j]) = make_uint2(oq[0], oq[1]);
             *reinterpret_cast<uint2 *>(e_t + o[j]) = make_uint2(oe[0], oe[1]);
             *reinterpret_cast<uint2 *>(k_t + o[j]) = make_uint2(ok[0], ok[1]);
+        }
+        if (i0 + RB < R) {
+#pragma unroll
+            for (int j = 0; j < RB; ++j) {
+                qw[j] = qn[j];
+                kw[j] = kn[j];
+                bw[j] = bn[j];
+            }
         }
     }
     if (hb == NB - 1) {
