@@ -122,29 +122,29 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// One warp: C (16 x 16, row stride LDA) = sign * Am (16 x K) Bm (K x 16), all in
-// fp32 shared memory with row stride LDA, products in tf32 on the tensor cores.
-// With a tile `tt`, C also goes, rounded to bf16, to rows trow.., columns
-// tcol.. of that 128-byte-swizzled 64 x 64 tile; keep_fp32 = false leaves
-// the fp32 copy out.
-template <int LDA, int K>
+// One warp: C (16 x 8 NNT, row stride LDA) = sign * Am (16 x K) Bm (K x 8 NNT),
+// all in fp32 shared memory with row stride LDA, products in tf32 on the
+// tensor cores.  With a tile `tt`, C also goes, rounded to bf16, to rows
+// trow.., columns tcol.. of that 128-byte-swizzled 64 x 64 tile; keep_fp32 =
+// false leaves the fp32 copy out.
+template <int LDA, int K, int NNT = 2>
 __device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, float *Cm, float sign, int lane,
                                             uint8_t *tt = nullptr, int trow = 0, int tcol = 0,
                                             bool keep_fp32 = true) {
     const int g = lane >> 2, q = lane & 3;
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float acc[NNT][4] = {};
 #pragma unroll
     for (int k0 = 0; k0 < K; k0 += 8) {
         const uint32_t a[4] = {to_tf32(Am[g * LDA + k0 + q]), to_tf32(Am[(g + 8) * LDA + k0 + q]),
                                to_tf32(Am[g * LDA + k0 + q + 4]), to_tf32(Am[(g + 8) * LDA + k0 + q + 4])};
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < NNT; ++nt) {
             const uint32_t bf[2] = {to_tf32(Bm[(k0 + q) * LDA + 8 * nt + g]), to_tf32(Bm[(k0 + q + 4) * LDA + 8 * nt + g])};
             mma_tf32(acc[nt], a, bf);
         }
     }
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < NNT; ++nt) {
         if (keep_fp32) {
             *reinterpret_cast<float2 *>(Cm + g * LDA + 8 * nt + 2 * q) = make_float2(sign * acc[nt][0], sign * acc[nt][1]);
             *reinterpret_cast<float2 *>(Cm + (g + 8) * LDA + 8 * nt + 2 * q) =
@@ -201,16 +201,17 @@ __device__ __forceinline__ void unit_lower_inverse64(float *sA, uint8_t *tt, int
         }
         named_bar(bar, 128);
     }
-    if (w < 2) {   // 2. 16 -> 32, warp p = w; Y_p in rows 16p.., cols 32..
-        const int R = 32 * w;
-        float *Y = sA + (16 * w) * LDA + 32;
-        warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R, sA + R * LDA + R, Y, 1.f, lane);
-        __syncwarp();
-        warp_gemm16<LDA, 16>(sA + (R + 16) * LDA + R + 16, Y, sA + (R + 16) * LDA + R, -1.f, lane, tt, R + 16, R);
-    } else {       // the diagonal blocks to the tile, 8 columns a thread, rows 8.. (0-7 come last)
-        for (int c = t - 64; c < 128; c += 64) {
+    {   // 2. 16 -> 32: pair p = w % 2 (Y_p in rows 16p.., cols 32..), 8-column half w / 2
+        const int pr = w & 1, half = 8 * (w >> 1), R = 32 * pr;
+        float *Y = sA + (16 * pr) * LDA + 32;
+        warp_gemm16<LDA, 16, 1>(sA + (R + 16) * LDA + R, sA + R * LDA + R + half, Y + half, 1.f, lane);
+        named_bar(bar, 128);   // both halves of each Y_p are written
+        warp_gemm16<LDA, 16, 1>(sA + (R + 16) * LDA + R + 16, Y + half, sA + (R + 16) * LDA + R + half, -1.f, lane,
+                                tt, R + 16, R + half);
+        // the diagonal blocks to the tile, 8 columns a thread, rows 8.. (0-7 come last)
+        if (t < 128 - 16) {
+            const int c = t + 16;   // 8-column pieces 16.. of the four blocks (rows 0-7 of block 0 skipped)
             const int b = c >> 5, row = 16 * b + ((c >> 1) & 15), col0 = 16 * b + 8 * (c & 1);
-            if (row < 8) continue;
             const float4 a = *reinterpret_cast<const float4 *>(sA + row * LDA + col0);
             const float4 d = *reinterpret_cast<const float4 *>(sA + row * LDA + col0 + 4);
             *reinterpret_cast<uint4 *>(tt + sw128_chunk(row, col0 >> 3)) =
