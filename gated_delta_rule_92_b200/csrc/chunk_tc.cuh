@@ -161,7 +161,7 @@ __device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, fl
 // T = (I + A)^{-1} for a strictly lower 64x64 A held in fp32 in sA (row
 // stride LDA), in place, by 128 threads (4 warps):
 //   1. each 16x16 diagonal block D_k = (I + A_kk)^{-1} by right-looking
-//      forward substitution in fp32, one column per thread (threads 0-63);
+//      forward substitution in fp32, warp k for block k, two lanes a column;
 //   2. 16 -> 32: T_{2p+1,2p} = -D_{2p+1} (A_{2p+1,2p} D_{2p}), p = 0, 1
 //      (warp p);
 //   3. 32 -> 64: T_ba = -T_b (A_ba T_a) with a = rows/cols 0-31, b = 32-63
@@ -179,26 +179,26 @@ __device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, fl
 template <int LDA>
 __device__ __forceinline__ void unit_lower_inverse64(float *sA, uint8_t *tt, int t, int bar) {
     const int w = t >> 5, lane = t & 31;
-    {   // 1. diagonal blocks
-        float x[16];
-        const int R = (t >> 4) * 16, j = t & 15;
-        if (t < 64) {
-            const float *blk = sA + R * LDA + R;
-            float sacc[16];
+    {   // 1. diagonal blocks: warp b takes block b; lanes 2j and 2j + 1 share column j
+        // (rows of parity lane % 2), right-looking: row i of the column is final
+        // once the rows above have applied their terms, and is broadcast
+        const int R = 16 * w, j = lane >> 1, hh = lane & 1;
+        const float *blk = sA + R * LDA + R;
+        float acc[8];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sacc[r] = (r == j) ? 1.f : 0.f;
+        for (int m = 0; m < 8; ++m) acc[m] = (2 * m + hh == j) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                x[i] = sacc[i];
+        for (int i = 0; i < 16; ++i) {
+            const float xi = __shfl_sync(0xffffffffu, acc[i >> 1], (lane & ~1) | (i & 1));
 #pragma unroll
-                for (int r = i + 1; r < 16; ++r) sacc[r] = fmaf(-blk[r * LDA + i], x[i], sacc[r]);
+            for (int m = i >> 1; m < 8; ++m) {
+                const int r = 2 * m + hh;
+                if (r > i) acc[m] = fmaf(-blk[r * LDA + i], xi, acc[m]);
             }
         }
-        named_bar(bar, 128);
-        if (t < 64) {
+        named_bar(bar, 128);   // every column has read A's block before D overwrites it
 #pragma unroll
-            for (int r = 0; r < 16; ++r) sA[(R + r) * LDA + R + j] = x[r];
-        }
+        for (int m = 0; m < 8; ++m) sA[(R + 2 * m + hh) * LDA + R + j] = acc[m];
         named_bar(bar, 128);
     }
     {   // 2. 16 -> 32: pair p = w % 2 (Y_p in rows 16p.., cols 32..), 8-column half w / 2
