@@ -475,7 +475,8 @@ template <int DK, int NV, bool PREP = false, bool EPI = false, bool VARLEN = fal
 __global__ void __launch_bounds__(kTcThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_w, const __nv_bfloat16 *__restrict__ la,
+                    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o,
+                    const __nv_bfloat16 *__restrict__ la,
                     const float *__restrict__ S0,
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int T, int H, int HV, int d_v,
                     const int *__restrict__ cu_seqlens, unsigned long long wait_ns, const FuseArgs fz) {
@@ -871,6 +872,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     umma_bf16(t_X, sdesc_sw128(sb + OQE + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                               sdesc_sw128(sb + Cfg::OFF_S + ks * 2048, 16384, 1024), ids, ks > 0 ? 1u : 0u);
                 umma_commit(bc1);
+                if (!EPI) bulk_wait_read_all();   // the previous O store has read the U tile
             }
             {
                 bool ok = mbar_wait(bc1, ph1, wait_ns);
@@ -962,7 +964,27 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
             tc_fence_after();
-            if ((warp & 3) < 2) {
+            // O leaves through the U tile (free once MMA_o has run) and one TMA store,
+            // except on the partial last chunk of a packed sequence, whose rows past
+            // the end belong to the next sequence
+            const bool o_tma = !EPI && (!VARLEN || (n + 1) * 64 <= len);
+            if ((warp & 3) < 2 && o_tma) {
+                const int r = t;   // output row r (TMEM lanes 0-63)
+#pragma unroll 1
+                for (int jc = 0; jc < NV / 32; ++jc) {
+                    float x[32];
+                    tmem_ld32(t_X + lane_q + jc * 32, x);
+                    const uint32_t tile = sb + Cfg::OFF_U + ((jc * 32) >> 6) * 8192u;
+                    const uint32_t ch0 = ((jc * 32) & 63) >> 3;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int e = 8 * q4;
+                        st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(x[e], x[e + 1]),
+                                     pack_bf16x2(x[e + 2], x[e + 3]), pack_bf16x2(x[e + 4], x[e + 5]),
+                                     pack_bf16x2(x[e + 6], x[e + 7]));
+                    }
+                }
+            } else if ((warp & 3) < 2) {
                 const int r = t;   // output row r (TMEM lanes 0-63); rows past T are padding
                 const bool valid = n * 64 + r < len;
                 const long orow_off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0;
@@ -1052,9 +1074,18 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(2, kChainThreads);
-            if (t == 0) mbar_arrive(&empty_pg[s]);
+            if (t == 0) {
+                mbar_arrive(&empty_pg[s]);
+                if (o_tma) {   // rows past T lie outside the tensor and are not written
+#pragma unroll
+                    for (int vb = 0; vb < Cfg::VB; ++vb)
+                        tma_store_4d(&tm_o, smem + Cfg::OFF_U + vb * 8192, j0 + vb * 64, hv, tma_t0 + n * 64, tma_b);
+                    bulk_commit_group();
+                }
+            }
         }
         if (t == 0) {
+            bulk_wait_all();
             umma_commit(&drain[1]);
             mbar_wait(&drain[1], 0u, wait_ns);
         }

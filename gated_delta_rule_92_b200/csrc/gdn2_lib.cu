@@ -93,14 +93,15 @@ gdn2_status_t launch_rmsnorm(void *o, const void *g, const float *weight, long r
 
 template <int DK, int NV, bool PREP, bool EPI, bool VARLEN>
 gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
-                               const CUtensorMap &tv, const CUtensorMap &tw, const void *la, const float *S0,
+                               const CUtensorMap &tv, const CUtensorMap &tw, const CUtensorMap &to, const void *la,
+                               const float *S0,
                                void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz) {
     using Cfg = TcCfg<DK, NV>;
     auto kern = chunk_fwd_tc_kernel<DK, NV, PREP, EPI, VARLEN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
     dim3 grid(sh.d_v / NV, sh.HV, sh.B);
-    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, static_cast<const __nv_bfloat16 *>(la),
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, to, static_cast<const __nv_bfloat16 *>(la),
                                                     S0, static_cast<__nv_bfloat16 *>(o), S_T, sh.T, sh.H, sh.HV,
                                                     sh.d_v, sh.cu, kWaitNs, fz);
     return from_cuda(cudaGetLastError());
@@ -110,21 +111,22 @@ gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, con
 // equal-length one has none of that code.
 template <int DK, int NV, bool PREP, bool EPI>
 gdn2_status_t launch_tc_seq(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
-                            const CUtensorMap &tv, const CUtensorMap &tw, const void *la, const float *S0,
-                            void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz) {
-    if (sh.cu) return launch_tc_kernel<DK, NV, PREP, EPI, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, fz);
-    return launch_tc_kernel<DK, NV, PREP, EPI, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, fz);
+                            const CUtensorMap &tv, const CUtensorMap &tw, const CUtensorMap &to, const void *la,
+                            const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
+                            const FuseArgs &fz) {
+    if (sh.cu) return launch_tc_kernel<DK, NV, PREP, EPI, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, fz);
+    return launch_tc_kernel<DK, NV, PREP, EPI, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, fz);
 }
 
 template <int DK, int NV>
 gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void *la, const void *b, const void *w,
                         const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
                         const FuseArgs *fz = nullptr) {
-    CUtensorMap tq, tk, tb, tv, tw;
+    CUtensorMap tq, tk, tb, tv, tw, to;
     const int Bt = sh.tensor_b();
     if (!make_token_map(&tq, q, Bt, sh.T, sh.H, DK) || !make_token_map(&tk, k, Bt, sh.T, sh.H, DK) ||
         !make_token_map(&tb, b, Bt, sh.T, sh.H, DK) || !make_token_map(&tv, v, Bt, sh.T, sh.HV, sh.d_v) ||
-        !make_token_map(&tw, w, Bt, sh.T, sh.HV, sh.d_v))
+        !make_token_map(&tw, w, Bt, sh.T, sh.HV, sh.d_v) || !make_token_map(&to, o, Bt, sh.T, sh.HV, sh.d_v))
         return GDN2_ERR_CUDA;
     const bool prep = fz != nullptr && fz->prep;
     // the in-kernel epilogue needs the whole d_v row in one CTA; otherwise one
@@ -132,10 +134,10 @@ gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void 
     const bool epi = fz != nullptr && fz->gate != nullptr && sh.d_v == NV;
     const FuseArgs kf = fz ? *fz : FuseArgs{};
     gdn2_status_t s;
-    if (prep && epi) s = launch_tc_seq<DK, NV, true, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
-    else if (prep) s = launch_tc_seq<DK, NV, true, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
-    else if (epi) s = launch_tc_seq<DK, NV, false, true>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
-    else s = launch_tc_seq<DK, NV, false, false>(tq, tk, tb, tv, tw, la, S0, o, S_T, sh, st, kf);
+    if (prep && epi) s = launch_tc_seq<DK, NV, true, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
+    else if (prep) s = launch_tc_seq<DK, NV, true, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
+    else if (epi) s = launch_tc_seq<DK, NV, false, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
+    else s = launch_tc_seq<DK, NV, false, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
     if (s != GDN2_OK || fz == nullptr || fz->gate == nullptr || epi) return s;
     return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, sh.rows(), sh.d_v, fz->norm_eps, st);
 }
