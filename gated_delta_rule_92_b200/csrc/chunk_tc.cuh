@@ -5,7 +5,7 @@
 //     G = cumsum_rows(log_alpha)  (per key channel)
 //     Q~ = Q.exp(G), K~ = K.exp(-G), E = B.K.exp(G)
 //     A = strict_lower(E K~^T),  P = lower(Q~ K~^T),  T = (I + A)^{-1}
-//     U = T (W.V) - (T E) S,     O = Q~ S + P U,      S' = diag(exp(G_C)) (S + K~^T U)
+//     U = T (W.V) - T (E S),     O = Q~ S + P U,      S' = diag(exp(G_C)) (S + K~^T U)
 // with S the fp32 state at the chunk start.
 //
 // One CTA (13 warps) owns one (b, h, NV-column slice of d_v) and walks the
@@ -23,17 +23,19 @@
 //              substitution, off-diagonal blocks by tf32 mma.sync block
 //              products), each block of T written to its bf16 MMA tile as soon
 //              as it is final
-//       MMA2   [. ; T] E       -> rows 64-127 = T E, back to bf16 over E
-//       MMA3   [. ; T] (W.V)   -> rows 64-127 = T (W.V); its commits free the
-//              v tile and hand T (W.V) to the chain
+//       MMA3   [. ; T] (W.V)   -> rows 64-127 = T (W.V) in TMEM; its commits
+//              free the v tile and hand T (W.V) to the chain
 //     as a two-stage pipeline: warps 0-3 solve chunk m while warps 4-7 run
 //     the prep of chunk m+1 (exp(G_C) is triple buffered for that)
 //   chain warps 8-11 chunk m-1, the sequential state pass:
-//       MMA_s  [Q~; T E] S -> X (rows 0-63 Q~ S, rows 64-127 T E S)
-//       U      = T (W.V) - T E S  (bf16 into shared memory)
+//       MMA_s  [Q~; E] S -> X (rows 0-63 Q~ S, rows 64-127 E S)
+//       -E S   to bf16 over the E tiles
+//       MMA_T  [. ; T] (-E S) accumulated onto T (W.V): rows 64-127 = U,
+//              bf16 into shared memory
 //       MMA_u  S += K~^T U   (the fp32 state stays in TMEM across chunks)
 //       MMA_o  X += [P; .] U (rows 0-63: O = Q~ S + P U)
 //       out    S rows *= exp(G_C) (+ bf16 copy for the next MMA_s); O -> HBM
+//              through the U tile and a TMA store
 // All MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> fp32).  The key and chain
 // warpgroups each issue their own MMAs from one thread and track them with
 // tcgen05.commit; hand-offs go through mbarriers.  Every wait is bounded; a
@@ -58,7 +60,7 @@ struct TcCfg {
     static constexpr uint32_t OFF_QE1 = 32768;
     static constexpr uint32_t OFF_K = 65536;               // K tiles [3 stages][kb][64 i][64 c]
     static constexpr uint32_t OFF_W = OFF_K + 3 * 16384;   // w [jb][64 i][64 j] (16 KB reserved); solve scratch
-    static constexpr uint32_t OFF_T = OFF_W + 16384;       // T [64 r][64 i]; its first KB also scratch
+    static constexpr uint32_t OFF_T = OFF_W + 16384 + 1024; // T [64 r][64 i], after the scratch's last KB
     static constexpr uint32_t OFF_V = OFF_T + 8192;        // v -> W.V
     static constexpr uint32_t OFF_P0 = OFF_V + VB * 8192u; // P [64 r][64 i], stage 0
     static constexpr uint32_t OFF_P1 = OFF_P0 + 8192;      // P, stage 1
@@ -72,13 +74,18 @@ struct TcCfg {
     static constexpr uint32_t OFF_TMEMP = OFF_BAR + 256;   // up to 32 mbarriers
     static constexpr uint32_t SMEM_BYTES = OFF_TMEMP + 16;
     static constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
-    // fp32 solve scratch A/T [64][68], in the w tile (dead once W.V is formed)
-    // and the first KB of the T tile (rewritten after the solve); the
-    // log_alpha tile is then free as soon as MMA_G has run
+    static_assert(OFF_T % 1024 == 0 && OFF_V % 1024 == 0 && OFF_S % 1024 == 0 && SMEM_ALLOC <= 232448, "layout");
+    // fp32 solve scratch A/T [64][68]: the w tile (dead once W.V is formed) and
+    // the KB after it; T itself is read by the chain's MMA_T while the next
+    // chunk's A is read out, so it does not overlap the scratch
     static constexpr int LDA = 68;
     static constexpr uint32_t OFF_SCR = OFF_W;
-    static_assert(64 * LDA * 4 <= 16384 + 8192, "solve scratch");
-    // TMEM columns: [KT 128: P'/A', then T E][T(W.V) NV][X NV][S NV]
+    // -E S of a chunk (64 tokens x NV, two 64-column halves) goes over the E
+    // tiles of its Q~/E stage (DK = 64: over Q~ and E)
+    __host__ __device__ static constexpr uint32_t es_tile(int half) { return DK == 128 ? 8192u + half * 16384u : half * 8192u; }
+    static constexpr uint32_t ES_LBO = DK == 128 ? 16384u : 8192u;
+    static_assert(64 * LDA * 4 <= 16384 + 1024, "solve scratch");
+    // TMEM columns: [KT 128: P'/A' (64 used)][T(W.V), then U NV][X NV][S NV]
     static constexpr uint32_t T_KT = 0, T_UT = 128, T_X = 128 + NV, T_S = 128 + 2 * NV;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int PREFETCH = 3;
@@ -170,12 +177,11 @@ __device__ __forceinline__ void warp_gemm16(const float *Am, const float *Bm, fl
 // accumulation); T is rounded to bf16, which dominates the tf32 input
 // rounding.  The intermediate products go to the upper-right 32x32 block of
 // the scratch.  T also goes, as bf16, to the 128-byte-swizzled MMA tile `tt`
-// as each block becomes final: the diagonal blocks while step 2 runs (warps
-// 2-3, idle there), T_{2p+1,2p} and T_ba from the products' fragments, and
-// rows 0-7 last, because the scratch's last rows overlap them.  Blocks above
-// the diagonal of `tt` are never written here: they keep the zeros the
-// kernel's setup wrote.  `bar` is a named barrier over exactly these 128
-// threads; they fence their tile writes for the tensor core before returning.
+// as each block becomes final: the diagonal blocks during step 2, T_{2p+1,2p}
+// and T_ba from the products' fragments.  Blocks above the diagonal of `tt`
+// are never written here: they keep the zeros the kernel's setup wrote.
+// `bar` is a named barrier over exactly these 128 threads; they fence their
+// tile writes for the tensor core before returning.
 template <int LDA>
 __device__ __forceinline__ void unit_lower_inverse64(float *sA, uint8_t *tt, int t, int bar) {
     const int w = t >> 5, lane = t & 31;
@@ -208,9 +214,9 @@ __device__ __forceinline__ void unit_lower_inverse64(float *sA, uint8_t *tt, int
         named_bar(bar, 128);   // both halves of each Y_p are written
         warp_gemm16<LDA, 16, 1>(sA + (R + 16) * LDA + R + 16, Y + half, sA + (R + 16) * LDA + R + half, -1.f, lane,
                                 tt, R + 16, R + half);
-        // the diagonal blocks to the tile, 8 columns a thread, rows 8.. (0-7 come last)
-        if (t < 128 - 16) {
-            const int c = t + 16;   // 8-column pieces 16.. of the four blocks (rows 0-7 of block 0 skipped)
+        // the diagonal blocks to the tile, 8 columns a thread
+        {
+            const int c = t;   // the 128 8-column pieces of the four blocks
             const int b = c >> 5, row = 16 * b + ((c >> 1) & 15), col0 = 16 * b + 8 * (c & 1);
             const float4 a = *reinterpret_cast<const float4 *>(sA + row * LDA + col0);
             const float4 d = *reinterpret_cast<const float4 *>(sA + row * LDA + col0 + 4);
@@ -226,17 +232,7 @@ __device__ __forceinline__ void unit_lower_inverse64(float *sA, uint8_t *tt, int
         warp_gemm16<LDA, 32>(sA + (32 + rm) * LDA + 32, sA + 32 + cn, nullptr, -1.f, lane, tt, 32 + rm, cn, false);
         named_bar(bar, 128);
     }
-    if (t < 64) {   // rows 0-7: D_0's first rows in columns 0-15, zeros elsewhere
-        const int row = t >> 3, ch = t & 7;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (ch < 2) {
-            const float4 a = *reinterpret_cast<const float4 *>(sA + row * LDA + 8 * ch);
-            const float4 d = *reinterpret_cast<const float4 *>(sA + row * LDA + 8 * ch + 4);
-            v = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(d.x, d.y), pack_bf16x2(d.z, d.w));
-        }
-        *reinterpret_cast<uint4 *>(tt + sw128_chunk(row, ch)) = v;
-    }
-    fence_proxy_async_smem();   // MMA2 and MMA3 read the tile
+    fence_proxy_async_smem();   // MMA3 and MMA_T read the tile
 }
 
 // 8 bf16 products of two 16-byte vectors, rounded back to bf16 (packed bf16x2
@@ -520,15 +516,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *v_free = bars + 7;      // MMA3 complete: the v tile (W.V) is free (tcgen05.commit)
     uint64_t *w_free = bars + 8;      // key done with the w tile (W.V formed, solve scratch released)
     uint64_t *full = bars + 9;        // [2] key products of a chunk ready
-    uint64_t *empty_qe = bars + 11;   // [2] chain's MMA_s done: Q~/(T E) tiles of the stage free
+    uint64_t *empty_qe = bars + 11;   // [2] chain's MMA_T done: Q~/E (then -E S) tiles of the stage free
     uint64_t *empty_k = bars + 13;    // [3] chain's MMA_u done: K~ tile of the stage free
     uint64_t *empty_pg = bars + 16;   // [2] chain done with P of the stage
-    uint64_t *utfree = bars + 18;     // chain read T(W.V) and MMA_s done
-    uint64_t *bk1 = bars + 19, *bk2 = bars + 20;
+    uint64_t *utfree = bars + 18;     // chain has read U out of TMEM
+    uint64_t *bk1 = bars + 19;        // MMA1 complete
+    uint64_t *bct = bars + 20;        // MMA_T complete (chain)
     uint64_t *bc1 = bars + 21, *bc2 = bars + 22, *bc3 = bars + 23;
     uint64_t *drain = bars + 24;      // [2] teardown: key and chain MMA issuers
     uint64_t *ut_ready = bars + 26;   // MMA3 of a chunk complete: T(W.V) in TMEM
-    constexpr int kNumBars = 27;
+    uint64_t *t_free = bars + 27;     // MMA_T complete: the T tile is free for the next solve
+    constexpr int kNumBars = 28;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_TMEMP);
     float *gC = reinterpret_cast<float *>(smem + Cfg::OFF_GC);
     float *sA = reinterpret_cast<float *>(smem + Cfg::OFF_SCR);
@@ -630,7 +628,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // else is done by all eight warps.
         const int t = tid, l = tid & 31, kq = warp & 3, kh = warp >> 2;   // lane quarter, column half
         const bool grp_b = t >= 128;
-        uint32_t ph1 = 0, ph2 = 0;
+        uint32_t ph1 = 0;
+        bool mma3_failed = false;   // thread 0 only
         float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
         float2 *nrm = reinterpret_cast<float2 *>(smem + Cfg::OFF_NRM);
         PrepLA<DK> lan;   // group B: log_alpha of the next chunk to prepare
@@ -695,7 +694,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 fence_proxy_async_smem();   // MMA3 reads W.V
             }
             {
-                bool ok = mbar_wait(bk1, ph1, wait_ns);
+                bool ok = !mma3_failed && mbar_wait(bk1, ph1, wait_ns);
                 ph1 ^= 1u;
                 // P of this stage was last read by the chain two chunks ago
                 if (m >= 2) ok = ok && mbar_wait(&empty_pg[s], static_cast<uint32_t>(((m >> 1) - 1) & 1), wait_ns);
@@ -741,7 +740,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ------------- group A: T = (I + A)^{-1};  group B: prep of chunk m+1
             bool ok_b = true;
             if (!grp_b) {
-                unit_lower_inverse64<Cfg::LDA>(sA, smem + Cfg::OFF_T, t, 3);
+                // the chain's MMA_T has read T of the previous chunk
+                if (m >= 1) ok_b = mbar_wait(t_free, static_cast<uint32_t>((m - 1) & 1), wait_ns);
+                ok_b = !group_any(3, 128, !ok_b);
+                if (ok_b) unit_lower_inverse64<Cfg::LDA>(sA, smem + Cfg::OFF_T, t, 3);
             } else if (m + 1 < NC) {
                 const int sn = (m + 1) & 1, s3n = (m + 1) % 3;
                 ok_b = mbar_wait(&qb_full[sn], static_cast<uint32_t>(((m + 1) >> 1) & 1), wait_ns);
@@ -752,24 +754,18 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                                  gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm,
                                                  min(64, len - (m + 1) * 64));
             }
+            // P (warps 0, 1, 4, 5), T and the prepared tiles are written: hand the
+            // chunk to the chain, then MMA3 [. ; T] (W.V) -> T (W.V) in TMEM, whose
+            // commits free the v tile and tell the chain; only the issuer waits
+            // for the chain to have read the previous U out of TMEM
+            fence_proxy_async_smem();
             if (group_any(1, kKeyThreads, !ok_b)) { failed = true; break; }
-            if (t == 0) mbar_arrive(w_free);   // w tile (solve scratch) is free
-            // ------------------------------------------------ MMA2 + MMA3
-            // MMA2 (T E) is committed on its own: the read-out below needs only it.
-            // MMA3 (T(W.V)) completes behind it and frees the v tile and hands
-            // T(W.V) to the chain through its own commits.  Only the issuer waits
-            // for the chain to have read the previous T(W.V) and run its MMA_s.
-            bool ok_ut = true;
             if (t == 0) {
-                if (m >= 1) ok_ut = mbar_wait(utfree, static_cast<uint32_t>((m - 1) & 1), wait_ns);
+                mbar_arrive(w_free);   // w tile (solve scratch) is free
+                mbar_arrive(&full[s]);
+                const bool ok_ut = (m == 0) || mbar_wait(utfree, static_cast<uint32_t>((m - 1) & 1), wait_ns);
                 if (ok_ut) {
                     tc_fence_after();
-                    const uint32_t id2 = idesc_bf16(128, DK, false, true);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(t_KT, sdesc_sw128(sb + Cfg::OFF_T - 8192 + ks * 32, 16, 1024),
-                                  sdesc_sw128(sb + OQE + 8192 + ks * 2048, 16384, 1024), id2, ks > 0 ? 1u : 0u);
-                    umma_commit(bk2);
                     const uint32_t id3 = idesc_bf16(128, NV, false, true);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
@@ -778,35 +774,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     umma_commit(v_free);
                     umma_commit(ut_ready);
                 } else {
-                    umma_commit(bk2);   // nothing issued: arrives at once, the group then stops below
+                    mma3_failed = true;   // the key group stops at the next MMA1 wait
                 }
             }
-            {
-                const bool ok = mbar_wait(bk2, ph2, wait_ns);
-                ph2 ^= 1u;
-                if (group_any(1, kKeyThreads, !(ok && ok_ut))) { failed = true; break; }
-            }
-            tc_fence_after();
-            // T E rows (TMEM lanes 64-127) -> bf16 over E; channel block kb = kh
-            if (kq >= 2 && kh < DK / 64) {
-                const int r = 32 * (kq - 2) + l;
-                const uint32_t eb = sb + OQE + kh * 16384 + 8192;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float x[32];
-                    tmem_ld32(t_KT + lane_q + kh * 64 + half * 32, x);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        st_shared_v4(eb + sw128_chunk(r, half * 4 + q4), pack_bf16x2(x[8 * q4], x[8 * q4 + 1]),
-                                     pack_bf16x2(x[8 * q4 + 2], x[8 * q4 + 3]), pack_bf16x2(x[8 * q4 + 4], x[8 * q4 + 5]),
-                                     pack_bf16x2(x[8 * q4 + 6], x[8 * q4 + 7]));
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar(1, kKeyThreads);
-            if (t == 0) mbar_arrive(&full[s]);
         }
+        if (mma3_failed) failed = true;
         if (t == 0) {   // wait (bounded) for this issuer's MMAs before teardown
             umma_commit(&drain[0]);
             mbar_wait(&drain[0], 0u, wait_ns);
@@ -848,7 +820,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             named_bar(2, kChainThreads);
         }
-        uint32_t ph1 = 0, ph2 = 0, ph3 = 0;
+        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, pht = 0;
         for (int n = 0; n < NC; ++n) {
             const int s = n & 1;
             if constexpr (EPI) {   // the epilogue's gate tile, into L2 a whole chain pass ahead
@@ -875,29 +847,71 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!EPI) bulk_wait_read_all();   // the previous O store has read the U tile
             }
             {
-                bool ok = mbar_wait(bc1, ph1, wait_ns);
+                const bool ok = mbar_wait(bc1, ph1, wait_ns);
                 ph1 ^= 1u;
-                ok = ok && mbar_wait(ut_ready, static_cast<uint32_t>(n & 1), wait_ns);   // T(W.V) of this chunk
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
-            if (t == 0) mbar_arrive(&empty_qe[s]);   // MMA_s has read Q~ and T E of this stage
             tc_fence_after();
+            // -E S (TMEM lanes 64-127 of X) -> bf16 over the E tiles of this stage
+            // (DK = 64: over Q~ and E), dead since MMA_s: the B operand of MMA_T
             if ((warp & 3) >= 2) {
-                const int r = t - 64;   // U row r (TMEM lanes 64-127)
+                const int r = t - 64;
 #pragma unroll 1
                 for (int jc = 0; jc < NV / 32; ++jc) {
-                    float x[32], ut[32];
+                    float x[32];
                     tmem_ld32(t_X + lane_q + jc * 32, x);
-                    tmem_ld32(t_UT + lane_q + jc * 32, ut);
+                    const uint32_t tile = sb + OQE + Cfg::es_tile((jc * 32) >> 6);
+                    const uint32_t ch0 = ((jc * 32) & 63) >> 3;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int e = 8 * q4;
+                        st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(-x[e], -x[e + 1]),
+                                     pack_bf16x2(-x[e + 2], -x[e + 3]), pack_bf16x2(-x[e + 4], -x[e + 5]),
+                                     pack_bf16x2(-x[e + 6], -x[e + 7]));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(2, kChainThreads);
+            // ------------------------------------------------------ MMA_T
+            // [. ; T] (-E S) accumulated onto MMA3's T (W.V): rows 64-127 = U; its
+            // commits free the T tile (next solve) and the Q~/E stage (producer)
+            bool ut_fail = false;
+            if (t == 0) {
+                ut_fail = !mbar_wait(ut_ready, static_cast<uint32_t>(n & 1), wait_ns);   // T(W.V) of this chunk
+                if (!ut_fail) {
+                    tc_fence_after();
+                    const uint32_t idt = idesc_bf16(128, NV, false, true);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(t_UT, sdesc_sw128(sb + Cfg::OFF_T - 8192 + ks * 32, 16, 1024),
+                                  sdesc_sw128(sb + OQE + Cfg::es_tile(0) + ks * 2048, Cfg::ES_LBO, 1024), idt, 1u);
+                    umma_commit(t_free);
+                    umma_commit(&empty_qe[s]);
+                }
+                umma_commit(bct);   // also when nothing was issued: the group then stops below
+            }
+            {
+                const bool ok = mbar_wait(bct, pht, wait_ns);
+                pht ^= 1u;
+                if (group_any(2, kChainThreads, !ok || ut_fail)) { failed = true; break; }
+            }
+            tc_fence_after();
+            if ((warp & 3) >= 2) {   // U -> bf16 (rows in TMEM lanes 64-127)
+                const int r = t - 64;
+#pragma unroll 1
+                for (int jc = 0; jc < NV / 32; ++jc) {
+                    float u[32];
+                    tmem_ld32(t_UT + lane_q + jc * 32, u);
                     const uint32_t tile = sb + Cfg::OFF_U + ((jc * 32) >> 6) * 8192u;
                     const uint32_t ch0 = ((jc * 32) & 63) >> 3;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const int e = 8 * q4;
-                        st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(ut[e] - x[e], ut[e + 1] - x[e + 1]),
-                                     pack_bf16x2(ut[e + 2] - x[e + 2], ut[e + 3] - x[e + 3]),
-                                     pack_bf16x2(ut[e + 4] - x[e + 4], ut[e + 5] - x[e + 5]),
-                                     pack_bf16x2(ut[e + 6] - x[e + 6], ut[e + 7] - x[e + 7]));
+                        st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(u[e], u[e + 1]),
+                                     pack_bf16x2(u[e + 2], u[e + 3]), pack_bf16x2(u[e + 4], u[e + 5]),
+                                     pack_bf16x2(u[e + 6], u[e + 7]));
                     }
                 }
             }
