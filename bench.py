@@ -10,8 +10,10 @@ resident in HBM (948 MB, larger than the 126 MB L2, so no flush is needed).
 `value` is tokens/s over all ranks (a token = one (b, t) position through all
 16 heads), timed on the device with CUDA events, max over ranks.  The same
 JSON line carries:
-  e2e          the same metric through the public API with pinned host
-               buffers: H2D inputs + call + D2H of o and S_T every step;
+  e2e          the same metric through the host-buffer C-ABI entry
+               (gdn2_chunk_fwd_host) on pinned host buffers: every step
+               copies the inputs in and o, S_T out, the library overlapping
+               the copies of one slice of sequences with the kernel of the next;
   roofline     the chunk kernel's algorithmic HBM bytes / launch time vs the
                measured copy bandwidth;
   decode       tokens/s of the decode workload (256 sequences x 16 heads x
@@ -359,31 +361,24 @@ def bench_decode_fused(g, wl, steps, rank, stream):
 
 
 def bench_chunk_e2e(g, wl, d, steps, stream):
-    """Same call through the public API, with pinned host inputs copied in
-    and o, S_T copied out inside the timed region, every step."""
+    """The same step through the host-buffer C-ABI entry (gdn2_chunk_fwd_host):
+    every step copies the pinned host inputs in and o, S_T out, the library
+    overlapping the copies of one slice of sequences with the kernel of the
+    next."""
     names = ("q", "k", "v", "log_alpha", "b", "w")
     host = {n: d[n].cpu().pin_memory() for n in names}
     s0_host = d["S0"].cpu().pin_memory() if d["S0"] is not None else None
-    dev = {n: torch.empty_like(d[n]) for n in names}
-    s0_dev = torch.empty_like(d["S0"]) if d["S0"] is not None else None
-    o_dev = torch.empty_like(d["v"])
-    st_dev = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
-    o_host = torch.empty(o_dev.shape, dtype=o_dev.dtype).pin_memory()
-    st_host = torch.empty(st_dev.shape, dtype=torch.float32).pin_memory()
+    o_host = torch.empty(d["v"].shape, dtype=d["v"].dtype).pin_memory()
+    st_host = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32).pin_memory()
+    ws = torch.empty(g.chunk_fwd_host_workspace_bytes(wl.B, wl.T, wl.H, wl.d_k, wl.d_v, d["q"].dtype),
+                     dtype=torch.uint8, device="cuda")
     h2d = sum(t.numel() * t.element_size() for t in host.values()) + \
         (s0_host.numel() * 4 if s0_host is not None else 0)
     d2h = o_host.numel() * o_host.element_size() + st_host.numel() * 4
 
     def step():
-        with torch.cuda.stream(stream):
-            for n in names:
-                dev[n].copy_(host[n], non_blocking=True)
-            if s0_dev is not None:
-                s0_dev.copy_(s0_host, non_blocking=True)
-            g.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["b"], dev["w"], s0_dev,
-                        o=o_dev, S_T=st_dev, stream=stream)
-            o_host.copy_(o_dev, non_blocking=True)
-            st_host.copy_(st_dev, non_blocking=True)
+        g.chunk_fwd_host(*(host[n] for n in names), s0_host, o=o_host, S_T=st_host, workspace=ws,
+                         stream=stream)
 
     step()
     torch.cuda.synchronize()

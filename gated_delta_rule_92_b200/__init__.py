@@ -32,7 +32,8 @@ IO_F32 = 0
 IO_BF16 = 1
 STATUS_NAMES = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
                 3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT"}
-EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_decode_step",
+EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_chunk_fwd_host",
+            "gdn2_chunk_fwd_host_workspace", "gdn2_decode_step",
             "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex", "gdn2_chunk_fwd_qed", "gdn2_decode_step_qed",
             "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_status_string",
             "gdn2_version")
@@ -61,6 +62,11 @@ def lib() -> ctypes.CDLL:
         for name in ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core"):
             getattr(L, name).argtypes = chunk_args
             getattr(L, name).restype = I
+        # (..., B, T, H, d_k, d_v, chunk, io, workspace, workspace_bytes, stream)
+        L.gdn2_chunk_fwd_host.argtypes = chunk_args[:-1] + [P, ctypes.c_size_t, P]
+        L.gdn2_chunk_fwd_host.restype = I
+        L.gdn2_chunk_fwd_host_workspace.argtypes = [I] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
+        L.gdn2_chunk_fwd_host_workspace.restype = I
         L.gdn2_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.gdn2_decode_step.restype = I
         F = ctypes.c_float
@@ -197,6 +203,61 @@ def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, chunk: int
               stream=None, want_state: bool = True):
     """Chunk-parallel forward; returns (o [B,T,H,d_v], S_T [B,H,d_k,d_v] or None)."""
     return _chunk("gdn2_chunk_fwd", q, k, v, log_alpha, b, w, S0, o, S_T, chunk, stream, want_state)
+
+
+def chunk_fwd_host_workspace_bytes(B: int, T: int, H: int, d_k: int, d_v: int, dtype) -> int:
+    """Device workspace bytes that chunk_fwd_host needs for this shape."""
+    n = ctypes.c_size_t(0)
+    st = lib().gdn2_chunk_fwd_host_workspace(int(B), int(T), int(H), int(d_k), int(d_v), _io(dtype),
+                                             ctypes.byref(n))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_chunk_fwd_host_workspace")
+    return int(n.value)
+
+
+def chunk_fwd_host(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, workspace=None,
+                   chunk: int = 64, stream=None, want_state: bool = True):
+    """chunk_fwd on HOST (CPU) tensors: the library copies each slice of whole
+    sequences in, runs it and copies it out, overlapping the three.  Host
+    tensors should be pinned for the copies to overlap.  `workspace` is a
+    CUDA uint8 tensor of at least chunk_fwd_host_workspace_bytes (allocated on
+    the current device if None).  Returns (o, S_T) as CPU tensors, valid once
+    the stream has been synchronised."""
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    for t in (q, k, v, log_alpha, b, w):
+        if t.is_cuda or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("token tensors must be contiguous CPU tensors of one dtype")
+    for t in (k, log_alpha, b):
+        if tuple(t.shape) != (B, T, H, dk):
+            raise ValueError("q, k, log_alpha, b must be [B, T, H, d_k]")
+    if tuple(v.shape) != (B, T, H, dv) or tuple(w.shape) != (B, T, H, dv):
+        raise ValueError("v, w must be [B, T, H, d_v]")
+    pin = q.is_pinned()
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, pin_memory=pin)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=pin)
+    for S in (S0, S_T):
+        if S is not None and (S.is_cuda or S.dtype != torch.float32 or not S.is_contiguous()
+                              or tuple(S.shape) != (B, H, dk, dv)):
+            raise ValueError(f"states must be contiguous float32 CPU tensors {(B, H, dk, dv)}")
+    if o.is_cuda or o.dtype != q.dtype or not o.is_contiguous() or tuple(o.shape) != (B, T, H, dv):
+        raise ValueError(f"o must be a contiguous CPU tensor {(B, T, H, dv)}")
+    need = chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or workspace.numel() < need:
+        raise ValueError(f"workspace must be a CUDA uint8 tensor of at least {need} bytes")
+    if stream is not None:
+        workspace.record_stream(stream)
+    with torch.cuda.device(workspace.device):
+        st = lib().gdn2_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),
+                                       _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk), _io(q.dtype),
+                                       _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_chunk_fwd_host")
+    return o, S_T
 
 
 def chunk_fwd_ex(q, k, v, log_alpha, b, w, S0=None, *, cu_seqlens=None, prep: bool = False,

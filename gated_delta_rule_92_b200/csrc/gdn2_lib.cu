@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <climits>
+#include <cstring>
 #include <mutex>
 
 #include "../../include/gdn2.h"
@@ -295,6 +296,161 @@ extern "C" gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void
     if (T == 0) return empty_sequence(S0, S_T, sh, st);
     if (io == GDN2_IO_F32 || chunk != 64) return dispatch_ffma(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io, st);
     return dispatch_tc(q, k, v, log_alpha, b, w, S0, o, S_T, sh, st);
+}
+
+// ------------------------------------------------ host buffers, pipelined
+// The batch is cut into slices of whole sequences.  Slice i is copied in on
+// one helper stream, computed on the caller's stream and copied out on a
+// second helper stream, so the copy-in of slice i + 1 and the copy-out of
+// slice i - 1 run under the kernel of slice i.  Device buffers come from the
+// caller's workspace: kHostBufs slice buffers, reused round robin.
+namespace {
+constexpr int kHostBufs = 2;
+constexpr int kHostMaxSlices = 64;
+constexpr size_t kHostAlign = 256;
+
+size_t round_up(size_t x) { return (x + kHostAlign - 1) / kHostAlign * kHostAlign; }
+
+// Helper streams and events of the host-buffer entry, created once per device
+// and kept for the life of the process (creating streams per call lets them
+// alias onto the hardware queues of earlier calls' streams).  `lock` is held
+// while a call enqueues its work; an event is re-recorded only after every
+// wait on its previous record has been enqueued.
+struct HostPipe {
+    std::mutex lock;
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t ev0 = nullptr, ev_in[kHostBufs] = {}, ev_k[kHostBufs] = {}, ev_out[kHostBufs] = {};
+    cudaError_t init() {
+        if (ready) return cudaSuccess;
+        cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev0, cudaEventDisableTiming);
+        for (int i = 0; i < kHostBufs && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_k[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming);
+        }
+        ready = e == cudaSuccess;
+        return e;
+    }
+};
+constexpr int kMaxDevices = 64;
+HostPipe g_host_pipes[kMaxDevices];
+
+struct HostSlicing {
+    int per, count;            // sequences per slice, number of slices
+    size_t key, val, state;    // bytes per sequence: one key tensor, one value tensor, one state
+    size_t buffer;             // bytes of one slice buffer
+};
+
+HostSlicing host_slicing(int B, int T, int H, int d_k, int d_v, gdn2_io_t io) {
+    HostSlicing h;
+    const size_t e = io == GDN2_IO_BF16 ? 2 : 4;
+    h.count = B < kHostMaxSlices ? B : kHostMaxSlices;
+    h.per = (B + h.count - 1) / h.count;
+    h.count = (B + h.per - 1) / h.per;
+    h.key = (size_t)T * H * d_k * e;
+    h.val = (size_t)T * H * d_v * e;
+    h.state = (size_t)H * d_k * d_v * sizeof(float);
+    // q, k, log_alpha, b; v, w, o; S0, S_T
+    h.buffer = 4 * round_up(h.per * h.key) + 3 * round_up(h.per * h.val) + 2 * round_up(h.per * h.state);
+    return h;
+}
+}  // namespace
+
+extern "C" gdn2_status_t gdn2_chunk_fwd_host_workspace(int B, int T, int H, int d_k, int d_v, gdn2_io_t io,
+                                                       size_t *bytes) {
+    if (!bytes || B <= 0 || T < 0 || H <= 0 || d_k <= 0 || d_v <= 0) return GDN2_ERR_INVALID_ARG;
+    if (io != GDN2_IO_F32 && io != GDN2_IO_BF16) return GDN2_ERR_INVALID_ARG;
+    const HostSlicing h = host_slicing(B, T, H, d_k, d_v, io);
+    *bytes = (h.count < kHostBufs ? h.count : kHostBufs) * h.buffer;
+    return GDN2_OK;
+}
+
+extern "C" gdn2_status_t gdn2_chunk_fwd_host(const void *q, const void *k, const void *v, const void *log_alpha,
+                                             const void *b, const void *w, const float *S0, void *o, float *S_T,
+                                             int B, int T, int H, int d_k, int d_v, int chunk, gdn2_io_t io,
+                                             void *workspace, size_t workspace_bytes, void *stream) {
+    const Shape sh{B, T, H, H, d_k, d_v, nullptr};
+    gdn2_status_t s = check_chunk(q, k, v, log_alpha, b, w, S0, o, S_T, sh, chunk, io);
+    if (s != GDN2_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const HostSlicing h = host_slicing(B, T, H, d_k, d_v, io);
+    if (T == 0) {   // S_T = S0 (or zeros); this case waits for the stream's earlier work
+        if (!S_T || S0 == S_T) return GDN2_OK;
+        const size_t bytes = (size_t)B * h.state;
+        const cudaError_t e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return from_cuda(e);
+        if (S0) memcpy(S_T, S0, bytes);
+        else memset(S_T, 0, bytes);
+        return GDN2_OK;
+    }
+    size_t need = 0;
+    gdn2_chunk_fwd_host_workspace(B, T, H, d_k, d_v, io, &need);
+    if (!workspace || workspace_bytes < need) return GDN2_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) % kHostAlign) return GDN2_ERR_MISALIGNED;
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (dev < 0 || dev >= kMaxDevices) return GDN2_ERR_UNSUPPORTED;
+    HostPipe &pp = g_host_pipes[dev];
+    std::lock_guard<std::mutex> guard(pp.lock);
+    if ((e = pp.init()) != cudaSuccess) return from_cuda(e);
+    cudaStream_t sin = pp.in, sout = pp.out;
+    cudaEvent_t *ev_in = pp.ev_in, *ev_k = pp.ev_k, *ev_out = pp.ev_out;
+    auto fail = [&](cudaError_t err) { return from_cuda(err); };
+    // the helper streams start after the work already on the caller's stream
+    e = cudaEventRecord(pp.ev0, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sin, pp.ev0, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, pp.ev0, 0);
+    if (e != cudaSuccess) return fail(e);
+
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k);
+    const char *hla = static_cast<const char *>(log_alpha), *hb = static_cast<const char *>(b);
+    const char *hv = static_cast<const char *>(v), *hw = static_cast<const char *>(w);
+    const char *hs0 = reinterpret_cast<const char *>(S0);
+    char *ho = static_cast<char *>(o), *hst = reinterpret_cast<char *>(S_T);
+    for (int i = 0; i < h.count; ++i) {
+        const int r = i % kHostBufs, b0 = i * h.per, nb = (B - b0 < h.per) ? B - b0 : h.per;
+        char *base = static_cast<char *>(workspace) + (size_t)r * h.buffer;
+        char *dq = base, *dk = dq + round_up(h.per * h.key), *dla = dk + round_up(h.per * h.key);
+        char *db = dla + round_up(h.per * h.key), *dv = db + round_up(h.per * h.key);
+        char *dw = dv + round_up(h.per * h.val), *dout = dw + round_up(h.per * h.val);
+        char *ds0 = dout + round_up(h.per * h.val), *dsT = ds0 + round_up(h.per * h.state);
+        const size_t kb = nb * h.key, vb = nb * h.val, sbytes = nb * h.state;
+        const size_t ko = b0 * h.key, vo = b0 * h.val, so = b0 * h.state;
+        // copy in, once the kernel that last read this buffer is done
+        if (i >= kHostBufs && (e = cudaStreamWaitEvent(sin, ev_k[r], 0)) != cudaSuccess) return fail(e);
+        const void *src[6] = {hq + ko, hk + ko, hla + ko, hb + ko, hv + vo, hw + vo};
+        void *dst[6] = {dq, dk, dla, db, dv, dw};
+        const size_t len[6] = {kb, kb, kb, kb, vb, vb};
+        for (int j = 0; j < 6 && e == cudaSuccess; ++j)
+            e = cudaMemcpyAsync(dst[j], src[j], len[j], cudaMemcpyHostToDevice, sin);
+        if (e == cudaSuccess && S0) e = cudaMemcpyAsync(ds0, hs0 + so, sbytes, cudaMemcpyHostToDevice, sin);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[r], sin);
+        // compute, once the inputs are in and the previous outputs of this buffer are out
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev_in[r], 0);
+        if (e == cudaSuccess && i >= kHostBufs) e = cudaStreamWaitEvent(st, ev_out[r], 0);
+        if (e != cudaSuccess) return fail(e);
+        const Shape ssh{nb, T, H, H, d_k, d_v, nullptr};
+        const float *s0p = S0 ? reinterpret_cast<const float *>(ds0) : nullptr;
+        float *stp = S_T ? reinterpret_cast<float *>(dsT) : nullptr;
+        s = (io == GDN2_IO_F32 || chunk != 64)
+                ? dispatch_ffma(dq, dk, dv, dla, db, dw, s0p, dout, stp, ssh, chunk, io, st)
+                : dispatch_tc(dq, dk, dv, dla, db, dw, s0p, dout, stp, ssh, st);
+        if (s != GDN2_OK) return s;
+        // copy out
+        if ((e = cudaEventRecord(ev_k[r], st)) != cudaSuccess) return fail(e);
+        if ((e = cudaStreamWaitEvent(sout, ev_k[r], 0)) != cudaSuccess) return fail(e);
+        e = cudaMemcpyAsync(ho + vo, dout, vb, cudaMemcpyDeviceToHost, sout);
+        if (e == cudaSuccess && S_T) e = cudaMemcpyAsync(hst + so, dsT, sbytes, cudaMemcpyDeviceToHost, sout);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out[r], sout);
+        if (e != cudaSuccess) return fail(e);
+    }
+    // the caller's stream ends after the last copy out
+    return from_cuda(cudaStreamWaitEvent(st, ev_out[(h.count - 1) % kHostBufs], 0));
 }
 
 extern "C" gdn2_status_t gdn2_chunk_fwd_ex(const void *q, const void *k, const void *v, const void *log_alpha,

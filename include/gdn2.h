@@ -47,6 +47,8 @@
 #ifndef GDN2_H
 #define GDN2_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -102,6 +104,50 @@ gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v,
                              const float *S0, void *o, float *S_T,
                              int B, int T, int H, int d_k, int d_v, int chunk,
                              gdn2_io_t io, void *stream);
+
+/*
+ * gdn2_chunk_fwd_host -- gdn2_chunk_fwd on HOST buffers: the same operation,
+ * shapes, dtypes and results (bit for bit: each sequence runs the same
+ * kernel), with the copies in and out done by the library.
+ *
+ *   q, k, log_alpha, b, v, w, S0 : in,  HOST pointers, layouts as above
+ *   o, S_T                       : out, HOST pointers (S_T may be NULL)
+ *   workspace                    : DEVICE buffer of at least the size that
+ *                                  gdn2_chunk_fwd_host_workspace returns,
+ *                                  256-byte aligned, owned by the caller and
+ *                                  not used by other work until this call's
+ *                                  work on `stream` has completed
+ *
+ * The batch is cut into slices of whole sequences.  Each slice is copied in
+ * on a helper stream, computed on `stream` and copied out on a second helper
+ * stream, so that the copy-in of the next slice, the kernel of this one and
+ * the copy-out of the previous one overlap; the helper streams start after
+ * the work already on `stream`, and `stream` waits for the last copy-out
+ * before anything enqueued after this call.  The two helper streams and
+ * their events are created on the first call on a device and kept for the
+ * life of the process; calls on one device enqueue one at a time.  Host buffers should be
+ * page-locked (cudaHostAlloc, or torch's pin_memory) for the copies to run
+ * asynchronously; pageable buffers give the same results, serialised.  The
+ * call returns once the work is enqueued: synchronise `stream` before
+ * reading o or S_T.  With T = 0 it waits for `stream` and sets S_T = S0 (or
+ * zeros) on the host.  An error returned after the first copy has been
+ * enqueued leaves o and S_T partly written.
+ */
+gdn2_status_t gdn2_chunk_fwd_host(const void *q, const void *k, const void *v,
+                                  const void *log_alpha, const void *b, const void *w,
+                                  const float *S0, void *o, float *S_T,
+                                  int B, int T, int H, int d_k, int d_v, int chunk,
+                                  gdn2_io_t io, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
+ * gdn2_chunk_fwd_host_workspace -- the device workspace, in bytes, that
+ * gdn2_chunk_fwd_host needs for this shape (two slice buffers of whole
+ * sequences: their token tensors, o, S0 and S_T).  Returns
+ * GDN2_ERR_INVALID_ARG for a null `bytes` or a non-positive size.
+ */
+gdn2_status_t gdn2_chunk_fwd_host_workspace(int B, int T, int H, int d_k, int d_v,
+                                            gdn2_io_t io, size_t *bytes);
 
 /*
  * gdn2_chunk_fwd_cuda_core -- the same operation and arguments as

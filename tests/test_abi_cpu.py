@@ -157,3 +157,30 @@ def test_qed_argument_validation_on_host(L):
         assert call(dk=96) == 2
         assert call(dv=96) == 2
     assert chunk_qed(T=0, ptr=None, c=None) == 0   # empty sequence, no state: nothing to do
+
+
+def test_host_entry_workspace_and_validation_on_host(L):
+    """The host-buffer entry: workspace sizing (pure host arithmetic) and the
+    argument errors it returns before any copy or launch."""
+    n = ctypes.c_size_t(0)
+    # headline shape: one sequence per slice, two slice buffers of
+    # 4 key tensors + v, w, o (16 MiB each) + S0, S_T (1 MiB each)
+    assert L.gdn2_chunk_fwd_host_workspace(8, 4096, 16, 128, 128, 1, ctypes.byref(n)) == 0
+    assert n.value == 2 * (7 * 16 * 2 ** 20 + 2 * 2 ** 20)
+    assert L.gdn2_chunk_fwd_host_workspace(1, 100, 2, 64, 64, 0, ctypes.byref(n)) == 0
+    one = 7 * (100 * 2 * 64 * 4) + 2 * (2 * 64 * 64 * 4)
+    assert n.value == one                                  # one slice: one buffer
+    assert L.gdn2_chunk_fwd_host_workspace(0, 64, 1, 64, 64, 1, ctypes.byref(n)) == 1
+    assert L.gdn2_chunk_fwd_host_workspace(1, 64, 1, 64, 64, 7, ctypes.byref(n)) == 1
+    assert L.gdn2_chunk_fwd_host_workspace(1, 64, 1, 64, 64, 1, None) == 1
+    P = ctypes.c_void_p
+    p = P(16)
+
+    def call(ws, ws_bytes, B=1, T=64, dk=64):
+        return L.gdn2_chunk_fwd_host(p, p, p, p, p, p, None, p, None, B, T, 1, dk, 64, 64, 1,
+                                     P(ws) if ws else None, ctypes.c_size_t(ws_bytes), None)
+    assert call(None, 0) == 1                              # no workspace
+    assert call(4096, 16) == 1                             # too small
+    assert call(16, 1 << 30) == 3                          # not 256-byte aligned
+    assert call(256, 1 << 30, dk=96) == 2                  # unsupported shape, as gdn2_chunk_fwd
+    assert call(256, 1 << 30, B=0) == 1
