@@ -88,7 +88,6 @@ struct TcCfg {
     // TMEM columns: [KT 128: P'/A' (64 used)][T(W.V), then U NV][X NV][S NV]
     static constexpr uint32_t T_KT = 0, T_UT = 128, T_X = 128 + NV, T_S = 128 + 2 * NV;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int PREFETCH = 3;
 };
 
 // Named barrier over `n` threads (a multiple of 32).
@@ -575,7 +574,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tma_prefetch_l2_4d(&tm_w, j0 + vb * 64, hv, r, tma_b);
                 }
             };
-            for (int p = 0; p < Cfg::PREFETCH && p < NC; ++p) prefetch(p);
+            // chunks requested into L2 ahead of their loads: one for the plain kernel,
+            // where a deeper prefetch competes with the demand loads; three with the
+            // fused prep or epilogue, whose longer chunk period leaves room for it
+            constexpr int kPrefetch = (PREP || EPI) ? 3 : 1;
+            for (int p = 0; p < kPrefetch && p < NC; ++p) prefetch(p);
             int nq = 0, nk = 0, nw = 0, nv = 0;   // next chunk to load for each group
             uint64_t t0 = globaltimer_ns();
             while (nq < NC || nk < NC || nw < NC || nv < NC) {
@@ -588,7 +591,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qb_full[s], kb * 64, h, r, tma_b);
                         tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qb_full[s], kb * 64, h, r, tma_b);
                     }
-                    if (nq + Cfg::PREFETCH < NC) prefetch(nq + Cfg::PREFETCH);
+                    if (nq + kPrefetch < NC) prefetch(nq + kPrefetch);
                     ++nq;
                     progress = true;
                 }
