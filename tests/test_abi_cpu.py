@@ -184,3 +184,22 @@ def test_host_entry_workspace_and_validation_on_host(L):
     assert call(16, 1 << 30) == 3                          # not 256-byte aligned
     assert call(256, 1 << 30, dk=96) == 2                  # unsupported shape, as gdn2_chunk_fwd
     assert call(256, 1 << 30, B=0) == 1
+
+
+def test_host_binding_rejects_bad_tensors_before_any_copy():
+    """chunk_fwd_host checks its CPU tensors in Python before it touches a device."""
+    import pytest
+    import torch
+    B, T, H, dk, dv = 1, 8, 1, 64, 64
+    q = torch.zeros(B, T, H, dk, dtype=torch.bfloat16)
+    v = torch.zeros(B, T, H, dv, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):   # v with the wrong width
+        g.chunk_fwd_host(q, q, v[..., :32], q, q, v)
+    q_strided = torch.zeros(B, T, H, 2 * dk, dtype=torch.bfloat16)[..., ::2]
+    assert q_strided.shape == q.shape and not q_strided.is_contiguous()
+    with pytest.raises(ValueError):   # non-contiguous input
+        g.chunk_fwd_host(q_strided, q, v, q, q, v)
+    with pytest.raises(ValueError):   # state of the wrong shape
+        g.chunk_fwd_host(q, q, v, q, q, v, torch.zeros(B, H, dk, dv + 1))
+    with pytest.raises(ValueError):   # mixed dtypes
+        g.chunk_fwd_host(q, q.float(), v, q, q, v)
