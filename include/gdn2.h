@@ -20,7 +20,9 @@
  *   gdn2_chunk_fwd   -- a whole sequence, chunk-parallel (chunked WY form);
  *   gdn2_decode_step -- one token per sequence against a caller-held state.
  * Their _ex forms also fuse the input prep (L2-norm of q and k, sigmoid
- * gates) and the gated RMS-norm output epilogue around the mixer.
+ * gates) and the gated RMS-norm output epilogue around the mixer, and
+ * gdn2_chunk_fwd_host runs gdn2_chunk_fwd on host buffers, overlapping the
+ * copies with the kernel.
  *
  * Common conventions
  * ------------------
