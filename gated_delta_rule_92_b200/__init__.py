@@ -33,12 +33,13 @@ IO_BF16 = 1
 STATUS_NAMES = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
                 3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT"}
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_chunk_fwd_host",
-            "gdn2_chunk_fwd_host_workspace", "gdn2_decode_step",
+            "gdn2_chunk_fwd_host_workspace", "gdn2_chunk_fwd_host_noalloc", "gdn2_decode_step",
             "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex", "gdn2_chunk_fwd_qed", "gdn2_decode_step_qed",
             "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_status_string",
             "gdn2_version")
 FUSE_INPUT_PREP = 1    # q, k, b, w are raw: L2-normalise q, k over d_k; b, w = sigmoid
 FUSE_NEG_EIGVAL = 2    # with FUSE_INPUT_PREP: b = 2 sigmoid(b)
+NOALLOC_WORKSPACE_BYTES = 64 << 20   # GDN2_NOALLOC_WORKSPACE_BYTES: the no-alloc entry's fixed workspace
 
 _lib = None
 
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.gdn2_chunk_fwd_host.restype = I
         L.gdn2_chunk_fwd_host_workspace.argtypes = [I] * 6 + [ctypes.POINTER(ctypes.c_size_t)]
         L.gdn2_chunk_fwd_host_workspace.restype = I
+        L.gdn2_chunk_fwd_host_noalloc.argtypes = chunk_args
+        L.gdn2_chunk_fwd_host_noalloc.restype = I
         L.gdn2_decode_step.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P]
         L.gdn2_decode_step.restype = I
         F = ctypes.c_float
@@ -257,6 +260,44 @@ def chunk_fwd_host(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, works
                                        _ptr(workspace), ctypes.c_size_t(workspace.numel()), _stream(stream))
     if st != 0:
         raise Gdn2Error(st, "gdn2_chunk_fwd_host")
+    return o, S_T
+
+
+def chunk_fwd_host_noalloc(q, k, v, log_alpha, b, w, S0, o, S_T=None, *, chunk: int = 64, stream=None):
+    """chunk_fwd_host for callers that cannot allocate device memory: the
+    library stages the slices in its own fixed 64 MiB device array instead of
+    a caller workspace, and this wrapper allocates nothing either (o and S_T
+    are the caller's CPU tensors; S0 and S_T may be None).  Shapes that need
+    more than that array raise ValueError.  The first call on a device sets
+    the array up, so make it before any stream capture; calls that can
+    overlap on the GPU (different streams, unordered) race on the shared
+    array.  Returns (o, S_T), valid once the stream has been synchronised."""
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    for t in (q, k, v, log_alpha, b, w, o):
+        if t.is_cuda or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError("token tensors and o must be contiguous CPU tensors of one dtype")
+    for t in (k, log_alpha, b):
+        if tuple(t.shape) != (B, T, H, dk):
+            raise ValueError("q, k, log_alpha, b must be [B, T, H, d_k]")
+    for t in (v, w, o):
+        if tuple(t.shape) != (B, T, H, dv):
+            raise ValueError("v, w, o must be [B, T, H, d_v]")
+    for S in (S0, S_T):
+        if S is not None and (S.is_cuda or S.dtype != torch.float32 or not S.is_contiguous()
+                              or tuple(S.shape) != (B, H, dk, dv)):
+            raise ValueError(f"states must be contiguous float32 CPU tensors {(B, H, dk, dv)}")
+    need = chunk_fwd_host_workspace_bytes(B, T, H, dk, dv, q.dtype)
+    if need > NOALLOC_WORKSPACE_BYTES:
+        raise ValueError(f"this shape needs a {need}-byte workspace, more than the no-alloc entry's "
+                         f"{NOALLOC_WORKSPACE_BYTES} bytes: use chunk_fwd_host with a workspace")
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        st = lib().gdn2_chunk_fwd_host_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                               _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, int(chunk),
+                                               _io(q.dtype), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_chunk_fwd_host_noalloc")
     return o, S_T
 
 

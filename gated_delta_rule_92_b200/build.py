@@ -8,6 +8,8 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "csrc", "gdn2_lib.cu")
+# the no-alloc host entry keeps its device array in a translation unit of its own
+SRC_NOALLOC = os.path.join(HERE, "csrc", "gdn2_noalloc.cu")
 LIB = os.path.join(HERE, "libgdn2.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
@@ -19,7 +21,7 @@ FLAGS = [
 
 
 def _sources():
-    return [SRC] + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + \
+    return [SRC, SRC_NOALLOC] + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + \
         [os.path.join(os.path.dirname(HERE), "include", "gdn2.h")]
 
 
@@ -34,7 +36,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
     cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + \
-        ["-o", LIB, SRC, "-ldl", "-lpthread", "-lrt"]
+        ["-o", LIB, SRC, SRC_NOALLOC, "-ldl", "-lpthread", "-lrt"]
     subprocess.check_call(cmd)
     return LIB
 

@@ -152,6 +152,42 @@ gdn2_status_t gdn2_chunk_fwd_host_workspace(int B, int T, int H, int d_k, int d_
                                             gdn2_io_t io, size_t *bytes);
 
 /*
+ * gdn2_chunk_fwd_host_noalloc -- gdn2_chunk_fwd_host without a workspace
+ * argument, for callers that cannot allocate device memory themselves (a
+ * plug-in handed host buffers and a CUDA context it does not own; a serving
+ * process whose device memory belongs to another allocator after start-up).
+ * This entry point is an addition of this library: the pages have no
+ * counterpart to it.
+ *
+ * Arguments, shapes, results and stream behaviour are those of
+ * gdn2_chunk_fwd_host (the results are equal bit for bit); the caller still
+ * passes every input and output, as HOST pointers.  The staging workspace is
+ * a fixed array of GDN2_NOALLOC_WORKSPACE_BYTES (64 MiB) in the library's
+ * own device memory.  It is reserved when the library's device code for it
+ * is loaded on a GPU (with CUDA's default lazy loading: at the first call of
+ * this function on that GPU) and held until the process exits.  The call
+ * itself allocates nothing.
+ *
+ * Shapes whose gdn2_chunk_fwd_host_workspace exceeds that size return
+ * GDN2_ERR_UNSUPPORTED before anything is enqueued; use gdn2_chunk_fwd_host
+ * with a larger workspace for them.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) and caches it: make that
+ * first call before any stream capture begins on the device.
+ *
+ * All calls on a device share the one array, and it keeps the last call's
+ * contents (nothing in it needs to start at zero).  Calls on one stream are
+ * ordered and safe.  Calls whose work can overlap on the GPU (different
+ * streams with no ordering between them) race on the array and corrupt each
+ * other's results: order them with events or use one stream.
+ */
+#define GDN2_NOALLOC_WORKSPACE_BYTES (64u << 20)
+gdn2_status_t gdn2_chunk_fwd_host_noalloc(const void *q, const void *k, const void *v,
+                                          const void *log_alpha, const void *b, const void *w,
+                                          const float *S0, void *o, float *S_T,
+                                          int B, int T, int H, int d_k, int d_v, int chunk,
+                                          gdn2_io_t io, void *stream);
+
+/*
  * gdn2_chunk_fwd_cuda_core -- the same operation and arguments as
  * gdn2_chunk_fwd, always on the CUDA-core (FFMA, fp32 products) chunk
  * kernel, for either I/O dtype.  It is the fp32-I/O path of gdn2_chunk_fwd
