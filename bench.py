@@ -360,7 +360,7 @@ def bench_decode_fused(g, wl, steps, rank, stream):
     return ms / steps
 
 
-def bench_chunk_e2e(g, wl, d, steps, stream):
+def bench_chunk_e2e(g, wl, d, steps, stream, o_dev=None, st_dev=None):
     """The same step through the host-buffer C-ABI entry (gdn2_chunk_fwd_host):
     every step copies the pinned host inputs in and o, S_T out, the library
     overlapping the copies of one slice of sequences with the kernel of the
@@ -383,7 +383,12 @@ def bench_chunk_e2e(g, wl, d, steps, stream):
     step()
     torch.cuda.synchronize()
     ms = device_time_ms(step, steps, stream)
-    return ms, h2d, d2h
+    torch.cuda.synchronize()
+    # the host-buffer results must equal the device entry's on the same inputs
+    same = None
+    if o_dev is not None and st_dev is not None:
+        same = bool(torch.equal(o_host, o_dev.cpu()) and torch.equal(st_host, st_dev.cpu()))
+    return ms, h2d, d2h, same
 
 
 def bench_decode(g, wl, steps, rank, stream):
@@ -542,7 +547,7 @@ def main():
     achieved = abytes / (launch_ms / 1e3) / 1e9
     flops = chunk_flops(wl)
 
-    e2e_ms, h2d, d2h = bench_chunk_e2e(g, wl, d, args.e2e_steps, stream)
+    e2e_ms, h2d, d2h, e2e_same = bench_chunk_e2e(g, wl, d, args.e2e_steps, stream, o, S_T)
     e2e_val, e2e_ms = aggregate_throughput(e2e_ms, args.e2e_steps, wl.B * wl.T, world)
     del d, o, S_T
     torch.cuda.empty_cache()
@@ -657,7 +662,8 @@ def main():
                          "tensor_tflops": flops / (launch_ms / 1e3) / 1e12,
                          "tensor_frac": flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
             "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps},
+                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                    "equals_device_path": e2e_same},
             "gpu_launches": args.steps,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,

@@ -253,6 +253,8 @@ def chunk_fwd_host(q, k, v, log_alpha, b, w, S0=None, *, o=None, S_T=None, works
     if not workspace.is_cuda or workspace.dtype != torch.uint8 or workspace.numel() < need:
         raise ValueError(f"workspace must be a CUDA uint8 tensor of at least {need} bytes")
     if stream is not None:
+        if stream.device != workspace.device:
+            raise ValueError(f"stream is on {stream.device} but the workspace is on {workspace.device}")
         workspace.record_stream(stream)
     with torch.cuda.device(workspace.device):
         st = lib().gdn2_chunk_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S0),

@@ -321,11 +321,14 @@ struct HostPipe {
     bool ready = false;
     cudaStream_t in = nullptr, out = nullptr;
     cudaEvent_t ev0 = nullptr, ev_in[kHostBufs] = {}, ev_k[kHostBufs] = {}, ev_out[kHostBufs] = {};
+    cudaEvent_t ev_end_in = nullptr, ev_end_out = nullptr;   // error exit: the helper streams' tails
     cudaError_t init() {
         if (ready) return cudaSuccess;
         cudaError_t e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev0, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_end_in, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_end_out, cudaEventDisableTiming);
         for (int i = 0; i < kHostBufs && e == cudaSuccess; ++i) {
             e = cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming);
             if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_k[i], cudaEventDisableTiming);
@@ -400,12 +403,20 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_host(const void *q, const void *k, const
     if ((e = pp.init()) != cudaSuccess) return from_cuda(e);
     cudaStream_t sin = pp.in, sout = pp.out;
     cudaEvent_t *ev_in = pp.ev_in, *ev_k = pp.ev_k, *ev_out = pp.ev_out;
-    auto fail = [&](cudaError_t err) { return from_cuda(err); };
     // the helper streams start after the work already on the caller's stream
     e = cudaEventRecord(pp.ev0, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(sin, pp.ev0, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, pp.ev0, 0);
-    if (e != cudaSuccess) return fail(e);
+    if (e != cudaSuccess) return from_cuda(e);
+    // An error after this point still leaves the call's work ordered on `st`:
+    // the caller's stream waits for whatever the helper streams have queued,
+    // so no copy into or out of the workspace outlives the call's stream order.
+    auto fail_status = [&](gdn2_status_t status) {
+        if (cudaEventRecord(pp.ev_end_in, sin) == cudaSuccess) cudaStreamWaitEvent(st, pp.ev_end_in, 0);
+        if (cudaEventRecord(pp.ev_end_out, sout) == cudaSuccess) cudaStreamWaitEvent(st, pp.ev_end_out, 0);
+        return status;
+    };
+    auto fail = [&](cudaError_t err) { return fail_status(from_cuda(err)); };
 
     const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k);
     const char *hla = static_cast<const char *>(log_alpha), *hb = static_cast<const char *>(b);
@@ -440,7 +451,7 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_host(const void *q, const void *k, const
         s = (io == GDN2_IO_F32 || chunk != 64)
                 ? dispatch_ffma(dq, dk, dv, dla, db, dw, s0p, dout, stp, ssh, chunk, io, st)
                 : dispatch_tc(dq, dk, dv, dla, db, dw, s0p, dout, stp, ssh, st);
-        if (s != GDN2_OK) return s;
+        if (s != GDN2_OK) return fail_status(s);
         // copy out
         if ((e = cudaEventRecord(ev_k[r], st)) != cudaSuccess) return fail(e);
         if ((e = cudaStreamWaitEvent(sout, ev_k[r], 0)) != cudaSuccess) return fail(e);
@@ -634,7 +645,7 @@ extern "C" gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream) 
     return gdn2_device_status(stream);
 }
 
-extern "C" const char *gdn2_status_string(int status) {
+extern "C" const char *gdn2_status_string(gdn2_status_t status) {
     switch (status) {
         case GDN2_OK: return "GDN2_OK";
         case GDN2_ERR_INVALID_ARG: return "GDN2_ERR_INVALID_ARG";

@@ -133,7 +133,9 @@ gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v,
  * call returns once the work is enqueued: synchronise `stream` before
  * reading o or S_T.  With T = 0 it waits for `stream` and sets S_T = S0 (or
  * zeros) on the host.  An error returned after the first copy has been
- * enqueued leaves o and S_T partly written.
+ * enqueued leaves o and S_T partly written; the work already enqueued stays
+ * ordered on `stream` (it waits for both helper streams before returning), so
+ * synchronising `stream` still waits for every copy of the failed call.
  */
 gdn2_status_t gdn2_chunk_fwd_host(const void *q, const void *k, const void *v,
                                   const void *log_alpha, const void *b, const void *w,
@@ -355,7 +357,7 @@ gdn2_status_t gdn2_device_status(void *stream);
 gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
-const char *gdn2_status_string(int status);
+const char *gdn2_status_string(gdn2_status_t status);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int gdn2_version(void);

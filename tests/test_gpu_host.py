@@ -53,3 +53,59 @@ def test_host_entry_empty_sequence(g):
     assert o.numel() == 0 and torch.equal(S, inp["S0"])
     o, S = g.chunk_fwd_host(e["q"], e["k"], e["v"], e["log_alpha"], e["b"], e["w"], None)
     assert torch.count_nonzero(S) == 0
+
+
+def _host_inputs(seed, B=2, T=130, H=2, dk=128, dv=128):
+    inp = W.draw(B, T, H, dk, dv, seed=seed, dtype=torch.bfloat16, s0_std=0.05)
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    return {n: inp[n].pin_memory() for n in names}, inp["S0"].pin_memory(), names
+
+
+def _device_ref(g, host, s0, names):
+    od, sd = g.chunk_fwd(*(host[n].cuda() for n in names), s0.cuda())
+    torch.cuda.synchronize()
+    return od.cpu(), sd.cpu()
+
+
+def test_host_entry_reuses_one_workspace(g):
+    """Two calls in a row on one stream and one workspace, different inputs:
+    the second must not see the first's data."""
+    a, s0a, names = _host_inputs(9700)
+    b, s0b, _ = _host_inputs(9701)
+    ws = torch.empty(g.chunk_fwd_host_workspace_bytes(2, 130, 2, 128, 128, torch.bfloat16),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    oa, sa = g.chunk_fwd_host(*(a[n] for n in names), s0a, workspace=ws, stream=stream)
+    ob, sb = g.chunk_fwd_host(*(b[n] for n in names), s0b, workspace=ws, stream=stream)
+    stream.synchronize()
+    for (o, S), (host, s0) in (((oa, sa), (a, s0a)), ((ob, sb), (b, s0b))):
+        ro, rs = _device_ref(g, host, s0, names)
+        assert torch.equal(o, ro) and torch.equal(S, rs)
+
+
+def test_host_entry_interleaved_streams(g):
+    """Calls on two streams with two workspaces, interleaved: the helper
+    streams are shared per device, the results must still be exact."""
+    ins = [_host_inputs(9710 + i) for i in range(4)]
+    names = ins[0][2]
+    need = g.chunk_fwd_host_workspace_bytes(2, 130, 2, 128, 128, torch.bfloat16)
+    wss = [torch.empty(need, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for i, (host, s0, _) in enumerate(ins):
+        outs.append(g.chunk_fwd_host(*(host[n] for n in names), s0, workspace=wss[i % 2],
+                                     stream=streams[i % 2]))
+    for st in streams:
+        st.synchronize()
+    assert g.device_status() == 0
+    for (o, S), (host, s0, _) in zip(outs, ins):
+        ro, rs = _device_ref(g, host, s0, names)
+        assert torch.equal(o, ro) and torch.equal(S, rs)
+
+
+def test_host_entry_rejects_stream_on_other_device(g):
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two devices")
+    a, s0a, names = _host_inputs(9720)
+    with pytest.raises(ValueError, match="stream"):
+        g.chunk_fwd_host(*(a[n] for n in names), s0a, stream=torch.cuda.Stream(device=1))
