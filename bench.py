@@ -287,6 +287,35 @@ def bench_chunk_general(g, wl, steps, rank, stream, *, H=None, HV=None, lengths=
     return ms / steps, nbytes, Bt * T
 
 
+def bench_chunk_decay(g, wl, steps, rank, stream, kind):
+    """The headline shape under strong decay: alpha ~ U[0.05, 0.5] (about 130 log2
+    units per chunk, still inside the tensor-core form's range) or mixed channels
+    (even ones alpha ~ 1e-3: every chunk runs token by token)."""
+    d = W.make_chunk_inputs(wl, seed=rank_seed(wl, rank) + 23, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed(wl, rank) + 24)
+    u = torch.rand(d["log_alpha"].shape, generator=gen, device="cuda")
+    if kind == "alpha_005_05":
+        la = torch.log(0.05 + 0.45 * u)
+    else:
+        even = (torch.arange(wl.d_k, device="cuda") % 2 == 0)
+        la = torch.where(even, torch.log(5e-4 + 1.5e-3 * u), torch.log(0.99 + 0.0099 * u))
+    d["log_alpha"] = la.to(d["log_alpha"].dtype).contiguous()
+    o = torch.empty_like(d["v"])
+    S_T = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
+
+    def step():
+        g.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], o=o, S_T=S_T, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+    torch.cuda.synchronize()
+    ms = device_time_ms(step, steps, stream)
+    if g.device_status() != 0:
+        raise RuntimeError("chunk kernel reported a device error")
+    return ms / steps
+
+
 def bench_chunk_qed(g, wl, steps, rank, stream):
     """The workload's shapes through the second, query-derived erase (CUDA cores)."""
     d = W.draw(wl.B, wl.T, wl.H, wl.d_k, wl.d_v, seed=rank_seed(wl, rank) + 17, dtype=wl.torch_dtype,
@@ -618,6 +647,17 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": bg / (lg / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": bg / (lg / 1e3) / 1e9 / peaks["hbm_gbs"],
                              "bytes_per_launch": bg}}
+            torch.cuda.empty_cache()
+
+        # strong decay: the tensor-core form near its range, and the token tail
+        for kind, nsd in (("alpha_005_05", max(10, args.steps // 4)), ("mixed", 3)):
+            ld = bench_chunk_decay(g, wl, nsd, rank, stream, kind)
+            extras["strong_decay_" + kind] = {
+                "workload": wl.describe() + (" with alpha ~ U[0.05, 0.5]" if kind == "alpha_005_05" else
+                                             " with even key channels alpha ~ 1e-3 (token tail)"),
+                "value": wl.B * wl.T / (ld / 1e3), "unit": "tokens/s", "ms_per_call": ld,
+                "roofline": {"bound": "hbm", "achieved": abytes / (ld / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": abytes / (ld / 1e3) / 1e9 / peaks["hbm_gbs"]}}
             torch.cuda.empty_cache()
 
         # f4: the second, query-derived erase direction (CUDA cores)

@@ -15,6 +15,9 @@
 // chunk: (I + A) U = W.V - E S.  Every product here is an fp32 FMA, so this
 // kernel meets fp32-I/O tolerances; it also cross-checks the tensor-core
 // kernel, which evaluates the same products on tcgen05 in a different order.
+// 1 / gamma grows with the chunk's decay: a chunk that decays by more than
+// e^-kMaxCudaCoreSpan in some channel runs token by token instead
+// (chunk_token_steps), which is exact for any decay.
 //
 // One block of 256 threads per (b, h, 64-column slice of d_v); everything
 // for one chunk lives in shared memory (about 215 KB at d_k = 128, C = 64).
@@ -23,6 +26,76 @@
 #include "gdn2_device.cuh"
 
 namespace gdn2 {
+
+// Largest decay of one chunk, in natural-log units (-sum_r log_alpha_r per
+// channel), for which the chunked products are evaluated: 1/gamma stays below
+// e^60, so neither the products nor the state update can overflow.  A chunk
+// past it runs token by token (chunk_token_steps), which is exact for any decay.
+constexpr float kMaxCudaCoreSpan = 60.f;
+
+// One chunk of the recurrence token by token on a 256-thread block, from the
+// chunk's tiles in shared memory (fp32, the input prep already applied):
+//     r_j = sum_c (b_c k_c alpha_c) S_cj,   p_j = sum_c (q_c alpha_c) S_cj,
+//     u_j = (w.v)_j - r_j,   S_cj <- alpha_c S_cj + k_c u_j,   o_j = p_j + (q . k) u_j
+// with P pseudo-rows per token (GDN-2: P = 1, row t; the second erase
+// direction: P = 2, rows 2t (key) and 2t + 1 (query direction, value 0)),
+// whose erase reads all see the same decayed state.  Row layouts: q [C][LK]
+// per token, kappa and erase vectors (erase already times kappa) [P C][LK],
+// alpha [C][LK] (already exp(log_alpha)), values [P C][LV], q . kappa [C][P];
+// the state slice S [DK][LV] is read at the start and written back at the end.
+// Thread (j, part): value column j = tid / 4, rows part, part + 4, ... of it.
+template <int DK, int NV, int P, typename IO>
+__device__ __forceinline__ void chunk_token_steps(const float *sQ, const float *sKap, const float *sEr,
+                                                  const float *sAl, const float *sVal, const float *sQK,
+                                                  float *sS, int LK, int LV, int rows, IO *__restrict__ o,
+                                                  long o_row0, long o_stride) {
+    static_assert(NV == 64, "one column per four threads");
+    constexpr int RPT = DK / 4;
+    const int tid = threadIdx.x, j = tid >> 2, part = tid & 3;
+    float Sr[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) Sr[i] = sS[(4 * i + part) * LV + j];
+    for (int t = 0; t < rows; ++t) {
+        float rr[P], pq = 0.f;
+#pragma unroll
+        for (int x = 0; x < P; ++x) rr[x] = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int c = 4 * i + part;
+            const float a = sAl[t * LK + c], sa = a * Sr[i];
+            pq = fmaf(sQ[t * LK + c], sa, pq);
+#pragma unroll
+            for (int x = 0; x < P; ++x) rr[x] = fmaf(sEr[(P * t + x) * LK + c], sa, rr[x]);
+        }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1) {
+            pq += __shfl_xor_sync(0xffffffffu, pq, off);
+#pragma unroll
+            for (int x = 0; x < P; ++x) rr[x] += __shfl_xor_sync(0xffffffffu, rr[x], off);
+        }
+        float u[P], ov = pq;
+#pragma unroll
+        for (int x = 0; x < P; ++x) {
+            u[x] = sVal[(P * t + x) * LV + j] - rr[x];
+            ov = fmaf(sQK[P * t + x], u[x], ov);
+        }
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int c = 4 * i + part;
+            float nv = sAl[t * LK + c] * Sr[i];
+#pragma unroll
+            for (int x = 0; x < P; ++x) nv = fmaf(sKap[(P * t + x) * LK + c], u[x], nv);
+            Sr[i] = nv;
+        }
+        if (part == 0) {
+            IO *dst = o + o_row0 + (long)t * o_stride + j;
+            if constexpr (sizeof(IO) == 4) *dst = ov;
+            else *dst = __float2bfloat16_rn(ov);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) sS[(4 * i + part) * LV + j] = Sr[i];
+}
 
 template <int DK, int CH = 64>
 struct FfmaCfg {
@@ -134,6 +207,34 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
                 }
             }
             __syncthreads();
+        }
+        // ---- the chunk's decay: past kMaxCudaCoreSpan it runs token by token
+        {
+            float tot = 0.f;
+            if (tid < DK)
+                for (int r = 0; r < C; ++r) tot += sG[r * LK + tid];
+            if (__syncthreads_or(tid < DK && !(tot >= -kMaxCudaCoreSpan))) {
+                // erase vectors b.k, alpha = exp(log_alpha) and q . k per token, in place
+                for (int idx = tid; idx < C * DK; idx += 256) {
+                    const int r = idx / DK, c = idx % DK;
+                    sE[r * LK + c] *= sK[r * LK + c];
+                    sG[r * LK + c] = __expf(sG[r * LK + c]);
+                }
+                {
+                    const int wp = tid >> 5, l = tid & 31;
+                    for (int r = wp; r < C; r += 8) {
+                        float qk = 0.f;
+                        for (int c = l; c < DK; c += 32) qk = fmaf(sQ[r * LK + c], sK[r * LK + c], qk);
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
+                        if (l == 0) sGC[r] = qk;
+                    }
+                }
+                __syncthreads();
+                chunk_token_steps<DK, NV, 1, IO>(sQ, sK, sE, sG, sWV, sGC, sS, LK, LV, rows, o,
+                                                 (tok0 * HV + hv) * (long)d_v + j0, (long)HV * d_v);
+                continue;   // the next chunk starts with a barrier
+            }
         }
         // ---- cumulative log-decay per key channel and the scaled operands
         if (tid < DK) {

@@ -2,11 +2,16 @@
 //
 // Chunk algebra (the burn-gdn2 README recurrence, "Architecture" section,
 // regrouped over chunks of C = 64 tokens as in its "Chunk WY (train)" mode):
-//     G = cumsum_rows(log_alpha)  (per key channel)
-//     Q~ = Q.exp(G), K~ = K.exp(-G), E = B.K.exp(G)
+//     G = cumsum_rows(log_alpha)  (per key channel),  ref = (G_0 + G_C) / 2
+//     Q~ = Q.exp(G - ref), K~ = K.exp(ref - G), E = B.K.exp(G - ref)
 //     A = strict_lower(E K~^T),  P = lower(Q~ K~^T),  T = (I + A)^{-1}
-//     U = T (W.V) - T (E S),     O = Q~ S + P U,      S' = diag(exp(G_C)) (S + K~^T U)
-// with S the fp32 state at the chunk start.
+//     U = T (W.V) - T (E S_r),   O = Q~ S_r + P U,    S' = diag(exp(G_C - ref)) (S_r + K~^T U)
+// with S the fp32 state at the chunk start and S_r = diag(exp(ref)) S the state
+// as the chain carries it.  The reference point in the middle of the chunk's
+// decay range keeps every operand within exp(+-span / 2), span = G_0 - G_C; a
+// chunk whose span passes kMaxChunkSpan2 (log2 units) is not evaluated this way:
+// it and the rest of its sequence run token by token (tc_token_tail), so the
+// kernel is exact for any decay.
 //
 // One CTA (13 warps) owns one (b, h, NV-column slice of d_v) and walks the
 // T/64 chunks in order as a pipeline:
@@ -15,8 +20,9 @@
 //                   as soon as its last reader is done), L2 prefetch ahead;
 //                   log_alpha goes straight to the prep threads' registers.
 //   key warps 0-7   chunk m, everything that does not depend on the state:
-//       prep   G by a running fp32 sum per channel pair, then Q~, E, K~ in
-//              place in the TMA tiles and exp(G_C) for the state update
+//       prep   G by a running fp32 sum per channel quad, the chunk's span and
+//              reference point, then Q~, E, K~ in place in the TMA tiles and
+//              exp(G_C - ref), exp(ref) for the state update
 //       W.V    in place in the v tile
 //       MMA1   [Q~; E] K~^T -> TMEM (rows 0-63 P', rows 64-127 A')
 //       solve  T = (I + A)^{-1} in fp32 (16x16 diagonal blocks by forward
@@ -26,7 +32,7 @@
 //       MMA3   [. ; T] (W.V)   -> rows 64-127 = T (W.V) in TMEM; its commits
 //              free the v tile and hand T (W.V) to the chain
 //     as a two-stage pipeline: warps 0-3 solve chunk m while warps 4-7 run
-//     the prep of chunk m+1 (exp(G_C) is triple buffered for that)
+//     the prep of chunk m+1 (the state factors are triple buffered for that)
 //   chain warps 8-11 chunk m-1, the sequential state pass:
 //       MMA_s  [Q~; E] S -> X (rows 0-63 Q~ S, rows 64-127 E S)
 //       -E S   to bf16 over the E tiles
@@ -34,8 +40,8 @@
 //              bf16 into shared memory
 //       MMA_u  S += K~^T U   (the fp32 state stays in TMEM across chunks)
 //       MMA_o  X += [P; .] U (rows 0-63: O = Q~ S + P U)
-//       out    S rows *= exp(G_C) (+ bf16 copy for the next MMA_s); O -> HBM
-//              through the U tile and a TMA store
+//       out    S rows *= exp(G_C - ref), then *= exp(ref') of the next chunk (+ bf16
+//              copy for the next MMA_s); O -> HBM through the U tile and a TMA store
 // All MMAs are tcgen05.mma kind::f16 (bf16 x bf16 -> fp32).  The key and chain
 // warpgroups each issue their own MMAs from one thread and track them with
 // tcgen05.commit; hand-offs go through mbarriers.  Every wait is bounded; a
@@ -66,13 +72,15 @@ struct TcCfg {
     static constexpr uint32_t OFF_P1 = OFF_P0 + 8192;      // P, stage 1
     static constexpr uint32_t OFF_S = OFF_P1 + 8192;       // bf16 S [jb][128 c][64 j]
     static constexpr uint32_t OFF_U = OFF_S + VB * 16384u; // U [jb][64 i][64 j]
-    static constexpr uint32_t OFF_CARRY = OFF_U + VB * 8192u;   // cumsum carries [row block][128]
-    static constexpr uint32_t OFF_GC = OFF_CARRY + 2048;         // exp(G_C) [3][128]
-    static constexpr uint32_t OFF_NRM = OFF_GC + 1536;           // fused prep: 1/|q_r|, 1/|k_r| [64][2]
+    static constexpr uint32_t OFF_CARRY = OFF_U + VB * 8192u;   // cumsum carries [row block][128], row 0 [128]
+    static constexpr uint32_t OFF_GC = OFF_CARRY + 2560;         // state factors [3][2][128]
+    static constexpr uint32_t OFF_NRM = OFF_GC + 3072;           // fused prep: 1/|q_r|, 1/|k_r| [64][2]
     static constexpr uint32_t OFF_NW = OFF_NRM + 512;            // fused epilogue: norm weight [NV]
     static constexpr uint32_t OFF_BAR = OFF_NW + 512;
     static constexpr uint32_t OFF_TMEMP = OFF_BAR + 256;   // up to 32 mbarriers
-    static constexpr uint32_t SMEM_BYTES = OFF_TMEMP + 16;
+    static constexpr uint32_t OFF_STOP = OFF_TMEMP + 4;    // first chunk handed to the token tail
+    static constexpr uint32_t OFF_SEQ = OFF_TMEMP + 8;     // this CTA's sequence: tok0 (8 B), len, bb
+    static constexpr uint32_t SMEM_BYTES = OFF_TMEMP + 24;
     static constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
     static_assert(OFF_T % 1024 == 0 && OFF_V % 1024 == 0 && OFF_S % 1024 == 0 && SMEM_ALLOC <= 232448, "layout");
     // fp32 solve scratch A/T [64][68]: the w tile (dead once W.V is formed) and
@@ -94,6 +102,11 @@ struct TcCfg {
 __device__ __forceinline__ void named_bar(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Arrive on named barrier `id` (of `n` threads) without waiting: the producer
+// side of a hand-off whose consumers wait with named_bar(id, n).
+__device__ __forceinline__ void named_bar_arrive(int id, int n) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 // Named barrier over `n` threads that also ORs a predicate across them.
 __device__ __forceinline__ bool group_any(int id, int n, bool p) {
     uint32_t r;
@@ -107,6 +120,15 @@ __device__ __forceinline__ bool group_any(int id, int n, bool p) {
         : "memory");
     return r != 0;
 }
+// Largest decay span, in log2 units, that a chunk may have for the tensor-core
+// form: over rows 1..63, sum_r log2(alpha_r) >= -kMaxChunkSpan2 in every channel.
+// The operands then stay within 2^(+-100): the masked (upper) products may
+// overflow and are discarded by selection, every kept product is bounded by
+// |q| |k|, and the state update K~^T U stays below 2^128 while |k| |U| < 2^22.
+// A chunk past it (a mean decay below about 0.11 per token over the chunk) and
+// the rest of its sequence go to the token tail.
+constexpr float kMaxChunkSpan2 = 200.f;
+
 constexpr int kKeyThreads = 256;     // warps 0-7
 constexpr int kChainThreads = 128;   // warps 8-11
 constexpr int kTcThreads = kKeyThreads + kChainThreads + 32;   // + producer warp 12
@@ -271,9 +293,12 @@ struct PrepLA {
 };
 
 // Prep of one chunk by 128 threads (thread g): the per-channel cumulative
-// log-decay G (fp32, in row order, kept as G log2(e)) and, in place in the TMA tiles,
-//     Q~ = q.exp(G),  E = b.k.exp(G),  K~ = k.exp(-G),
-// plus exp(G_C) (last row) into gc.  Thread g owns the channel quad
+// log-decay G (fp32, in row order, kept as G log2(e)), the reference point
+// ref = (G_0 + G_C) / 2 and, in place in the TMA tiles,
+//     Q~ = q.exp(G - ref),  E = b.k.exp(G - ref),  K~ = k.exp(ref - G),
+// plus exp(G_C - ref) and exp(ref) into gc[0..127] and gc[128..255].  A chunk whose
+// span G_0 - G_C passes kMaxChunkSpan2 in any channel sets *stop_at = chunk (its
+// tiles are then never used).  Thread g owns the channel quad
 // p = g % (DK/4) over a block of R consecutive rows (its log_alpha values in
 // `law`); the running sum enters a block with the totals of the blocks above
 // it (exchanged through `carry` and named barrier `bar` over the 128
@@ -289,7 +314,8 @@ struct PrepLA {
 // only on a sequence's partial last chunk and leaves the loop below as is.
 template <int DK, bool PREP = false, bool VARLEN = false>
 __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLA<DK> &law,
-                                           float *gc, float *carry, int g, int bar, const FuseArgs &fz = {},
+                                           float *gc, float *carry, int g, int bar, int chunk,
+                                           volatile int *stop_at, const FuseArgs &fz = {},
                                            float2 *nrm = nullptr, int rows_valid = 64) {
     constexpr int NP = PrepLA<DK>::NP, NB = PrepLA<DK>::NB, R = PrepLA<DK>::R;
     static_assert(NB * R == 64 && NB <= 8, "prep split");
@@ -336,19 +362,32 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
         sum[2] = fmaf(bf16_lo(law.v[i].y), kLog2e, sum[2]);
         sum[3] = fmaf(bf16_hi(law.v[i].y), kLog2e, sum[3]);
     }
-    reinterpret_cast<float4 *>(carry)[hb * NP + p] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+    float4 *carry4 = reinterpret_cast<float4 *>(carry);
+    carry4[hb * NP + p] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+    if (hb == 0)   // row 0 on its own: the reference point is taken from G_0 and G_C
+        carry4[NB * NP + p] = make_float4(bf16_lo(law.v[0].x) * kLog2e, bf16_hi(law.v[0].x) * kLog2e,
+                                          bf16_lo(law.v[0].y) * kLog2e, bf16_hi(law.v[0].y) * kLog2e);
     named_bar(bar, 128);
+    // Reference point ref = (G_0 + G_C) / 2 per channel: the operands are scaled by
+    // 2^(G_r - ref) and 2^(ref - G_r), both within 2^(+-span / 2) with span = G_0 - G_C
+    // (the decay of rows 1..63; row 0's own decay only scales the incoming state).
+    // The running sum enters this thread's rows at (sum of the blocks above) - ref
+    //   = sum_h2 (h2 < hb ? 1/2 : -1/2) carry[h2] - G_0 / 2.
+    {
+        const float4 r4 = carry4[NB * NP + p];
+        sum[0] = -0.5f * r4.x;
+        sum[1] = -0.5f * r4.y;
+        sum[2] = -0.5f * r4.z;
+        sum[3] = -0.5f * r4.w;
+    }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) sum[e] = 0.f;
-#pragma unroll
-    for (int h2 = 0; h2 < NB - 1; ++h2) {
-        if (h2 < hb) {
-            const float4 c4 = reinterpret_cast<const float4 *>(carry)[h2 * NP + p];
-            sum[0] += c4.x;
-            sum[1] += c4.y;
-            sum[2] += c4.z;
-            sum[3] += c4.w;
-        }
+    for (int h2 = 0; h2 < NB; ++h2) {
+        const float4 c4 = carry4[h2 * NP + p];
+        const float wgt = h2 < hb ? 0.5f : -0.5f;
+        sum[0] = fmaf(wgt, c4.x, sum[0]);
+        sum[1] = fmaf(wgt, c4.y, sum[1]);
+        sum[2] = fmaf(wgt, c4.z, sum[2]);
+        sum[3] = fmaf(wgt, c4.w, sum[3]);
     }
     // rows in batches of RB, software-pipelined: the tiles are rewritten in
     // place, so the compiler keeps every load behind the earlier stores; the
@@ -427,8 +466,18 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
         }
     }
     if (hb == NB - 1) {
+        // the last rows end at G_C - ref = -span / 2: 2^(G_C - ref) is the factor applied
+        // after the state update, 2^ref = 2^(G_0 - span / 2) the scale of the incoming state
+        const float4 r4 = carry4[NB * NP + p];
+        const float g0[4] = {r4.x, r4.y, r4.z, r4.w};
+        bool out = false;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) gc[4 * p + e] = ex2(sum[e]);
+        for (int e = 0; e < 4; ++e) {
+            out |= !(-2.f * sum[e] <= kMaxChunkSpan2);   // also catches NaN from infinite decays
+            gc[4 * p + e] = ex2(sum[e]);
+            gc[128 + 4 * p + e] = ex2(g0[e] + sum[e]);
+        }
+        if (out) *stop_at = chunk;   // every writer stores the same value
     }
     fence_proxy_async_smem();
 }
@@ -464,6 +513,234 @@ __device__ __forceinline__ int longest_first_sequence(const int *__restrict__ cu
     return r;
 }
 
+// N consecutive bf16 values (N = 2 or 4) read with one 4- or 8-byte load.
+template <int N>
+struct BfVec {
+    static_assert(N == 2 || N == 4, "bf16 vector");
+    uint32_t w[N / 2];
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+        if constexpr (N == 4) {
+            const uint2 x = __ldg(reinterpret_cast<const uint2 *>(p));
+            w[0] = x.x;
+            w[1] = x.y;
+        } else {
+            w[0] = __ldg(reinterpret_cast<const unsigned int *>(p));
+        }
+    }
+    __device__ __forceinline__ float get(int e) const { return (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]); }
+};
+
+// Raw token pointers for the token tail (the main loop reads through TMA maps).
+struct TailArgs {
+    const __nv_bfloat16 *q, *k, *b, *v, *w;
+};
+
+// Token tail: a chunk whose decay span passes kMaxChunkSpan2, and every later
+// chunk of its sequence, run here token by token, straight from the step
+//     r_j = sum_c (b_c k_c alpha_c) S_cj,   p_j = sum_c (q_c alpha_c) S_cj,
+//     u_j = w_j v_j - r_j,   S_cj <- alpha_c S_cj + k_c u_j,   o_j = p_j + (q . k) u_j
+// with alpha = exp(log_alpha) per token, so a decay of any strength is exact to
+// fp32 rounding.  `smem` holds the state at the start of token t_begin as fp32
+// [DK][NV + 4] (row c, column j).
+//   warps 0-7   arithmetic: lane = 8 cb + rb; thread (warp, cb, rb) holds rows
+//               rb, rb + 8, ... (DK / 8 of them) of the NV / 32 columns
+//               (4 warp + cb) NV / 32 .. in registers; the column sums over the
+//               rows reduce across the 8 rb lanes by shuffles
+//   warps 8-12  stage the inputs of TB tokens at a time into one of two
+//               buffers (warp 8 + s: tokens s, s + 5, ...), handed over with
+//               named barriers (full: staging arrives, arithmetic waits; empty:
+//               the other way round)
+// Every thread of the block calls it.
+template <int DK, int NV, bool PREP, bool EPI>
+__device__ __noinline__ void tc_token_tail(uint8_t *smem, const TailArgs ta, const __nv_bfloat16 *__restrict__ la,
+                                           __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, long tok0,
+                                           int t_begin, int len, int h, int H, int hv, int HV, int j0, int d_v,
+                                           long head, const FuseArgs fz) {
+    constexpr int TB = 16, LS = NV + 4;
+    constexpr int RR = DK / 8, CJ = NV / 32;      // rows and columns of S per arithmetic thread
+    constexpr int CPL = DK / 32, JPL = NV / 32;   // channels / columns per lane when staging
+    constexpr int kStage = 5, kAll = kTcThreads;  // staging warps; threads on the hand-off barriers
+    constexpr int BAR_FULL = 5, BAR_EMPTY = 7, BAR_MATH = 9;   // ids 5-6, 7-8 by buffer; 9: arithmetic only
+    const float *sS = reinterpret_cast<const float *>(smem);
+    float4 *rowd = reinterpret_cast<float4 *>(smem + DK * LS * 4);    // [2][TB][DK]: alpha, b k alpha, q alpha, k
+    float2 *cold = reinterpret_cast<float2 *>(rowd + 2 * TB * DK);     // [2][TB][NV]: w v, gate
+    float *qkb = reinterpret_cast<float *>(cold + 2 * TB * NV);        // [2][TB]: q . k
+    float *obuf = qkb + 2 * TB;                                        // [TB][NV] (EPI)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nb = (len - t_begin + TB - 1) / TB;   // batches
+    if (warp < 8) {
+        // ============================================================ arithmetic
+        const int rb = lane & 7, cb = lane >> 3, jb = (4 * warp + cb) * CJ;
+        float Sr[RR][CJ];
+#pragma unroll
+        for (int i = 0; i < RR; ++i)
+#pragma unroll
+            for (int x = 0; x < CJ; ++x) Sr[i][x] = sS[(8 * i + rb) * LS + jb + x];
+        for (int k = 0; k < nb; ++k) {
+            const int buf = k & 1, tb = t_begin + k * TB, nt = min(TB, len - tb);
+            named_bar(BAR_FULL + buf, kAll);
+            const float4 *rdb = rowd + buf * TB * DK;
+            for (int tt = 0; tt < nt; ++tt) {
+                const float4 *rd = rdb + tt * DK;
+                float r[CJ], pq[CJ];
+#pragma unroll
+                for (int x = 0; x < CJ; ++x) r[x] = pq[x] = 0.f;
+#pragma unroll
+                for (int i = 0; i < RR; ++i) {
+                    const float4 xr = rd[8 * i + rb];
+#pragma unroll
+                    for (int x = 0; x < CJ; ++x) {
+                        r[x] = fmaf(xr.y, Sr[i][x], r[x]);
+                        pq[x] = fmaf(xr.z, Sr[i][x], pq[x]);
+                    }
+                }
+#pragma unroll
+                for (int off = 1; off < 8; off <<= 1)
+#pragma unroll
+                    for (int x = 0; x < CJ; ++x) {
+                        r[x] += __shfl_xor_sync(0xffffffffu, r[x], off);
+                        pq[x] += __shfl_xor_sync(0xffffffffu, pq[x], off);
+                    }
+                const float qk = qkb[buf * TB + tt];
+                float u[CJ], ov[CJ];
+#pragma unroll
+                for (int x = 0; x < CJ; ++x) {
+                    u[x] = cold[(buf * TB + tt) * NV + jb + x].x - r[x];
+                    ov[x] = fmaf(qk, u[x], pq[x]);
+                }
+#pragma unroll
+                for (int i = 0; i < RR; ++i) {
+                    const float4 xr = rd[8 * i + rb];
+#pragma unroll
+                    for (int x = 0; x < CJ; ++x) Sr[i][x] = fmaf(xr.x, Sr[i][x], xr.w * u[x]);
+                }
+                if (rb == 0) {
+                    if constexpr (EPI) {
+#pragma unroll
+                        for (int x = 0; x < CJ; ++x) obuf[tt * NV + jb + x] = ov[x];
+                    } else {
+                        __nv_bfloat16 *dst = o + ((tok0 + tb + tt) * HV + hv) * (long)d_v + j0 + jb;
+#pragma unroll
+                        for (int x = 0; x < CJ; x += 2)
+                            *reinterpret_cast<uint32_t *>(dst + x) = pack_bf16x2(ov[x], ov[x + 1]);
+                    }
+                }
+            }
+            if constexpr (EPI) {   // y = o / sqrt(mean(o^2) + eps) . weight . silu(gate), a warp per token
+                named_bar(BAR_MATH, 256);
+                for (int tt = warp; tt < nt; tt += 8) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < JPL; ++e) {
+                        const float x = obuf[tt * NV + lane + 32 * e];
+                        ss = fmaf(x, x, ss);
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float inv = rsqrtf(ss / (float)NV + fz.norm_eps);
+                    const long vro = ((tok0 + tb + tt) * HV + hv) * (long)d_v + j0;
+#pragma unroll
+                    for (int e = 0; e < JPL; ++e) {
+                        const int jj = lane + 32 * e;
+                        const float gt = cold[(buf * TB + tt) * NV + jj].y;
+                        o[vro + jj] = __float2bfloat16_rn(obuf[tt * NV + jj] * inv * fz.norm_weight[j0 + jj] * gt *
+                                                          sigmoid_f32(gt));
+                    }
+                }
+                named_bar(BAR_MATH, 256);   // obuf is rewritten by the next batch
+            }
+            if (k + 2 < nb) named_bar_arrive(BAR_EMPTY + buf, kAll);   // the staging warps refill it
+        }
+        if (S_T != nullptr) {
+#pragma unroll
+            for (int i = 0; i < RR; ++i) {
+                float *dst = S_T + (head * DK + 8 * i + rb) * d_v + j0 + jb;
+#pragma unroll
+                for (int x = 0; x < CJ; ++x) dst[x] = Sr[i][x];
+            }
+        }
+    } else {
+        // ============================================================ staging
+        // warp 8 + sw takes tokens sw, sw + 5, ... of a batch (MT at most); every
+        // load of its tokens is issued (as 4- or 8-byte vectors) before any is used
+        constexpr int MT = (TB + kStage - 1) / kStage;
+        const float bscale = (PREP && fz.neg_eigval) ? 2.f : 1.f;
+        const int sw = warp - 8;
+        for (int k = 0; k < nb; ++k) {
+            const int buf = k & 1, tb = t_begin + k * TB, nt = min(TB, len - tb);
+            if (k >= 2) named_bar(BAR_EMPTY + buf, kAll);
+            BfVec<CPL> rq[MT], rk[MT], rbv[MT], rl[MT];
+            BfVec<JPL> rv[MT], rw[MT], rg[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const int tt = sw + kStage * m;
+                if (tt < nt) {
+                    const long tok = tok0 + tb + tt;
+                    const long kro = (tok * H + h) * DK + CPL * lane;
+                    const long vro = (tok * HV + hv) * (long)d_v + j0 + JPL * lane;
+                    rq[m].load(ta.q + kro);
+                    rk[m].load(ta.k + kro);
+                    rbv[m].load(ta.b + kro);
+                    rl[m].load(la + kro);
+                    rv[m].load(ta.v + vro);
+                    rw[m].load(ta.w + vro);
+                    if constexpr (EPI) rg[m].load(static_cast<const __nv_bfloat16 *>(fz.gate) + vro);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const int tt = sw + kStage * m;
+                if (tt >= nt) continue;   // warp-uniform
+                float qv[CPL], kv[CPL], bv[CPL];
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    qv[e] = rq[m].get(e);
+                    kv[e] = rk[m].get(e);
+                    bv[e] = rbv[m].get(e);
+                }
+                if constexpr (PREP) {   // q, k L2-normalised over d_k; b = sigmoid (x2 with neg_eigval)
+                    float sq = 0.f, sk = 0.f;
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) {
+                        sq = fmaf(qv[e], qv[e], sq);
+                        sk = fmaf(kv[e], kv[e], sk);
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) {
+                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    }
+                    const float iq = l2_inv(sq, fz.l2_eps), ik = l2_inv(sk, fz.l2_eps);
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e) {
+                        qv[e] *= iq;
+                        kv[e] *= ik;
+                        bv[e] = bscale * sigmoid_f32(bv[e]);
+                    }
+                }
+                float dot = 0.f;
+                float4 *rdst = rowd + (buf * TB + tt) * DK + CPL * lane;
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    const float a = __expf(rl[m].get(e));
+                    dot = fmaf(qv[e], kv[e], dot);
+                    rdst[e] = make_float4(a, bv[e] * kv[e] * a, qv[e] * a, kv[e]);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+                if (lane == 0) qkb[buf * TB + tt] = dot;
+                float2 *cdst = cold + (buf * TB + tt) * NV + JPL * lane;
+#pragma unroll
+                for (int e = 0; e < JPL; ++e) {
+                    const float wv = rw[m].get(e), vv = rv[m].get(e);
+                    cdst[e] = make_float2((PREP ? sigmoid_f32(wv) : wv) * vv, EPI ? rg[m].get(e) : 0.f);
+                }
+            }
+            named_bar_arrive(BAR_FULL + buf, kAll);
+        }
+    }
+}
+
 // PREP fuses the input prep (raw q, k, b, w); EPI the gated RMS norm of each
 // output row before it is stored (d_v == NV: one CTA holds the whole row).
 template <int DK, int NV, bool PREP = false, bool EPI = false, bool VARLEN = false>
@@ -474,7 +751,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __nv_bfloat16 *__restrict__ la,
                     const float *__restrict__ S0,
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int T, int H, int HV, int d_v,
-                    const int *__restrict__ cu_seqlens, unsigned long long wait_ns, const FuseArgs fz) {
+                    const int *__restrict__ cu_seqlens, unsigned long long wait_ns, const FuseArgs fz,
+                    const TailArgs ta) {
     static_assert(!EPI || NV <= 128, "epilogue weight slice");
     using Cfg = TcCfg<DK, NV>;
     extern __shared__ uint8_t smem_raw[];
@@ -532,7 +810,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     // ---------------------------------------------------------------- setup
     for (uint32_t off = tid * 16u; off < Cfg::OFF_CARRY; off += kTcThreads * 16u) st_shared_v4(sb + off, 0u, 0u, 0u, 0u);
-    for (int i = tid; i < 3 * 128; i += kTcThreads) gC[i] = 1.f;   // channels >= d_k keep exp(G_C) = 1
+    for (int i = tid; i < 3 * 256; i += kTcThreads) gC[i] = 1.f;   // channels >= d_k keep factors of 1
+    volatile int *stop_at = reinterpret_cast<volatile int *>(smem + Cfg::OFF_STOP);
+    if (tid == 0) {
+        *stop_at = 0x7fffffff;
+        // kept for the teardown, so that no register holds them through the main loop
+        *reinterpret_cast<long *>(smem + Cfg::OFF_SEQ) = tok0;
+        reinterpret_cast<int *>(smem + Cfg::OFF_SEQ)[2] = len;
+        reinterpret_cast<int *>(smem + Cfg::OFF_SEQ)[3] = bb;
+    }
     if constexpr (EPI) {
         float *nw = reinterpret_cast<float *>(smem + Cfg::OFF_NW);
         for (int i = tid; i < NV; i += kTcThreads) nw[i] = fz.norm_weight[j0 + i];
@@ -580,10 +866,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             constexpr int kPrefetch = (PREP || EPI) ? 3 : 1;
             for (int p = 0; p < kPrefetch && p < NC; ++p) prefetch(p);
             int nq = 0, nk = 0, nw = 0, nv = 0;   // next chunk to load for each group
+            int lim = NC;                         // chunks from a handed-off one on are not loaded
             uint64_t t0 = globaltimer_ns();
-            while (nq < NC || nk < NC || nw < NC || nv < NC) {
+            while (nq < lim || nk < lim || nw < lim || nv < lim) {
                 bool progress = false;
-                if (nq < NC && (nq < 2 || mbar_test_wait(&empty_qe[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
+                if (nq < lim && (nq < 2 || mbar_test_wait(&empty_qe[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
                     const int s = nq & 1, r = tma_t0 + nq * 64;
                     const uint32_t oqe = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0;
                     mbar_arrive_expect_tx(&qb_full[s], 2u * Cfg::KEY_TILE);
@@ -595,7 +882,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ++nq;
                     progress = true;
                 }
-                if (nk < NC && (nk < 3 || mbar_test_wait(&empty_k[nk % 3], static_cast<uint32_t>((nk / 3 - 1) & 1)))) {
+                if (nk < lim && (nk < 3 || mbar_test_wait(&empty_k[nk % 3], static_cast<uint32_t>((nk / 3 - 1) & 1)))) {
                     const int s3 = nk % 3, r = tma_t0 + nk * 64;
                     mbar_arrive_expect_tx(&k_full[s3], Cfg::KEY_TILE);
                     for (int kb = 0; kb < DK / 64; ++kb)
@@ -603,7 +890,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ++nk;
                     progress = true;
                 }
-                if (nw < NC && (nw < 1 || mbar_test_wait(w_free, static_cast<uint32_t>((nw - 1) & 1)))) {
+                if (nw < lim && (nw < 1 || mbar_test_wait(w_free, static_cast<uint32_t>((nw - 1) & 1)))) {
                     const int r = tma_t0 + nw * 64;
                     mbar_arrive_expect_tx(w_full, Cfg::VAL_TILE);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
@@ -611,7 +898,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ++nw;
                     progress = true;
                 }
-                if (nv < NC && (nv < 1 || mbar_test_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
+                if (nv < lim && (nv < 1 || mbar_test_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
                     const int r = tma_t0 + nv * 64;
                     mbar_arrive_expect_tx(v_full, Cfg::VAL_TILE);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
@@ -619,9 +906,22 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ++nv;
                     progress = true;
                 }
+                lim = min(NC, *stop_at);
                 const uint64_t now = globaltimer_ns();
                 if (progress) t0 = now;
                 else if (now - t0 > wait_ns) { failed = true; break; }
+            }
+            if (!failed && lim < NC) {
+                // handed off: let every issued load land before the shared memory is reused
+                // (the last load of each barrier slot completes that slot's last phase)
+                bool ok = true;
+                for (int j = max(0, nq - 2); j < nq; ++j)
+                    ok = ok && mbar_wait(&qb_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), wait_ns);
+                for (int j = max(0, nk - 3); j < nk; ++j)
+                    ok = ok && mbar_wait(&k_full[j % 3], static_cast<uint32_t>((j / 3) & 1), wait_ns);
+                if (nv > 0) ok = ok && mbar_wait(v_full, static_cast<uint32_t>((nv - 1) & 1), wait_ns);
+                if (nw > 0) ok = ok && mbar_wait(w_full, static_cast<uint32_t>((nw - 1) & 1), wait_ns);
+                if (!ok) failed = true;
             }
         }
     } else if (tid < kKeyThreads) {
@@ -642,8 +942,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK, PREP, VARLEN>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, fz, nrm,
-                                                 min(64, len));
+            else if (grp_b) prep_chunk<DK, PREP, VARLEN>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, 0,
+                                                         stop_at, fz, nrm, min(64, len));
         }
         for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
@@ -652,6 +952,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // prep of chunk m is complete: chunk 0 here, later chunks before the
             // barriers that close the previous iteration
             if (m == 0) named_bar(1, kKeyThreads);
+            if (*stop_at <= m) {   // chunk m and the rest of the sequence go to the token tail
+                if (t == 0) mbar_arrive(&full[s]);   // the chain stops at the same chunk
+                break;
+            }
             // log_alpha of chunk m+1, a whole iteration ahead of its use
             if (grp_b && m + 1 < NC) lan.load(la, tok0, m + 1, h, len, H, t - 128);
             // ---------------------------------------------------------- MMA1
@@ -754,8 +1058,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
                     prep_chunk<DK, PREP, VARLEN>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
-                                                 gC + ((m + 1) % 3) * 128, carry, t - 128, 4, fz, nrm,
-                                                 min(64, len - (m + 1) * 64));
+                                                 gC + ((m + 1) % 3) * 256, carry, t - 128, 4, m + 1, stop_at, fz,
+                                                 nrm, min(64, len - (m + 1) * 64));
             }
             // P (warps 0, 1, 4, 5), T and the prepared tiles are written: hand the
             // chunk to the chain, then MMA3 [. ; T] (W.V) -> T (W.V) in TMEM, whose
@@ -823,8 +1127,41 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             named_bar(2, kChainThreads);
         }
+        if (NC > 0 && S0 != nullptr) {
+            // the chain carries the state scaled by 2^ref of the chunk it enters: S0
+            // takes chunk 0's factor once chunk 0 is prepared (later chunks get theirs
+            // with the state update); the loop's own wait on full[0] then passes at once
+            const bool ok = mbar_wait(&full[0], 0u, wait_ns);
+            if (group_any(2, kChainThreads, !ok)) failed = true;
+            else if (*stop_at > 0) {
+                const int c = t;
+                const float f = gC[128 + c];
+#pragma unroll 1
+                for (int jc = 0; jc < NV / 32; ++jc) {
+                    float sv[32];
+                    tmem_ld32(t_S + lane_q + jc * 32, sv);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sv[e] *= f;
+                    tmem_st32(t_S + lane_q + jc * 32, sv);
+                    if (c < DK) {
+                        const uint32_t tile = sb + Cfg::OFF_S + ((jc * 32) >> 6) * 16384u;
+                        const uint32_t ch0 = ((jc * 32) & 63) >> 3;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            st_shared_v4(tile + sw128_chunk(c, ch0 + q4), pack_bf16x2(sv[8 * q4], sv[8 * q4 + 1]),
+                                         pack_bf16x2(sv[8 * q4 + 2], sv[8 * q4 + 3]),
+                                         pack_bf16x2(sv[8 * q4 + 4], sv[8 * q4 + 5]),
+                                         pack_bf16x2(sv[8 * q4 + 6], sv[8 * q4 + 7]));
+                    }
+                }
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(2, kChainThreads);
+            }
+        }
         uint32_t ph1 = 0, ph2 = 0, ph3 = 0, pht = 0;
-        for (int n = 0; n < NC; ++n) {
+        for (int n = 0; n < NC && !failed; ++n) {
             const int s = n & 1;
             if constexpr (EPI) {   // the epilogue's gate tile, into L2 a whole chain pass ahead
                 const int r = t >> 1;   // two threads per row: 2 x 128-byte lines of the NV slice
@@ -838,6 +1175,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((n >> 1) & 1), wait_ns);
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
+            const int stop_now = *stop_at;   // includes chunk n + 1's decision (its prep is done)
+            if (stop_now <= n) break;        // handed to the token tail from chunk n on
             // ------------------------------------------------------ MMA_s
             if (t == 0) {
                 tc_fence_after();
@@ -947,14 +1286,26 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_after();
             {
                 const int c = t;
-                const float gcv = gC[(n % 3) * 128 + c];
+                // 2^(G_C - ref) of this chunk, then 2^ref of the next one (unless the
+                // next one is handed to the token tail, which takes the plain state).
+                // Two multiplies, each rounded, as a call resumed from S_T takes them
+                // (S_T, then S0 * 2^ref): resuming is exact to the bit.
+                const float gca = gC[(n % 3) * 256 + c];
+                const float gcb = (n + 1 < NC && n + 1 < stop_now) ? gC[((n + 1) % 3) * 256 + 128 + c] : 1.f;
                 const bool last = (n + 1 == NC);
 #pragma unroll 1
                 for (int jc = 0; jc < NV / 32; ++jc) {
                     float sv[32];
                     tmem_ld32(t_S + lane_q + jc * 32, sv);
+                    if (last && S_T != nullptr && c < DK) {
+                        float4 *dst = reinterpret_cast<float4 *>(S_T + (head * DK + c) * d_v + j0 + jc * 32);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) sv[e] *= gcv;
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(sv[4 * e] * gca, sv[4 * e + 1] * gca, sv[4 * e + 2] * gca,
+                                                 sv[4 * e + 3] * gca);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sv[e] = (sv[e] * gca) * gcb;
                     tmem_st32(t_S + lane_q + jc * 32, sv);
                     if (c < DK) {
                         const uint32_t tile = sb + Cfg::OFF_S + ((jc * 32) >> 6) * 16384u;
@@ -965,12 +1316,6 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             st_shared_v4(tile + sw128_chunk(c, ch0 + q4), pack_bf16x2(sv[e], sv[e + 1]),
                                          pack_bf16x2(sv[e + 2], sv[e + 3]), pack_bf16x2(sv[e + 4], sv[e + 5]),
                                          pack_bf16x2(sv[e + 6], sv[e + 7]));
-                        }
-                        if (last && S_T != nullptr) {
-                            float4 *dst = reinterpret_cast<float4 *>(S_T + (head * DK + c) * d_v + j0 + jc * 32);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                dst[e] = make_float4(sv[4 * e], sv[4 * e + 1], sv[4 * e + 2], sv[4 * e + 3]);
                         }
                     }
                 }
@@ -1111,11 +1456,38 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // ------------------------------------------------------------- teardown
     const bool any_failed = __syncthreads_or(failed);
     if (any_failed && tid == 0) record_timeout();
+    // every role has stopped at the same chunk and drained its loads, MMAs and stores
+    const int len_s = reinterpret_cast<const int *>(smem + Cfg::OFF_SEQ)[2];
+    const int nc_s = (len_s + Cfg::C - 1) / Cfg::C;
+    const int stop = any_failed ? nc_s : min(nc_s, *stop_at);
+    if (stop < nc_s && warp >= 8 && warp < 12) {   // the chain warps copy the state out of TMEM
+        tc_fence_after();
+        float *sS = reinterpret_cast<float *>(smem);
+        const int c = tid - kKeyThreads;
+#pragma unroll 1
+        for (int jc = 0; jc < NV / 32; ++jc) {
+            float x[32];
+            tmem_ld32(t_S + lane_q + jc * 32, x);
+            if (c < DK) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(sS + c * (NV + 4) + jc * 32 + e) =
+                        make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::TMEM_COLS);
+    }
+    if (stop < nc_s) {
+        const long tok0_s = *reinterpret_cast<const long *>(smem + Cfg::OFF_SEQ);
+        const int bb_s = reinterpret_cast<const int *>(smem + Cfg::OFF_SEQ)[3];
+        const int hv_s = blockIdx.y;
+        tc_token_tail<DK, NV, PREP, EPI>(smem, ta, la, o, S_T, tok0_s, stop * Cfg::C, len_s, hv_s / (HV / H), H,
+                                         hv_s, HV, blockIdx.x * NV, d_v, (long)bb_s * HV + hv_s, fz);
     }
 }
 

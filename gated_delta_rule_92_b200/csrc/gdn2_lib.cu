@@ -96,7 +96,8 @@ template <int DK, int NV, bool PREP, bool EPI, bool VARLEN>
 gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
                                const CUtensorMap &tv, const CUtensorMap &tw, const CUtensorMap &to, const void *la,
                                const float *S0,
-                               void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz) {
+                               void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz,
+                               const TailArgs &ta) {
     using Cfg = TcCfg<DK, NV>;
     auto kern = chunk_fwd_tc_kernel<DK, NV, PREP, EPI, VARLEN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
@@ -104,7 +105,7 @@ gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, con
     dim3 grid(sh.d_v / NV, sh.HV, sh.B);
     kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, to, static_cast<const __nv_bfloat16 *>(la),
                                                     S0, static_cast<__nv_bfloat16 *>(o), S_T, sh.T, sh.H, sh.HV,
-                                                    sh.d_v, sh.cu, kWaitNs, fz);
+                                                    sh.d_v, sh.cu, kWaitNs, fz, ta);
     return from_cuda(cudaGetLastError());
 }
 
@@ -114,9 +115,10 @@ template <int DK, int NV, bool PREP, bool EPI>
 gdn2_status_t launch_tc_seq(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tb,
                             const CUtensorMap &tv, const CUtensorMap &tw, const CUtensorMap &to, const void *la,
                             const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
-                            const FuseArgs &fz) {
-    if (sh.cu) return launch_tc_kernel<DK, NV, PREP, EPI, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, fz);
-    return launch_tc_kernel<DK, NV, PREP, EPI, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, fz);
+                            const FuseArgs &fz, const TailArgs &ta) {
+    if (sh.cu)
+        return launch_tc_kernel<DK, NV, PREP, EPI, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, fz, ta);
+    return launch_tc_kernel<DK, NV, PREP, EPI, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, fz, ta);
 }
 
 template <int DK, int NV>
@@ -134,11 +136,14 @@ gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void 
     // more pass normalises o in place
     const bool epi = fz != nullptr && fz->gate != nullptr && sh.d_v == NV;
     const FuseArgs kf = fz ? *fz : FuseArgs{};
+    const TailArgs ta{static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                      static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(v),
+                      static_cast<const __nv_bfloat16 *>(w)};
     gdn2_status_t s;
-    if (prep && epi) s = launch_tc_seq<DK, NV, true, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
-    else if (prep) s = launch_tc_seq<DK, NV, true, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
-    else if (epi) s = launch_tc_seq<DK, NV, false, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
-    else s = launch_tc_seq<DK, NV, false, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf);
+    if (prep && epi) s = launch_tc_seq<DK, NV, true, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf, ta);
+    else if (prep) s = launch_tc_seq<DK, NV, true, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf, ta);
+    else if (epi) s = launch_tc_seq<DK, NV, false, true>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf, ta);
+    else s = launch_tc_seq<DK, NV, false, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf, ta);
     if (s != GDN2_OK || fz == nullptr || fz->gate == nullptr || epi) return s;
     return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, sh.rows(), sh.d_v, fz->norm_eps, st);
 }

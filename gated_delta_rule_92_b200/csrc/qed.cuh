@@ -156,6 +156,8 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
 // with Gamma_t the cumulative decay, Q~ = q.Gamma, K~ = kappa/Gamma, E = eps.Gamma.
 // C = 32 tokens make the 64 pseudo-rows of the CUDA-core solve; one block of
 // 256 threads per (b, h, 64-column slice of d_v), everything in shared memory.
+// A chunk that decays by more than e^-kMaxCudaCoreSpan in some channel runs
+// token by token (chunk_token_steps with two pseudo-rows per token) instead.
 template <int DK>
 struct QedCfg {
     static constexpr int C = 32;        // tokens per chunk
@@ -257,6 +259,42 @@ chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
             }
         }
         __syncthreads();
+        // ---- the chunk's decay: past kMaxCudaCoreSpan it runs token by token
+        {
+            float tot = 0.f;
+            if (tid < DK)
+                for (int t = 0; t < C; ++t) tot += sG[t * LK + tid];
+            if (__syncthreads_or(tid < DK && !(tot >= -kMaxCudaCoreSpan))) {
+                // alpha = exp(log_alpha) in place; q . k and q . u per token
+                for (int idx = tid; idx < C * DK; idx += 256) {
+                    const int t = idx / DK, c = idx % DK;
+                    sG[t * LK + c] = __expf(sG[t * LK + c]);
+                }
+                {
+                    const int wp = tid >> 5, l = tid & 31;
+                    for (int t = wp; t < C; t += 8) {
+                        float qk = 0.f, qu = 0.f;
+                        for (int c = l; c < DK; c += 32) {
+                            qk = fmaf(sQ[t * LK + c], sK[(2 * t) * LK + c], qk);
+                            qu = fmaf(sQ[t * LK + c], sK[(2 * t + 1) * LK + c], qu);
+                        }
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) {
+                            qk += __shfl_xor_sync(0xffffffffu, qk, off);
+                            qu += __shfl_xor_sync(0xffffffffu, qu, off);
+                        }
+                        if (l == 0) {
+                            sGC[2 * t] = qk;
+                            sGC[2 * t + 1] = qu;
+                        }
+                    }
+                }
+                __syncthreads();
+                chunk_token_steps<DK, NV, 2, IO>(sQ, sK, sE, sG, sWV, sGC, sS, LK, LV, rows, o,
+                                                 (tok0 * H + h) * (long)d_v + j0, (long)H * d_v);
+                continue;   // the next chunk starts with a barrier
+            }
+        }
         // ---- cumulative log-decay per channel and the scaled operands
         if (tid < DK) {
             const int c = tid;

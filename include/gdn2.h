@@ -34,7 +34,10 @@
  *     S0, S_T, S         : [B, H, d_k, d_v]   always float32
  * Token tensors (q, k, v, log_alpha, b, w, o) share one I/O dtype `io`:
  * GDN2_IO_F32 (float32) or GDN2_IO_BF16 (bfloat16).  log_alpha holds natural
- * logarithms.  Every pointer must be 16-byte aligned.
+ * logarithms: any value in [-inf, 0] is accepted, -inf (alpha = 0) clearing
+ * the state, and every entry point is exact (to rounding) for any decay,
+ * however strong.  Positive values (alpha > 1, a growing state) are outside
+ * the recurrence's domain.  Every pointer must be 16-byte aligned.
  *
  * The caller owns every buffer; the library allocates no device memory.
  * Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = the
@@ -100,6 +103,16 @@ typedef enum {
  * and bf16 I/O with chunk 16 or 32, run the CUDA-core kernel with fp32
  * products throughout.  o is rounded to the I/O
  * dtype (round to nearest even); S_T is fp32.
+ *
+ * Decay range: the chunked form scales its operands by exponentials of the
+ * cumulative decay inside a chunk.  The tensor-core kernel takes those
+ * relative to the middle of the chunk's range and uses the chunked form while
+ * a chunk decays by at most 2^-200 (about e^-139, a mean alpha of 0.11 per
+ * token) over its rows 1..63 in every channel; the first chunk that decays
+ * more, and the rest of its sequence, run token by token in fp32 (slower per
+ * token than the chunked form).  The
+ * CUDA-core kernel makes the same choice chunk by chunk at e^-60.  Either way
+ * the result is the recurrence's, for any log_alpha in [-inf, 0].
  */
 gdn2_status_t gdn2_chunk_fwd(const void *q, const void *k, const void *v,
                              const void *log_alpha, const void *b, const void *w,

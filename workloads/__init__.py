@@ -226,3 +226,41 @@ def gdn_collapse(inp: dict, seed: int, b_scale: float = 1.0) -> dict:
     la = inp["log_alpha"]
     out["log_alpha"] = la[..., :1].expand_as(la).contiguous()
     return out
+
+
+# ------------------------------------------------ strong-decay input variants
+# These only replace log_alpha with other random draws; the recurrence itself
+# accepts any log_alpha <= 0 and these cover the regimes where a chunked
+# evaluation has to keep its exponents in range.
+
+def with_mixed_decay(inp: dict, seed: int, fast=(5e-4, 2e-3), slow=(0.99, 0.9999)) -> dict:
+    """Even key channels decay fast (alpha ~ U[fast]), odd ones barely (alpha ~ U[slow])."""
+    g = torch.Generator().manual_seed(seed)
+    la = inp["log_alpha"]
+    shape = la.shape
+    u = torch.rand(shape, generator=g, dtype=torch.float64)
+    lo = torch.tensor([fast[0], slow[0]], dtype=torch.float64)[torch.arange(shape[-1]) % 2]
+    hi = torch.tensor([fast[1], slow[1]], dtype=torch.float64)[torch.arange(shape[-1]) % 2]
+    out = dict(inp)
+    out["log_alpha"] = torch.log(lo + (hi - lo) * u).to(la.dtype).contiguous()
+    return out
+
+
+def with_decay_spikes(inp: dict, seed: int, prob: float = 0.03, value: float = -20.0) -> dict:
+    """Each (b, t, h) token independently, with probability `prob`, gets
+    log_alpha = `value` on every key channel (a near-reset of the state)."""
+    g = torch.Generator().manual_seed(seed)
+    la = inp["log_alpha"]
+    hit = torch.rand(la.shape[:-1], generator=g) < prob
+    out = dict(inp)
+    out["log_alpha"] = torch.where(hit[..., None], torch.full_like(la, value), la).contiguous()
+    return out
+
+
+def with_decay_burst(inp: dict, t0: int, t1: int, value: float) -> dict:
+    """Tokens t0 <= t < t1 of every sequence and head get log_alpha = `value` (token axis 1)."""
+    la = inp["log_alpha"].clone()
+    la[:, t0:t1] = value
+    out = dict(inp)
+    out["log_alpha"] = la.contiguous()
+    return out
