@@ -15,9 +15,13 @@ JSON line carries:
                copies the inputs in and o, S_T out, the library overlapping
                the copies of one slice of sequences with the kernel of the next;
   roofline     the chunk kernel's algorithmic HBM bytes / launch time vs the
-               measured copy bandwidth;
+               measured copy bandwidth, the tensor-pipe fraction of its useful
+               FLOPs, and the attainable fraction max(t_flop, t_byte) / t;
+  steady       after the K timed steps, rounds of 50 calls over at least
+               0.5 s (per-call median, min, max), under the same clock sampler;
   decode       tokens/s of the decode workload (256 sequences x 16 heads x
-               d128, 1024 consecutive steps) with its own HBM roofline;
+               d128, 1024 consecutive steps) with its own HBM roofline, timed
+               as plain launches and as one captured CUDA graph;
   expanded_v   the d_v=256, b in (0,2) chunk workload;
   cpu_baseline the fp64 oracle on the host cores over a bounded sample.
 With torchrun (N > 1) every rank runs its own batch (weak scaling, no
@@ -204,7 +208,20 @@ def aggregate_throughput(ms_local: float, steps: int, tokens_per_rank_step: int,
 
 
 # ------------------------------------------------------- our measurements
-def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None):
+def steady_rounds(step, stream, min_s: float = 0.5, per_round: int = 50, max_rounds: int = 400):
+    """Rounds of `per_round` back-to-back calls, each timed with CUDA events on
+    `stream`, until `min_s` of device time has been covered; returns the
+    per-call median, min and max over the rounds (ms) and the time covered (s)."""
+    per, total = [], 0.0
+    while total < min_s * 1e3 and len(per) < max_rounds:
+        ms = device_time_ms(step, per_round, stream)
+        per.append(ms / per_round)
+        total += ms
+    return {"rounds": len(per), "calls_per_round": per_round, "ms_per_call_median": statistics.median(per),
+            "ms_per_call_min": min(per), "ms_per_call_max": max(per), "seconds": total / 1e3}
+
+
+def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None, steady_s: float = 0.0):
     d = W.make_chunk_inputs(wl, seed=rank_seed(wl, rank), device="cuda")
     o = torch.empty_like(d["v"])
     S_T = torch.empty(wl.B, wl.H, wl.d_k, wl.d_v, dtype=torch.float32, device="cuda")
@@ -219,15 +236,23 @@ def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    steady = None
     if sampler is not None:
+        # the sampler covers the timed steps and the steady rounds after them
         with sampler:
             ms = device_time_ms(step, steps, stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            if steady_s > 0:
+                steady = steady_rounds(step, stream, steady_s)
     else:
         ms = device_time_ms(step, steps, stream)
-    torch.cuda.synchronize()
-    barrier(world)
+        torch.cuda.synchronize()
+        barrier(world)
     if g.device_status() != 0:
         raise RuntimeError("chunk kernel reported a device timeout")
+    if sampler is not None:
+        return ms, d, o, S_T, steady
     return ms, d, o, S_T
 
 
@@ -420,17 +445,20 @@ def bench_chunk_e2e(g, wl, d, steps, stream, o_dev=None, st_dev=None):
     return ms, h2d, d2h, same
 
 
-def bench_decode(g, wl, steps, rank, stream):
+def bench_decode(g, wl, steps, rank, stream, graph: bool = False):
+    """The decode workload: `steps` consecutive steps, timed on the device.  With
+    graph=True the same steps are also captured once as one CUDA graph and the
+    graph replay is timed; returns (plain ms, graph ms or None)."""
     d = W.make_decode_inputs(wl, steps, seed=rank_seed(wl, rank), device="cuda")
     S = d["S0"].clone()
     o = torch.empty(wl.B, wl.H, wl.d_v, dtype=wl.torch_dtype, device="cuda")
     it = {"s": 0}
 
-    def step():
+    def step(st=stream):
         s = it["s"] % steps
         it["s"] += 1
         g.decode_step(d["q"][s], d["k"][s], d["v"][s], d["log_alpha"][s], d["b"][s], d["w"][s], S,
-                      o=o, stream=stream)
+                      o=o, stream=st)
 
     for _ in range(8):
         step()
@@ -440,7 +468,30 @@ def bench_decode(g, wl, steps, rank, stream):
     ms = device_time_ms(step, steps, stream)
     if g.device_status() != 0:
         raise RuntimeError("decode kernel reported a device timeout")
-    return ms
+    ms_graph = None
+    if graph:
+        cg = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        it["s"] = 0
+        with torch.cuda.graph(cg, stream=cap):
+            for _ in range(steps):
+                step(cap)
+        torch.cuda.synchronize()
+        for _ in range(2):   # warm the graph
+            cg.replay()
+        torch.cuda.synchronize()
+        S.copy_(d["S0"])
+        with torch.cuda.stream(stream):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            cg.replay()
+            e1.record(stream)
+        e1.synchronize()
+        ms_graph = e0.elapsed_time(e1)
+        del cg
+        if g.device_status() != 0:
+            raise RuntimeError("decode kernel reported a device timeout")
+    return ms, ms_graph
 
 
 # --------------------------------------------------------- oracle (CPU)
@@ -476,7 +527,7 @@ def profile_case(g, args, stream):
     import dataclasses
     if args.profile_case == "decode":
         wl = dataclasses.replace(W.BY_NAME["decode_bf16"], decode_steps=args.warmup + args.steps)
-        ms = bench_decode(g, wl, wl.decode_steps, 0, stream)
+        ms, _ = bench_decode(g, wl, wl.decode_steps, 0, stream)
         print(json.dumps({"profile_case": "decode", "workload": wl.describe(),
                           "us_per_step": 1e3 * ms / wl.decode_steps}))
         return
@@ -543,6 +594,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--steady-s", type=float, default=0.5,
+                    help="after the timed steps, time rounds of 50 calls for at least this long (median reported)")
     ap.add_argument("--no-extras", action="store_true", help="skip decode/expanded-value/CPU legs")
     ap.add_argument("--profile-case", choices=["chunk", "chunk_v256", "decode"], default=None,
                     help="only launch one kernel on a reduced batch (inputs still larger than L2), "
@@ -568,8 +621,9 @@ def main():
         profile_case(g, args, stream)
         return
 
-    sampler = ClockSampler()
-    ms, d, o, S_T = bench_chunk(g, wl, args.steps, args.warmup, rank, world, stream, sampler)
+    sampler = ClockSampler(period_s=0.002)
+    ms, d, o, S_T, steady = bench_chunk(g, wl, args.steps, args.warmup, rank, world, stream, sampler,
+                                        steady_s=args.steady_s)
     value, ms_max = aggregate_throughput(ms, args.steps, wl.B * wl.T, world)
     launch_ms = ms / args.steps
     abytes = chunk_bytes(wl, with_s0=d["S0"] is not None)
@@ -595,9 +649,10 @@ def main():
         del d3
         torch.cuda.empty_cache()
         wl4 = W.BY_NAME["decode_bf16"]
-        with ClockSampler() as s4:
-            ms4 = bench_decode(g, wl4, wl4.decode_steps, rank, stream)
+        with ClockSampler(period_s=0.002) as s4:
+            ms4, ms4g = bench_decode(g, wl4, wl4.decode_steps, rank, stream, graph=True)
         ms4 = max_over_ranks(ms4, world)
+        ms4g = max_over_ranks(ms4g, world)
         per = ms4 / wl4.decode_steps
         b4 = decode_bytes(wl4)
         extras["decode"] = {
@@ -606,6 +661,10 @@ def main():
             "roofline": {"bound": "hbm", "achieved": b4 / (per / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": b4 / (per / 1e3) / 1e9 / peaks["hbm_gbs"],
                          "bytes_per_step": b4, "traffic": measured_traffic("decode_step", wl4.B)},
+            "graph": {"value": wl4.B * world * wl4.decode_steps / (ms4g / 1e3), "unit": "tokens/s",
+                      "us_per_step": 1e3 * ms4g / wl4.decode_steps,
+                      "frac": b4 / (ms4g / wl4.decode_steps / 1e3) / 1e9 / peaks["hbm_gbs"],
+                      "how": f"the {wl4.decode_steps} steps captured once as one CUDA graph, one replay timed"},
             "clocks": s4.summary()}
         torch.cuda.empty_cache()
         # f1 + f2: the headline chunk workload and the decode workload from raw
@@ -700,7 +759,11 @@ def main():
                          "traffic": measured_traffic("chunk_fwd_tc", wl.B),
                          "peak_source": peaks["source"], "bytes_per_launch": abytes,
                          "tensor_tflops": flops / (launch_ms / 1e3) / 1e12,
-                         "tensor_frac": flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+                         "tensor_frac": flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                         # max(t_flop, t_byte) / t: the fraction of the tighter of the two bounds
+                         "attainable_frac": max(abytes / (peaks["hbm_gbs"] * 1e9),
+                                                flops / (peaks["bf16_tflops"] * 1e12)) / (launch_ms / 1e3)},
+            "steady": steady,
             "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                     "equals_device_path": e2e_same},

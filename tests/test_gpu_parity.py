@@ -121,29 +121,36 @@ def test_workload_chunk_bf16_small(g):
     _check_chunk(g, g.chunk_fwd, W.make_chunk_inputs(wl))
 
 
+# Sampled heads of the full-size workloads (flat b * H + h): spread over every
+# batch row, first and last head of a row, the very last head included.
+H2048_HEADS = [0, 15, 16, 37, 64, 90, 111, 127]       # B8 x H16
+NEGEIG_HEADS = [0, 15, 17, 30, 33, 47, 50, 63]        # B4 x H16
+
+
 @cuda
 def test_workload_chunk_bf16_h2048_sampled_heads(g):
     wl = W.BY_NAME["chunk_bf16_h2048"]
     inp = W.make_chunk_inputs(wl)
-    _check_chunk(g, g.chunk_fwd, inp, heads=[0, 37, 127])
+    _check_chunk(g, g.chunk_fwd, inp, heads=H2048_HEADS)
 
 
 @cuda
 def test_workload_chunk_bf16_negeig_sampled_heads(g):
     wl = W.BY_NAME["chunk_bf16_negeig"]
     inp = W.make_chunk_inputs(wl)
-    _check_chunk(g, g.chunk_fwd, inp, heads=[0, 63])
+    _check_chunk(g, g.chunk_fwd, inp, heads=NEGEIG_HEADS)
 
 
 @cuda
 @pytest.mark.parametrize("collapse", ["kda", "gdn"])
 def test_workload_negeig_collapses(g, collapse):
-    """Same inputs as the expanded-value workload with b = w = beta (KDA) and
-    additionally a scalar decay per head (Gated DeltaNet)."""
+    """The expanded-value workload at its full size (B4 T8192 H16 d_k 128 d_v 256)
+    with b = w = beta (KDA) and additionally a scalar decay per head (Gated
+    DeltaNet), on sampled heads over all T tokens."""
     wl = W.BY_NAME["chunk_bf16_negeig"]
-    inp = W.make_chunk_inputs(wl, B=1, T=2048)
+    inp = W.make_chunk_inputs(wl)
     f = W.kda_collapse if collapse == "kda" else W.gdn_collapse
-    _check_chunk(g, g.chunk_fwd, f(inp, seed=77, b_scale=wl.b_scale))
+    _check_chunk(g, g.chunk_fwd, f(inp, seed=77, b_scale=wl.b_scale), heads=NEGEIG_HEADS)
 
 
 # ------------------------------------------------------------- decode
@@ -174,6 +181,37 @@ def test_decode_small_all_heads(g, dt, dk, dv):
     tol = TOL[dt]
     assert rel_inf(go, ro) <= tol
     assert rel_inf(state_heads(S, range(B * H), H), rS) <= tol
+
+
+@cuda
+def test_workload_decode_all_1024_steps(g):
+    """The decode workload as specified: 256 sequences x H16 x d128 for 1024
+    consecutive steps from S0 ~ N(0, 0.02).  Every step's o and the final state
+    of 16 sampled heads (spread over the sequences, the last head included)
+    against the oracle run over the same 1024 steps.  The 6.4 GB of inputs are
+    drawn on the device with the workload's recipe; the oracle reads the same
+    cast values of the sampled heads."""
+    import oracle
+    wl = W.BY_NAME["decode_bf16"]
+    steps, H = wl.decode_steps, wl.H
+    heads = [0, 17, 300, 1023, 1500, 2047, 2100, 2600, 3000, 3333, 3600, 3900, 4000, 4050, 4094, 4095]
+    d = W.make_decode_inputs(wl, steps, device="cuda")
+    bi = torch.tensor([x // H for x in heads], device="cuda")
+    hi = torch.tensor([x % H for x in heads], device="cuda")
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    sample = {n: d[n][:, bi, hi].unsqueeze(1).cpu() for n in names}     # [steps, 1, n, d]
+    S0 = d["S0"][bi, hi].unsqueeze(0).cpu()                             # [1, n, d_k, d_v]
+    S = d["S0"].clone()
+    o_hist = torch.empty(steps, len(heads), wl.d_v, dtype=torch.bfloat16, device="cuda")
+    for s in range(steps):
+        o = g.decode_step(*(d[n][s] for n in names), S)
+        o_hist[s] = o[bi, hi]
+    torch.cuda.synchronize()
+    assert g.device_status() == 0
+    ro, rS = oracle.decode_steps(*(sample[n] for n in names), S0)
+    go = o_hist.float().cpu().numpy().transpose(1, 0, 2)               # [n, steps, d_v]
+    assert rel_inf(go, ro) <= TOL[torch.bfloat16]
+    assert rel_inf(S[bi, hi].double().cpu().numpy(), rS) <= TOL[torch.bfloat16]
 
 
 @cuda
