@@ -304,6 +304,8 @@ struct PrepLA {
 // it (exchanged through `carry` and named barrier `bar` over the 128
 // threads).  A half-warp covers 16 consecutive quads = one 128-byte swizzled
 // row, so the 8-byte shared accesses are conflict-free.
+// PACKED takes the products as packed bf16x2 multiplies of the bf16 inputs by
+// the bf16-rounded factors (about one more bf16 rounding per operand).
 // With PREP, q, k, b arrive raw: each row of q and k is scaled by
 // 1 / sqrt(sum^2 + l2_eps) (a pre-pass: thread t sums row t % 64 of q (t < 64)
 // or of k, and leaves the factor in `nrm`) and b becomes sigmoid(b) (x2 with
@@ -312,7 +314,7 @@ struct PrepLA {
 // chunk) hold the next sequence's tokens: they are cleared in the raw q, b, k
 // tiles first, which makes them the same exact no-ops as padding.  This runs
 // only on a sequence's partial last chunk and leaves the loop below as is.
-template <int DK, bool PREP = false, bool VARLEN = false>
+template <int DK, bool PREP = false, bool VARLEN = false, bool PACKED = false>
 __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLA<DK> &law,
                                            float *gc, float *carry, int g, int bar, int chunk,
                                            volatile int *stop_at, const FuseArgs &fz = {},
@@ -433,24 +435,38 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
             sum[3] = fmaf(bf16_hi(la2.y), kLog2e, sum[3]);
             const uint32_t qv[2] = {qw[j].x, qw[j].y}, kv[2] = {kw[j].x, kw[j].y}, bv[2] = {bw[j].x, bw[j].y};
             uint32_t oq[2], oe[2], ok[2];
+            if constexpr (PACKED) {
+                // the scale factors rounded to bf16 and the products taken as packed
+                // bf16x2 multiplies (each rounded once): fewer instructions, about one
+                // more bf16 rounding per operand
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float ga0 = ex2(sum[2 * h]), ga1 = ex2(sum[2 * h + 1]);
-                const float iv0 = ex2(-sum[2 * h]), iv1 = ex2(-sum[2 * h + 1]);
-                float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
-                float b0 = bf16_lo(bv[h]), b1 = bf16_hi(bv[h]);
-                float q0 = bf16_lo(qv[h]), q1 = bf16_hi(qv[h]);
-                if constexpr (PREP) {
-                    k0 *= rk;
-                    k1 *= rk;
-                    q0 *= rq;
-                    q1 *= rq;
-                    b0 = bs * sigmoid_tanh(b0);
-                    b1 = bs * sigmoid_tanh(b1);
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t gap = pack_bf16x2(ex2(sum[2 * h]), ex2(sum[2 * h + 1]));
+                    const uint32_t ivp = pack_bf16x2(ex2(-sum[2 * h]), ex2(-sum[2 * h + 1]));
+                    oq[h] = mul_bf16x2(qv[h], gap);
+                    oe[h] = mul_bf16x2(mul_bf16x2(bv[h], kv[h]), gap);
+                    ok[h] = mul_bf16x2(kv[h], ivp);
                 }
-                oq[h] = pack_bf16x2(q0 * ga0, q1 * ga1);
-                oe[h] = pack_bf16x2(b0 * k0 * ga0, b1 * k1 * ga1);
-                ok[h] = pack_bf16x2(k0 * iv0, k1 * iv1);
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float ga0 = ex2(sum[2 * h]), ga1 = ex2(sum[2 * h + 1]);
+                    const float iv0 = ex2(-sum[2 * h]), iv1 = ex2(-sum[2 * h + 1]);
+                    float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
+                    float b0 = bf16_lo(bv[h]), b1 = bf16_hi(bv[h]);
+                    float q0 = bf16_lo(qv[h]), q1 = bf16_hi(qv[h]);
+                    if constexpr (PREP) {
+                        k0 *= rk;
+                        k1 *= rk;
+                        q0 *= rq;
+                        q1 *= rq;
+                        b0 = bs * sigmoid_tanh(b0);
+                        b1 = bs * sigmoid_tanh(b1);
+                    }
+                    oq[h] = pack_bf16x2(q0 * ga0, q1 * ga1);
+                    oe[h] = pack_bf16x2(b0 * k0 * ga0, b1 * k1 * ga1);
+                    ok[h] = pack_bf16x2(k0 * iv0, k1 * iv1);
+                }
             }
             *reinterpret_cast<uint2 *>(q_t + o[j]) = make_uint2(oq[0], oq[1]);
             *reinterpret_cast<uint2 *>(e_t + o[j]) = make_uint2(oe[0], oe[1]);
@@ -755,6 +771,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const TailArgs ta) {
     static_assert(!EPI || NV <= 128, "epilogue weight slice");
     using Cfg = TcCfg<DK, NV>;
+    // packed bf16x2 operand products in the prep, except where an output epilogue
+    // normalises each row (it turns the extra rounding of small rows into a large
+    // relative error) or the input prep rescales the rows
+    constexpr bool kPackedPrep = !PREP && !EPI;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -942,7 +962,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK, PREP, VARLEN>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, 0,
+            else if (grp_b) prep_chunk<DK, PREP, VARLEN, kPackedPrep>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, 0,
                                                          stop_at, fz, nrm, min(64, len));
         }
         for (int m = 0; m < NC && !failed; ++m) {
@@ -1057,7 +1077,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = ok_b && mbar_wait(&k_full[s3n], static_cast<uint32_t>(((m + 1) / 3) & 1), wait_ns);
                 ok_b = !group_any(4, 128, !ok_b);
                 if (ok_b)
-                    prep_chunk<DK, PREP, VARLEN>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u, lan,
+                    prep_chunk<DK, PREP, VARLEN, kPackedPrep>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0,
+                                                              Cfg::OFF_K + s3n * 16384u, lan,
                                                  gC + ((m + 1) % 3) * 256, carry, t - 128, 4, m + 1, stop_at, fz,
                                                  nrm, min(64, len - (m + 1) * 64));
             }
