@@ -340,7 +340,7 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
         const int r = g & 63;
         const uint8_t *base = (g < 64) ? smem + oqe : smem + okt;
         const uint32_t kstride = (g < 64) ? 16384u : 8192u;
-        float ss = 0.f;
+        float ss[4] = {0.f, 0.f, 0.f, 0.f};   // four partial sums: short dependency chains
 #pragma unroll
         for (int c8 = 0; c8 < DK / 8; ++c8) {
             uint32_t a0, a1, a2, a3;
@@ -348,11 +348,11 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
             const uint32_t aa[4] = {a0, a1, a2, a3};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                ss = fmaf(bf16_lo(aa[e]), bf16_lo(aa[e]), ss);
-                ss = fmaf(bf16_hi(aa[e]), bf16_hi(aa[e]), ss);
+                ss[e] = fmaf(bf16_lo(aa[e]), bf16_lo(aa[e]), ss[e]);
+                ss[e] = fmaf(bf16_hi(aa[e]), bf16_hi(aa[e]), ss[e]);
             }
         }
-        reinterpret_cast<float *>(nrm)[2 * r + (g >> 6)] = l2_inv(ss, fz.l2_eps);
+        reinterpret_cast<float *>(nrm)[2 * r + (g >> 6)] = l2_inv((ss[0] + ss[1]) + (ss[2] + ss[3]), fz.l2_eps);
     }
     // running sums in log2 units (G log2(e)), so that exp(+-G) = 2^(+-sum)
     constexpr float kLog2e = 1.4426950408889634f;
@@ -1326,7 +1326,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                                  sv[4 * e + 3] * gca);
                     }
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) sv[e] = (sv[e] * gca) * gcb;
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 x = mul_f32x2(mul_f32x2(make_float2(sv[e], sv[e + 1]), make_float2(gca, gca)),
+                                                   make_float2(gcb, gcb));
+                        sv[e] = x.x;
+                        sv[e + 1] = x.y;
+                    }
                     tmem_st32(t_S + lane_q + jc * 32, sv);
                     if (c < DK) {
                         const uint32_t tile = sb + Cfg::OFF_S + ((jc * 32) >> 6) * 16384u;

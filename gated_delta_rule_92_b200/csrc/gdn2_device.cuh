@@ -299,6 +299,15 @@ __device__ __forceinline__ float sigmoid_tanh(float x) {
     return fmaf(0.5f, t, 0.5f);
 }
 
+// Two fp32 products in one paired instruction (each rounded as a single multiply).
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
