@@ -47,6 +47,8 @@
 // tcgen05.commit; hand-offs go through mbarriers.  Every wait is bounded; a
 // timeout records an error, drains this CTA's MMAs and returns.
 #pragma once
+#include <type_traits>
+
 #include "decode.cuh"
 #include "gdn2_device.cuh"
 
@@ -498,6 +500,137 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
     fence_proxy_async_smem();
 }
 
+// ------------------------------------------------ second erase direction (QED)
+// With the query-derived erase direction ("The Query Knows What to Forget",
+// mlsanity 2608.13668, abstract; reading in qed.cuh) a chunk is 32 tokens and
+// 64 pseudo-rows: row 2t is token t's key (erase b_t.k_t, value w_t.v_t), row
+// 2t + 1 its query direction u_t (erase c_t.u_t, value 0).  Both rows of a token
+// read the state before the token, so A is strictly lower by token, and only
+// the 32 token rows carry a query (P and O rows 0-31, rows 32-63 zero).  The
+// tiles keep their 64-row shapes; the TMA brings the 32 token rows in as
+//     Q~ rows 0-31: q      Q~ rows 32-63: c      E rows 32-63: b
+//     K~ rows 32-63: k     v rows 32-63: v       w rows 0-31: w
+// and the prep and W.V expand them in place into the pseudo-rows.
+
+// log_alpha of one 32-token chunk for prep thread c (key channel c), 32 values
+// as bf16 pairs (tokens 2i, 2i + 1); tokens past the sequence end read as 0.
+template <int DK>
+struct PrepLAQ {
+    uint32_t v[16];
+    __device__ __forceinline__ void load(const __nv_bfloat16 *la, long tok0, int n, int h, int len, int H, int c) {
+        const unsigned short *p = reinterpret_cast<const unsigned short *>(la);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int r0 = n * 32 + 2 * i;
+            uint32_t lo = 0u, hi = 0u;
+            if (c < DK) {
+                if (r0 < len) lo = __ldg(p + ((tok0 + r0) * H + h) * DK + c);
+                if (r0 + 1 < len) hi = __ldg(p + ((tok0 + r0 + 1) * H + h) * DK + c);
+            }
+            v[i] = lo | (hi << 16);
+        }
+    }
+};
+
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, unsigned short x) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(x) : "memory");
+}
+__device__ __forceinline__ unsigned short bf16_bits(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// Prep of one QED chunk by 128 threads (thread g):
+//  1. per token t (warp g / 32 takes tokens 8 (g / 32) .., lane = channel quad):
+//     coef_t = q.k / k.k (0 when k = 0), r = q - coef_t k, nu_t = 1 / sqrt(r.r + eps)
+//     (0 when that is 0), into scal[t];
+//  2. thread g = key channel c: the running log2-decay G_t over the 32 tokens,
+//     ref = (G_0 + G_31) / 2, and, in place, u_t = (q_t - coef_t k_t) nu_t and
+//     Q~_t = q.2^(G-ref), E_2t = b.k.2^(G-ref), E_2t+1 = c.u.2^(G-ref),
+//     K~_2t = k.2^(ref-G), K~_2t+1 = u.2^(ref-G), Q~ rows 32-63 cleared.
+// Every read and write of channel c in step 2 is thread c's, in token order, so
+// the pseudo-row writes of token t only ever overwrite raw rows of tokens
+// <= t that the thread has already read.  gc and the stop flag as prep_chunk.
+template <int DK>
+__device__ __forceinline__ void prep_chunk_qed(uint8_t *smem, uint32_t oqe, uint32_t okt, const PrepLAQ<DK> &law,
+                                               float *gc, float2 *scal, int g, int bar, int chunk,
+                                               volatile int *stop_at, float qed_eps) {
+    {   // 1. per-token coefficients of the query direction
+        const int w = g >> 5, l = g & 31, p = l;   // channel quad p (4 channels) of tokens 8 w ..
+        const bool act = 4 * p < DK;
+        const int kb = (4 * p) >> 6, cb = ((4 * p) & 63) * 2;   // channel block, byte in the 128-byte row
+        const uint8_t *qt = smem + oqe + kb * 16384, *kt = smem + okt + kb * 8192;
+        auto off = [&](int r) { return r * 128 + ((((cb >> 4) ^ r) & 7) << 4) + (cb & 15); };
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+            const int t = 8 * w + i;
+            float qv[4] = {0.f, 0.f, 0.f, 0.f}, kv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (act) {
+                const uint2 q2 = *reinterpret_cast<const uint2 *>(qt + off(t));
+                const uint2 k2 = *reinterpret_cast<const uint2 *>(kt + off(32 + t));
+                qv[0] = bf16_lo(q2.x); qv[1] = bf16_hi(q2.x); qv[2] = bf16_lo(q2.y); qv[3] = bf16_hi(q2.y);
+                kv[0] = bf16_lo(k2.x); kv[1] = bf16_hi(k2.x); kv[2] = bf16_lo(k2.y); kv[3] = bf16_hi(k2.y);
+            }
+            float qk = 0.f, kk = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                qk = fmaf(qv[e], kv[e], qk);
+                kk = fmaf(kv[e], kv[e], kk);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                qk += __shfl_xor_sync(0xffffffffu, qk, o);
+                kk += __shfl_xor_sync(0xffffffffu, kk, o);
+            }
+            const float coef = kk > 0.f ? qk / kk : 0.f;
+            float rr = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float r = qv[e] - coef * kv[e];
+                rr = fmaf(r, r, rr);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
+            const float den = rr + qed_eps;
+            if (l == 0) scal[t] = make_float2(coef, den > 0.f ? rsqrtf(den) : 0.f);
+        }
+    }
+    named_bar(bar, 128);
+    constexpr float kLog2e = 1.4426950408889634f;
+    const int c = g;
+    if (c < DK) {
+        float total = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) total += (bf16_lo(law.v[i]) + bf16_hi(law.v[i])) * kLog2e;
+        const float g0 = bf16_lo(law.v[0]) * kLog2e;
+        float sum = -0.5f * (g0 + total);   // the running sum enters at -ref
+        const int kb = c >> 6, cc = c & 63;
+        const uint32_t qt = smem_u32(smem + oqe + kb * 16384), et = qt + 8192u, kt = smem_u32(smem + okt + kb * 8192);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const uint32_t lp = law.v[t >> 1];
+            sum = fmaf((t & 1) ? bf16_hi(lp) : bf16_lo(lp), kLog2e, sum);
+            const float ga = ex2(sum), iv = ex2(-sum);
+            const float q = ld_shared_bf16(qt + sw128_off(t, cc));
+            const float cg = ld_shared_bf16(qt + sw128_off(32 + t, cc));
+            const float k = ld_shared_bf16(kt + sw128_off(32 + t, cc));
+            const float b = ld_shared_bf16(et + sw128_off(32 + t, cc));
+            const float2 sc = scal[t];
+            const float u = (q - sc.x * k) * sc.y;
+            st_shared_u16(qt + sw128_off(t, cc), bf16_bits(q * ga));
+            st_shared_u16(qt + sw128_off(32 + t, cc), 0);
+            st_shared_u16(et + sw128_off(2 * t, cc), bf16_bits(b * k * ga));
+            st_shared_u16(et + sw128_off(2 * t + 1, cc), bf16_bits(cg * u * ga));
+            st_shared_u16(kt + sw128_off(2 * t, cc), bf16_bits(k * iv));
+            st_shared_u16(kt + sw128_off(2 * t + 1, cc), bf16_bits(u * iv));
+        }
+        // sum ends at G_31 - ref = -span / 2 (span: the decay of tokens 1..31)
+        gc[c] = ex2(sum);
+        gc[128 + c] = ex2(g0 + sum);
+        if (!(-2.f * sum <= kMaxChunkSpan2)) *stop_at = chunk;
+    }
+    fence_proxy_async_smem();
+}
+
 // Packed sequences: grid slot z runs the sequence of length rank z (longest
 // first, ties by index), so that blocks, which start in z order, begin with
 // the long sequences and the short ones fill in behind them (longest-
@@ -549,6 +682,8 @@ struct BfVec {
 // Raw token pointers for the token tail (the main loop reads through TMA maps).
 struct TailArgs {
     const __nv_bfloat16 *q, *k, *b, *v, *w;
+    const __nv_bfloat16 *c = nullptr;   // QED: the second erase gate
+    float qed_eps = 0.f;                 // QED: epsilon of the direction's norm
 };
 
 // Token tail: a chunk whose decay span passes kMaxChunkSpan2, and every later
@@ -757,20 +892,190 @@ __device__ __noinline__ void tc_token_tail(uint8_t *smem, const TailArgs ta, con
     }
 }
 
+// Token tail of the QED variant: the same hand-off as tc_token_tail, with the
+// rank-2 step of the second erase direction,
+//     u = (q - (q.k / k.k) k) / sqrt(|.|^2 + eps),
+//     r1_j = sum_c (b k alpha)_c S_cj,  r2_j = sum_c (c u alpha)_c S_cj,  p_j = sum_c (q alpha)_c S_cj,
+//     x_j = w_j v_j - r1_j,  S_cj <- alpha_c S_cj + k_c x_j - u_c r2_j,
+//     o_j = p_j + (q . k) x_j - (q . u) r2_j.
+// Layout and hand-off as tc_token_tail; value heads equal key heads.
+template <int DK, int NV>
+__device__ __noinline__ void tc_token_tail_qed(uint8_t *smem, const TailArgs ta, const __nv_bfloat16 *__restrict__ la,
+                                               __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, long tok0,
+                                               int t_begin, int len, int h, int H, int j0, int d_v, long head) {
+    constexpr int TB = 16, LS = NV + 4;
+    constexpr int RR = DK / 8, CJ = NV / 32;
+    constexpr int CPL = DK / 32, JPL = NV / 32;
+    constexpr int kStage = 5, kAll = kTcThreads;
+    constexpr int BAR_FULL = 5, BAR_EMPTY = 7;
+    const float *sS = reinterpret_cast<const float *>(smem);
+    float4 *rowd = reinterpret_cast<float4 *>(smem + DK * LS * 4);     // [2][TB][DK]: alpha, b k alpha, q alpha, k
+    float2 *rowe = reinterpret_cast<float2 *>(rowd + 2 * TB * DK);      // [2][TB][DK]: c u alpha, u
+    float *cold = reinterpret_cast<float *>(rowe + 2 * TB * DK);         // [2][TB][NV]: w v
+    float2 *qkb = reinterpret_cast<float2 *>(cold + 2 * TB * NV);        // [2][TB]: q . k, q . u
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nb = (len - t_begin + TB - 1) / TB;
+    if (warp < 8) {
+        const int rb = lane & 7, cb = lane >> 3, jb = (4 * warp + cb) * CJ;
+        float Sr[RR][CJ];
+#pragma unroll
+        for (int i = 0; i < RR; ++i)
+#pragma unroll
+            for (int x = 0; x < CJ; ++x) Sr[i][x] = sS[(8 * i + rb) * LS + jb + x];
+        for (int k = 0; k < nb; ++k) {
+            const int buf = k & 1, tb = t_begin + k * TB, nt = min(TB, len - tb);
+            named_bar(BAR_FULL + buf, kAll);
+            for (int tt = 0; tt < nt; ++tt) {
+                const float4 *rd = rowd + (buf * TB + tt) * DK;
+                const float2 *re = rowe + (buf * TB + tt) * DK;
+                float r1[CJ], r2[CJ], pq[CJ];
+#pragma unroll
+                for (int x = 0; x < CJ; ++x) r1[x] = r2[x] = pq[x] = 0.f;
+#pragma unroll
+                for (int i = 0; i < RR; ++i) {
+                    const float4 xr = rd[8 * i + rb];
+                    const float2 xe = re[8 * i + rb];
+#pragma unroll
+                    for (int x = 0; x < CJ; ++x) {
+                        r1[x] = fmaf(xr.y, Sr[i][x], r1[x]);
+                        r2[x] = fmaf(xe.x, Sr[i][x], r2[x]);
+                        pq[x] = fmaf(xr.z, Sr[i][x], pq[x]);
+                    }
+                }
+#pragma unroll
+                for (int off = 1; off < 8; off <<= 1)
+#pragma unroll
+                    for (int x = 0; x < CJ; ++x) {
+                        r1[x] += __shfl_xor_sync(0xffffffffu, r1[x], off);
+                        r2[x] += __shfl_xor_sync(0xffffffffu, r2[x], off);
+                        pq[x] += __shfl_xor_sync(0xffffffffu, pq[x], off);
+                    }
+                const float2 qs = qkb[buf * TB + tt];
+                float x1[CJ], ov[CJ];
+#pragma unroll
+                for (int x = 0; x < CJ; ++x) {
+                    x1[x] = cold[(buf * TB + tt) * NV + jb + x] - r1[x];
+                    ov[x] = fmaf(qs.x, x1[x], fmaf(-qs.y, r2[x], pq[x]));
+                }
+#pragma unroll
+                for (int i = 0; i < RR; ++i) {
+                    const float4 xr = rd[8 * i + rb];
+                    const float2 xe = re[8 * i + rb];
+#pragma unroll
+                    for (int x = 0; x < CJ; ++x)
+                        Sr[i][x] = fmaf(xr.x, Sr[i][x], fmaf(xr.w, x1[x], -xe.y * r2[x]));
+                }
+                if (rb == 0) {
+                    __nv_bfloat16 *dst = o + ((tok0 + tb + tt) * H + h) * (long)d_v + j0 + jb;
+#pragma unroll
+                    for (int x = 0; x < CJ; x += 2)
+                        *reinterpret_cast<uint32_t *>(dst + x) = pack_bf16x2(ov[x], ov[x + 1]);
+                }
+            }
+            if (k + 2 < nb) named_bar_arrive(BAR_EMPTY + buf, kAll);
+        }
+        if (S_T != nullptr) {
+#pragma unroll
+            for (int i = 0; i < RR; ++i) {
+                float *dst = S_T + (head * DK + 8 * i + rb) * d_v + j0 + jb;
+#pragma unroll
+                for (int x = 0; x < CJ; ++x) dst[x] = Sr[i][x];
+            }
+        }
+    } else {
+        constexpr int MT = (TB + kStage - 1) / kStage;
+        const int sw = warp - 8;
+        for (int k = 0; k < nb; ++k) {
+            const int buf = k & 1, tb = t_begin + k * TB, nt = min(TB, len - tb);
+            if (k >= 2) named_bar(BAR_EMPTY + buf, kAll);
+            BfVec<CPL> rq[MT], rk[MT], rbv[MT], rc[MT], rl[MT];
+            BfVec<JPL> rv[MT], rw[MT];
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const int tt = sw + kStage * m;
+                if (tt < nt) {
+                    const long tok = tok0 + tb + tt;
+                    const long kro = (tok * H + h) * DK + CPL * lane;
+                    const long vro = (tok * H + h) * (long)d_v + j0 + JPL * lane;
+                    rq[m].load(ta.q + kro);
+                    rk[m].load(ta.k + kro);
+                    rbv[m].load(ta.b + kro);
+                    rc[m].load(ta.c + kro);
+                    rl[m].load(la + kro);
+                    rv[m].load(ta.v + vro);
+                    rw[m].load(ta.w + vro);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const int tt = sw + kStage * m;
+                if (tt >= nt) continue;   // warp-uniform
+                float qv[CPL], kv[CPL];
+                float qk = 0.f, kk = 0.f;
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    qv[e] = rq[m].get(e);
+                    kv[e] = rk[m].get(e);
+                    qk = fmaf(qv[e], kv[e], qk);
+                    kk = fmaf(kv[e], kv[e], kk);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    qk += __shfl_xor_sync(0xffffffffu, qk, off);
+                    kk += __shfl_xor_sync(0xffffffffu, kk, off);
+                }
+                const float coef = kk > 0.f ? qk / kk : 0.f;
+                float rr = 0.f;
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    const float r = qv[e] - coef * kv[e];
+                    rr = fmaf(r, r, rr);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, off);
+                const float den = rr + ta.qed_eps, nu = den > 0.f ? rsqrtf(den) : 0.f;
+                float qu = 0.f;
+                float4 *rdst = rowd + (buf * TB + tt) * DK + CPL * lane;
+                float2 *edst = rowe + (buf * TB + tt) * DK + CPL * lane;
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) {
+                    const float a = __expf(rl[m].get(e));
+                    const float u = (qv[e] - coef * kv[e]) * nu;
+                    qu = fmaf(qv[e], u, qu);
+                    rdst[e] = make_float4(a, rbv[m].get(e) * kv[e] * a, qv[e] * a, kv[e]);
+                    edst[e] = make_float2(rc[m].get(e) * u * a, u);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) qu += __shfl_xor_sync(0xffffffffu, qu, off);
+                if (lane == 0) qkb[buf * TB + tt] = make_float2(qk, qu);
+                float *cdst = cold + (buf * TB + tt) * NV + JPL * lane;
+#pragma unroll
+                for (int e = 0; e < JPL; ++e) cdst[e] = rw[m].get(e) * rv[m].get(e);
+            }
+            named_bar_arrive(BAR_FULL + buf, kAll);
+        }
+    }
+}
+
 // PREP fuses the input prep (raw q, k, b, w); EPI the gated RMS norm of each
 // output row before it is stored (d_v == NV: one CTA holds the whole row).
-template <int DK, int NV, bool PREP = false, bool EPI = false, bool VARLEN = false>
+template <int DK, int NV, bool PREP = false, bool EPI = false, bool VARLEN = false, bool QED = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
 chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o,
+                    const __grid_constant__ CUtensorMap tm_c,
                     const __nv_bfloat16 *__restrict__ la,
                     const float *__restrict__ S0,
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ S_T, int T, int H, int HV, int d_v,
                     const int *__restrict__ cu_seqlens, unsigned long long wait_ns, const FuseArgs fz,
                     const TailArgs ta) {
     static_assert(!EPI || NV <= 128, "epilogue weight slice");
+    static_assert(!QED || (!PREP && !EPI && !VARLEN), "the QED variant has no fusion and no packing");
     using Cfg = TcCfg<DK, NV>;
+    // tokens per chunk: 64, or 32 with the query direction (two pseudo-rows each)
+    constexpr int CH = QED ? 32 : 64;
+    constexpr uint32_t KEY_BYTES = CH * DK * 2u, VAL_BYTES = CH * NV * 2u;   // one tensor, one chunk (TMA)
     // packed bf16x2 operand products in the prep, except where an output epilogue
     // normalises each row (it turns the extra rounding of small rows into a large
     // relative error) or the input prep rescales the rows
@@ -802,7 +1107,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         tma_t0 = a;
         tma_b = 0;
     }
-    const int NC = (len + Cfg::C - 1) / Cfg::C;   // the last chunk may be partial
+    const int NC = (len + CH - 1) / CH;   // the last chunk may be partial
     const long head = (long)bb * HV + hv;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
@@ -869,11 +1174,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // padded tokens exact no-ops of the recurrence (k = q = b = w = 0 and
             // log_alpha = 0).
             auto prefetch = [&](int n) {
-                const int r = tma_t0 + n * 64;
+                const int r = tma_t0 + n * CH;
                 for (int kb = 0; kb < DK / 64; ++kb) {
                     tma_prefetch_l2_4d(&tm_q, kb * 64, h, r, tma_b);
                     tma_prefetch_l2_4d(&tm_k, kb * 64, h, r, tma_b);
                     tma_prefetch_l2_4d(&tm_b, kb * 64, h, r, tma_b);
+                    if constexpr (QED) tma_prefetch_l2_4d(&tm_c, kb * 64, h, r, tma_b);
                 }
                 for (int vb = 0; vb < Cfg::VB; ++vb) {
                     tma_prefetch_l2_4d(&tm_v, j0 + vb * 64, hv, r, tma_b);
@@ -891,38 +1197,46 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             while (nq < lim || nk < lim || nw < lim || nv < lim) {
                 bool progress = false;
                 if (nq < lim && (nq < 2 || mbar_test_wait(&empty_qe[nq & 1], static_cast<uint32_t>(((nq >> 1) - 1) & 1)))) {
-                    const int s = nq & 1, r = tma_t0 + nq * 64;
+                    const int s = nq & 1, r = tma_t0 + nq * CH;
                     const uint32_t oqe = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0;
-                    mbar_arrive_expect_tx(&qb_full[s], 2u * Cfg::KEY_TILE);
+                    mbar_arrive_expect_tx(&qb_full[s], (QED ? 3u : 2u) * KEY_BYTES);
                     for (int kb = 0; kb < DK / 64; ++kb) {
                         tma_load_4d(smem + oqe + kb * 16384, &tm_q, &qb_full[s], kb * 64, h, r, tma_b);
-                        tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qb_full[s], kb * 64, h, r, tma_b);
+                        if constexpr (QED) {   // c into Q~ rows 32-63, b into E rows 32-63
+                            tma_load_4d(smem + oqe + kb * 16384 + 4096, &tm_c, &qb_full[s], kb * 64, h, r, tma_b);
+                            tma_load_4d(smem + oqe + kb * 16384 + 8192 + 4096, &tm_b, &qb_full[s], kb * 64, h, r,
+                                        tma_b);
+                        } else {
+                            tma_load_4d(smem + oqe + kb * 16384 + 8192, &tm_b, &qb_full[s], kb * 64, h, r, tma_b);
+                        }
                     }
                     if (nq + kPrefetch < NC) prefetch(nq + kPrefetch);
                     ++nq;
                     progress = true;
                 }
                 if (nk < lim && (nk < 3 || mbar_test_wait(&empty_k[nk % 3], static_cast<uint32_t>((nk / 3 - 1) & 1)))) {
-                    const int s3 = nk % 3, r = tma_t0 + nk * 64;
-                    mbar_arrive_expect_tx(&k_full[s3], Cfg::KEY_TILE);
-                    for (int kb = 0; kb < DK / 64; ++kb)
-                        tma_load_4d(smem + Cfg::OFF_K + s3 * 16384 + kb * 8192, &tm_k, &k_full[s3], kb * 64, h, r, tma_b);
+                    const int s3 = nk % 3, r = tma_t0 + nk * CH;
+                    mbar_arrive_expect_tx(&k_full[s3], KEY_BYTES);
+                    for (int kb = 0; kb < DK / 64; ++kb)   // QED: k into K~ rows 32-63
+                        tma_load_4d(smem + Cfg::OFF_K + s3 * 16384 + kb * 8192 + (QED ? 4096 : 0), &tm_k, &k_full[s3],
+                                    kb * 64, h, r, tma_b);
                     ++nk;
                     progress = true;
                 }
                 if (nw < lim && (nw < 1 || mbar_test_wait(w_free, static_cast<uint32_t>((nw - 1) & 1)))) {
-                    const int r = tma_t0 + nw * 64;
-                    mbar_arrive_expect_tx(w_full, Cfg::VAL_TILE);
+                    const int r = tma_t0 + nw * CH;
+                    mbar_arrive_expect_tx(w_full, VAL_BYTES);
                     for (int vb = 0; vb < Cfg::VB; ++vb)
                         tma_load_4d(smem + Cfg::OFF_W + vb * 8192, &tm_w, w_full, j0 + vb * 64, hv, r, tma_b);
                     ++nw;
                     progress = true;
                 }
                 if (nv < lim && (nv < 1 || mbar_test_wait(v_free, static_cast<uint32_t>((nv - 1) & 1)))) {
-                    const int r = tma_t0 + nv * 64;
-                    mbar_arrive_expect_tx(v_full, Cfg::VAL_TILE);
-                    for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_load_4d(smem + Cfg::OFF_V + vb * 8192, &tm_v, v_full, j0 + vb * 64, hv, r, tma_b);
+                    const int r = tma_t0 + nv * CH;
+                    mbar_arrive_expect_tx(v_full, VAL_BYTES);
+                    for (int vb = 0; vb < Cfg::VB; ++vb)   // QED: v into rows 32-63
+                        tma_load_4d(smem + Cfg::OFF_V + vb * 8192 + (QED ? 4096 : 0), &tm_v, v_full, j0 + vb * 64, hv,
+                                    r, tma_b);
                     ++nv;
                     progress = true;
                 }
@@ -955,15 +1269,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         bool mma3_failed = false;   // thread 0 only
         float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
         float2 *nrm = reinterpret_cast<float2 *>(smem + Cfg::OFF_NRM);
-        PrepLA<DK> lan;   // group B: log_alpha of the next chunk to prepare
+        // group B: log_alpha of the next chunk to prepare
+        typename std::conditional<QED, PrepLAQ<DK>, PrepLA<DK>>::type lan;
+        // prep of chunk n (stage sn of the Q~/E tiles, stage s3n of K~) by group B
+        auto prep = [&](int n, uint32_t oqe, uint32_t okt) {
+            if constexpr (QED)
+                prep_chunk_qed<DK>(smem, oqe, okt, lan, gC + (n % 3) * 256, nrm, t - 128, 4, n, stop_at, ta.qed_eps);
+            else
+                prep_chunk<DK, PREP, VARLEN, kPackedPrep>(smem, oqe, okt, lan, gC + (n % 3) * 256, carry, t - 128, 4,
+                                                          n, stop_at, fz, nrm, min(64, len - n * 64));
+        };
         // prologue: prep of chunk 0 (group B)
         if (NC > 0) {
             if (grp_b) lan.load(la, tok0, 0, h, len, H, t - 128);
             bool ok = mbar_wait(&qb_full[0], 0u, wait_ns);
             ok = ok && mbar_wait(&k_full[0], 0u, wait_ns);
             if (group_any(1, kKeyThreads, !ok)) failed = true;
-            else if (grp_b) prep_chunk<DK, PREP, VARLEN, kPackedPrep>(smem, Cfg::OFF_QE0, Cfg::OFF_K, lan, gC, carry, t - 128, 4, 0,
-                                                         stop_at, fz, nrm, min(64, len));
+            else if (grp_b) prep(0, Cfg::OFF_QE0, Cfg::OFF_K);
         }
         for (int m = 0; m < NC && !failed; ++m) {
             const int s = m & 1;
@@ -995,8 +1317,32 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 bool ok = mbar_wait(v_full, static_cast<uint32_t>(m & 1), wait_ns);
                 ok = ok && mbar_wait(w_full, static_cast<uint32_t>(m & 1), wait_ns);
                 if (group_any(1, kKeyThreads, !ok)) { failed = true; break; }
+                if constexpr (QED) {
+                    // 32 tokens of v (rows 32-63) and w (rows 0-31) -> pseudo-rows 2t = w.v,
+                    // 2t + 1 = 0: every raw row is read before any expanded row is written
+                    constexpr int CPR = NV / 8, PPT = 32 * CPR / kKeyThreads;   // 16-byte chunks
+                    uint4 wv[PPT];
 #pragma unroll
-                for (int it = 0; it < Cfg::VAL_TILE / 16 / kKeyThreads; ++it) {
+                    for (int i = 0; i < PPT; ++i) {
+                        const int idx = t + i * kKeyThreads, tok = idx / CPR, ch = idx % CPR;
+                        const uint32_t sub = (ch >> 3) * 8192u;
+                        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+                        ld_shared_v4(sb + Cfg::OFF_V + sub + sw128_chunk(32 + tok, ch & 7), a0, a1, a2, a3);
+                        ld_shared_v4(sb + Cfg::OFF_W + sub + sw128_chunk(tok, ch & 7), b0, b1, b2, b3);
+                        wv[i] = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));
+                    }
+                    named_bar(1, kKeyThreads);
+#pragma unroll
+                    for (int i = 0; i < PPT; ++i) {
+                        const int idx = t + i * kKeyThreads, tok = idx / CPR, ch = idx % CPR;
+                        const uint32_t sub = (ch >> 3) * 8192u;
+                        st_shared_v4(sb + Cfg::OFF_V + sub + sw128_chunk(2 * tok, ch & 7), wv[i].x, wv[i].y, wv[i].z,
+                                     wv[i].w);
+                        st_shared_v4(sb + Cfg::OFF_V + sub + sw128_chunk(2 * tok + 1, ch & 7), 0u, 0u, 0u, 0u);
+                    }
+                }
+#pragma unroll
+                for (int it = 0; it < (QED ? 0 : Cfg::VAL_TILE / 16 / kKeyThreads); ++it) {
                     const uint32_t off = (t + it * kKeyThreads) * 16u;
                     uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
                     ld_shared_v4(sb + Cfg::OFF_V + off, a0, a1, a2, a3);
@@ -1036,8 +1382,18 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // warp-uniform block position: columns 32 kh.. against rows 32 (kq % 2)..;
                 // only the diagonal block needs per-element masks
                 const int rb = kq & 1, r = 32 * rb + l;
+                if constexpr (QED) {   // masks by token: pseudo-rows 2t, 2t + 1 belong to token t
+                    if (kq < 2) {   // P: token row r (rows 32-63 hold no token) sees rows <= 2r + 1
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = (rb == 0 && 32 * kh + e <= 2 * l + 1) ? x[e] : 0.f;
+                    } else {        // A: pseudo-row r sees the rows of earlier tokens only
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = (32 * kh + e < (r & ~1)) ? x[e] : 0.f;
+                    }
+                }
                 if (kq < 2) {   // P = lower(Q~ K~^T), diagonal included
-                    if (kh > rb) {
+                    if (QED) {
+                    } else if (kh > rb) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) x[e] = 0.f;
                     } else if (kh == rb) {
@@ -1050,7 +1406,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                      pack_bf16x2(x[8 * q4 + 2], x[8 * q4 + 3]), pack_bf16x2(x[8 * q4 + 4], x[8 * q4 + 5]),
                                      pack_bf16x2(x[8 * q4 + 6], x[8 * q4 + 7]));
                 } else {        // A = strict_lower(E K~^T), fp32 into the solve scratch
-                    if (kh > rb) {
+                    if (QED) {
+                    } else if (kh > rb) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) x[e] = 0.f;
                     } else if (kh == rb) {
@@ -1076,11 +1433,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok_b = mbar_wait(&qb_full[sn], static_cast<uint32_t>(((m + 1) >> 1) & 1), wait_ns);
                 ok_b = ok_b && mbar_wait(&k_full[s3n], static_cast<uint32_t>(((m + 1) / 3) & 1), wait_ns);
                 ok_b = !group_any(4, 128, !ok_b);
-                if (ok_b)
-                    prep_chunk<DK, PREP, VARLEN, kPackedPrep>(smem, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0,
-                                                              Cfg::OFF_K + s3n * 16384u, lan,
-                                                 gC + ((m + 1) % 3) * 256, carry, t - 128, 4, m + 1, stop_at, fz,
-                                                 nrm, min(64, len - (m + 1) * 64));
+                if (ok_b) prep(m + 1, sn ? Cfg::OFF_QE1 : Cfg::OFF_QE0, Cfg::OFF_K + s3n * 16384u);
             }
             // P (warps 0, 1, 4, 5), T and the prepared tiles are written: hand the
             // chunk to the chain, then MMA3 [. ; T] (W.V) -> T (W.V) in TMEM, whose
@@ -1356,7 +1709,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // except on the partial last chunk of a packed sequence, whose rows past
             // the end belong to the next sequence
             const bool o_tma = !EPI && (!VARLEN || (n + 1) * 64 <= len);
-            if ((warp & 3) < 2 && o_tma) {
+            if ((warp & 3) < (QED ? 1 : 2) && o_tma) {   // QED: the 32 token rows only
                 const int r = t;   // output row r (TMEM lanes 0-63)
 #pragma unroll 1
                 for (int jc = 0; jc < NV / 32; ++jc) {
@@ -1372,7 +1725,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                      pack_bf16x2(x[e + 6], x[e + 7]));
                     }
                 }
-            } else if ((warp & 3) < 2) {
+            } else if ((warp & 3) < 2 && !o_tma) {
                 const int r = t;   // output row r (TMEM lanes 0-63); rows past T are padding
                 const bool valid = n * 64 + r < len;
                 const long orow_off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0;
@@ -1467,7 +1820,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (o_tma) {   // rows past T lie outside the tensor and are not written
 #pragma unroll
                     for (int vb = 0; vb < Cfg::VB; ++vb)
-                        tma_store_4d(&tm_o, smem + Cfg::OFF_U + vb * 8192, j0 + vb * 64, hv, tma_t0 + n * 64, tma_b);
+                        tma_store_4d(&tm_o, smem + Cfg::OFF_U + vb * 8192, j0 + vb * 64, hv, tma_t0 + n * CH, tma_b);
                     bulk_commit_group();
                 }
             }
@@ -1484,7 +1837,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (any_failed && tid == 0) record_timeout();
     // every role has stopped at the same chunk and drained its loads, MMAs and stores
     const int len_s = reinterpret_cast<const int *>(smem + Cfg::OFF_SEQ)[2];
-    const int nc_s = (len_s + Cfg::C - 1) / Cfg::C;
+    const int nc_s = (len_s + CH - 1) / CH;
     const int stop = any_failed ? nc_s : min(nc_s, *stop_at);
     if (stop < nc_s && warp >= 8 && warp < 12) {   // the chain warps copy the state out of TMEM
         tc_fence_after();
@@ -1512,8 +1865,12 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const long tok0_s = *reinterpret_cast<const long *>(smem + Cfg::OFF_SEQ);
         const int bb_s = reinterpret_cast<const int *>(smem + Cfg::OFF_SEQ)[3];
         const int hv_s = blockIdx.y;
-        tc_token_tail<DK, NV, PREP, EPI>(smem, ta, la, o, S_T, tok0_s, stop * Cfg::C, len_s, hv_s / (HV / H), H,
-                                         hv_s, HV, blockIdx.x * NV, d_v, (long)bb_s * HV + hv_s, fz);
+        if constexpr (QED)
+            tc_token_tail_qed<DK, NV>(smem, ta, la, o, S_T, tok0_s, stop * CH, len_s, hv_s, H, blockIdx.x * NV, d_v,
+                                      (long)bb_s * HV + hv_s);
+        else
+            tc_token_tail<DK, NV, PREP, EPI>(smem, ta, la, o, S_T, tok0_s, stop * CH, len_s, hv_s / (HV / H), H,
+                                             hv_s, HV, blockIdx.x * NV, d_v, (long)bb_s * HV + hv_s, fz);
     }
 }
 

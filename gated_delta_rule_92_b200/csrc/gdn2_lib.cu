@@ -59,15 +59,16 @@ EncodeTiledFn encode_fn() {
 }
 
 // Token tensor [B, T, H, d] bf16 viewed as 4-D (d, H, T, B); box = 64 channels
-// x 1 head x 64 tokens x 1 sequence, 128-byte swizzle.  Boxes that run past T
-// are zero-filled by the TMA unit (a partial last chunk).
-bool make_token_map(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
+// x 1 head x `rows` tokens (64, or 32 for the QED chunks) x 1 sequence,
+// 128-byte swizzle.  Boxes that run past T are zero-filled by the TMA unit (a
+// partial last chunk).
+bool make_token_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, int rows = 64) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)d * 2u, (cuuint64_t)H * (cuuint64_t)d * 2u,
                              (cuuint64_t)T * (cuuint64_t)H * (cuuint64_t)d * 2u};
-    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -103,7 +104,7 @@ gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, con
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return GDN2_ERR_CUDA;
     dim3 grid(sh.d_v / NV, sh.HV, sh.B);
-    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, to, static_cast<const __nv_bfloat16 *>(la),
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, to, tq, static_cast<const __nv_bfloat16 *>(la),
                                                     S0, static_cast<__nv_bfloat16 *>(o), S_T, sh.T, sh.H, sh.HV,
                                                     sh.d_v, sh.cu, kWaitNs, fz, ta);
     return from_cuda(cudaGetLastError());
@@ -146,6 +147,34 @@ gdn2_status_t launch_tc(const void *q, const void *k, const void *v, const void 
     else s = launch_tc_seq<DK, NV, false, false>(tq, tk, tb, tv, tw, to, la, S0, o, S_T, sh, st, kf, ta);
     if (s != GDN2_OK || fz == nullptr || fz->gate == nullptr || epi) return s;
     return launch_rmsnorm<__nv_bfloat16>(o, fz->gate, fz->norm_weight, sh.rows(), sh.d_v, fz->norm_eps, st);
+}
+
+// The second erase direction on the tensor-core kernel (bf16 I/O): 32 tokens a
+// chunk, token maps with 32-row boxes, the gate c through its own map.
+template <int DK, int NV>
+gdn2_status_t launch_tc_qed(const void *q, const void *k, const void *v, const void *la, const void *b,
+                            const void *c, const void *w, const float *S0, void *o, float *S_T, int B, int T, int H,
+                            int d_v, float eps, cudaStream_t st) {
+    using Cfg = TcCfg<DK, NV>;
+    CUtensorMap tq, tk, tb, tc, tv, tw, to;
+    if (!make_token_map(&tq, q, B, T, H, DK, 32) || !make_token_map(&tk, k, B, T, H, DK, 32) ||
+        !make_token_map(&tb, b, B, T, H, DK, 32) || !make_token_map(&tc, c, B, T, H, DK, 32) ||
+        !make_token_map(&tv, v, B, T, H, d_v, 32) || !make_token_map(&tw, w, B, T, H, d_v, 32) ||
+        !make_token_map(&to, o, B, T, H, d_v, 32))
+        return GDN2_ERR_CUDA;
+    auto kern = chunk_fwd_tc_kernel<DK, NV, false, false, false, true>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC) != cudaSuccess)
+        return GDN2_ERR_CUDA;
+    TailArgs ta{static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                static_cast<const __nv_bfloat16 *>(b), static_cast<const __nv_bfloat16 *>(v),
+                static_cast<const __nv_bfloat16 *>(w)};
+    ta.c = static_cast<const __nv_bfloat16 *>(c);
+    ta.qed_eps = eps;
+    dim3 grid(d_v / NV, H, B);
+    kern<<<grid, kTcThreads, Cfg::SMEM_ALLOC, st>>>(tq, tk, tb, tv, tw, to, tc, static_cast<const __nv_bfloat16 *>(la),
+                                                    S0, static_cast<__nv_bfloat16 *>(o), S_T, T, H, H, d_v, nullptr,
+                                                    kWaitNs, FuseArgs{}, ta);
+    return from_cuda(cudaGetLastError());
 }
 
 template <typename IO, int DK, int CH>
@@ -597,9 +626,13 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_qed(const void *q, const void *k, const 
         if (d_k == 64) return launch_qed_chunk<float, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
         return launch_qed_chunk<float, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
     }
+    // bf16 I/O: the tensor-core kernel
+    const bool wide = (d_v % 128 == 0);
     if (d_k == 64)
-        return launch_qed_chunk<__nv_bfloat16, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
-    return launch_qed_chunk<__nv_bfloat16, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
+        return wide ? launch_tc_qed<64, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st)
+                    : launch_tc_qed<64, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
+    return wide ? launch_tc_qed<128, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st)
+                : launch_tc_qed<128, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
 }
 
 extern "C" gdn2_status_t gdn2_decode_step_qed(const void *q, const void *k, const void *v, const void *log_alpha,

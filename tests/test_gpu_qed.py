@@ -70,8 +70,50 @@ def test_chunk_qed_zero_epsilon(g):
 
 
 def test_chunk_qed_headline_size_sampled(g):
-    """B8 T4096 H16 d128 bf16, sampled heads."""
-    _check_chunk(g, 8, 4096, 16, 128, 128, torch.bfloat16, seed=8200, heads=[0, 45, 127])
+    """B8 T4096 H16 d128 bf16 (the tensor-core kernel), 8 heads over every batch row."""
+    _check_chunk(g, 8, 4096, 16, 128, 128, torch.bfloat16, seed=8200, heads=[0, 15, 16, 45, 64, 90, 111, 127])
+
+
+# bf16 I/O runs the tensor-core kernel: 32 tokens (64 pseudo-rows) a chunk
+TC_CASES = [  # B, T, H, d_k, d_v
+    (2, 200, 2, 128, 256),   # two 128-column slices, partial last chunk
+    (1, 97, 2, 64, 128),     # 3 chunks + 1 token
+    (1, 32, 1, 128, 128),    # exactly one chunk
+    (1, 1, 1, 128, 64),      # a single token
+    (3, 64, 1, 64, 64),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "B%dT%dH%dk%dv%d" % c)
+def test_chunk_qed_tensor_core(g, case):
+    B, T, H, dk, dv = case
+    _check_chunk(g, B, T, H, dk, dv, torch.bfloat16, seed=8250 + T + dv)
+
+
+def test_chunk_qed_tensor_core_zero_gate_matches_gdn2(g):
+    """c = 0 leaves GDN-2: the tensor-core QED kernel (32-token chunks) and the
+    GDN-2 tensor-core kernel (64-token chunks) agree within the bf16 bar."""
+    inp = to_dev(_inputs(2, 300, 2, 128, 128, torch.bfloat16, 8410))
+    inp["c"] = torch.zeros_like(inp["c"])
+    o1, S1 = _run_chunk(g, inp)
+    o2, S2 = g.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["b"], inp["w"], inp["S0"])
+    torch.cuda.synchronize()
+    assert float((o1.float() - o2.float()).abs().max()) <= 2e-2 * float(o2.float().abs().max())
+    assert float((S1 - S2).abs().max()) <= 2e-2 * float(S2.abs().max())
+
+
+def test_chunk_qed_tensor_core_state_split_resume(g):
+    """A run resumed from S_T at a chunk boundary equals the whole run bit for bit."""
+    inp = to_dev(_inputs(1, 256, 2, 128, 128, torch.bfloat16, 8420))
+    names = ("q", "k", "v", "log_alpha", "b", "c", "w")
+    part = lambda sl: {**{n: inp[n][:, sl].contiguous() for n in names}}
+    o, S = g.chunk_fwd_qed(*(inp[n] for n in ("q", "k", "v", "log_alpha", "b", "c", "w")), inp["S0"])
+    a, b = part(slice(0, 96)), part(slice(96, 256))
+    o1, S1 = g.chunk_fwd_qed(*(a[n] for n in ("q", "k", "v", "log_alpha", "b", "c", "w")), inp["S0"])
+    o2, S2 = g.chunk_fwd_qed(*(b[n] for n in ("q", "k", "v", "log_alpha", "b", "c", "w")), S1)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([o1, o2], 1), o)
+    assert torch.equal(S2, S)
 
 
 def test_chunk_qed_empty_sequence(g):
