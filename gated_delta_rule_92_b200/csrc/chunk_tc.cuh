@@ -512,24 +512,22 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
 //     K~ rows 32-63: k     v rows 32-63: v       w rows 0-31: w
 // and the prep and W.V expand them in place into the pseudo-rows.
 
-// log_alpha of one 32-token chunk for prep thread c (key channel c), 32 values
-// as bf16 pairs (tokens 2i, 2i + 1); tokens past the sequence end read as 0.
+// log_alpha of one 32-token chunk for prep thread c (key channel c): 32 bf16
+// values, one per register and untouched until the prep uses them (a whole
+// iteration later), so the loads' latency stays hidden; tokens past the
+// sequence end read as 0.
 template <int DK>
 struct PrepLAQ {
-    uint32_t v[16];
+    uint32_t v[32];
     __device__ __forceinline__ void load(const __nv_bfloat16 *la, long tok0, int n, int h, int len, int H, int c) {
         const unsigned short *p = reinterpret_cast<const unsigned short *>(la);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int r0 = n * 32 + 2 * i;
-            uint32_t lo = 0u, hi = 0u;
-            if (c < DK) {
-                if (r0 < len) lo = __ldg(p + ((tok0 + r0) * H + h) * DK + c);
-                if (r0 + 1 < len) hi = __ldg(p + ((tok0 + r0 + 1) * H + h) * DK + c);
-            }
-            v[i] = lo | (hi << 16);
+        for (int i = 0; i < 32; ++i) {
+            const int r = n * 32 + i;
+            v[i] = (c < DK && r < len) ? static_cast<uint32_t>(__ldg(p + ((tok0 + r) * H + h) * DK + c)) : 0u;
         }
     }
+    __device__ __forceinline__ float get(int i) const { return __uint_as_float(v[i] << 16); }
 };
 
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, unsigned short x) {
@@ -560,38 +558,58 @@ __device__ __forceinline__ void prep_chunk_qed(uint8_t *smem, uint32_t oqe, uint
         const int kb = (4 * p) >> 6, cb = ((4 * p) & 63) * 2;   // channel block, byte in the 128-byte row
         const uint8_t *qt = smem + oqe + kb * 16384, *kt = smem + okt + kb * 8192;
         auto off = [&](int r) { return r * 128 + ((((cb >> 4) ^ r) & 7) << 4) + (cb & 15); };
+        // four tokens at a time, their reductions interleaved (independent shuffle chains)
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
-            const int t = 8 * w + i;
-            float qv[4] = {0.f, 0.f, 0.f, 0.f}, kv[4] = {0.f, 0.f, 0.f, 0.f};
-            if (act) {
-                const uint2 q2 = *reinterpret_cast<const uint2 *>(qt + off(t));
-                const uint2 k2 = *reinterpret_cast<const uint2 *>(kt + off(32 + t));
-                qv[0] = bf16_lo(q2.x); qv[1] = bf16_hi(q2.x); qv[2] = bf16_lo(q2.y); qv[3] = bf16_hi(q2.y);
-                kv[0] = bf16_lo(k2.x); kv[1] = bf16_hi(k2.x); kv[2] = bf16_lo(k2.y); kv[3] = bf16_hi(k2.y);
-            }
-            float qk = 0.f, kk = 0.f;
+        for (int i0 = 0; i0 < 8; i0 += 4) {
+            uint2 q2[4], k2[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                qk = fmaf(qv[e], kv[e], qk);
-                kk = fmaf(kv[e], kv[e], kk);
+            for (int j = 0; j < 4; ++j) {
+                const int t = 8 * w + i0 + j;
+                q2[j] = act ? *reinterpret_cast<const uint2 *>(qt + off(t)) : make_uint2(0u, 0u);
+                k2[j] = act ? *reinterpret_cast<const uint2 *>(kt + off(32 + t)) : make_uint2(0u, 0u);
             }
+            float qk[4], kk[4];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                qk += __shfl_xor_sync(0xffffffffu, qk, o);
-                kk += __shfl_xor_sync(0xffffffffu, kk, o);
-            }
-            const float coef = kk > 0.f ? qk / kk : 0.f;
-            float rr = 0.f;
+            for (int j = 0; j < 4; ++j) {
+                const float qv[4] = {bf16_lo(q2[j].x), bf16_hi(q2[j].x), bf16_lo(q2[j].y), bf16_hi(q2[j].y)};
+                const float kv[4] = {bf16_lo(k2[j].x), bf16_hi(k2[j].x), bf16_lo(k2[j].y), bf16_hi(k2[j].y)};
+                qk[j] = 0.f;
+                kk[j] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float r = qv[e] - coef * kv[e];
-                rr = fmaf(r, r, rr);
+                for (int e = 0; e < 4; ++e) {
+                    qk[j] = fmaf(qv[e], kv[e], qk[j]);
+                    kk[j] = fmaf(kv[e], kv[e], kk[j]);
+                }
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
-            const float den = rr + qed_eps;
-            if (l == 0) scal[t] = make_float2(coef, den > 0.f ? rsqrtf(den) : 0.f);
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    qk[j] += __shfl_xor_sync(0xffffffffu, qk[j], o);
+                    kk[j] += __shfl_xor_sync(0xffffffffu, kk[j], o);
+                }
+            float coef[4], rr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                coef[j] = kk[j] > 0.f ? qk[j] / kk[j] : 0.f;
+                const float qv[4] = {bf16_lo(q2[j].x), bf16_hi(q2[j].x), bf16_lo(q2[j].y), bf16_hi(q2[j].y)};
+                const float kv[4] = {bf16_lo(k2[j].x), bf16_hi(k2[j].x), bf16_lo(k2[j].y), bf16_hi(k2[j].y)};
+                rr[j] = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float r = qv[e] - coef[j] * kv[e];
+                    rr[j] = fmaf(r, r, rr[j]);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) rr[j] += __shfl_xor_sync(0xffffffffu, rr[j], o);
+            if (l < 4) {   // lane j writes token 8 w + i0 + j (selects keep the arrays in registers)
+                const float cf = l == 0 ? coef[0] : l == 1 ? coef[1] : l == 2 ? coef[2] : coef[3];
+                const float den = (l == 0 ? rr[0] : l == 1 ? rr[1] : l == 2 ? rr[2] : rr[3]) + qed_eps;
+                scal[8 * w + i0 + l] = make_float2(cf, den > 0.f ? rsqrtf(den) : 0.f);
+            }
         }
     }
     named_bar(bar, 128);
@@ -600,28 +618,33 @@ __device__ __forceinline__ void prep_chunk_qed(uint8_t *smem, uint32_t oqe, uint
     if (c < DK) {
         float total = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) total += (bf16_lo(law.v[i]) + bf16_hi(law.v[i])) * kLog2e;
-        const float g0 = bf16_lo(law.v[0]) * kLog2e;
+        for (int i = 0; i < 32; ++i) total = fmaf(law.get(i), kLog2e, total);
+        const float g0 = law.get(0) * kLog2e;
         float sum = -0.5f * (g0 + total);   // the running sum enters at -ref
         const int kb = c >> 6, cc = c & 63;
         const uint32_t qt = smem_u32(smem + oqe + kb * 16384), et = qt + 8192u, kt = smem_u32(smem + okt + kb * 8192);
+        // the column part of the swizzled offset for each row phase (row & 7, a
+        // constant in the unrolled loop): element (row, cc) sits at row * 128 + cx[row & 7]
+        uint32_t cx[8];
+#pragma unroll
+        for (int r8 = 0; r8 < 8; ++r8) cx[r8] = ((((cc >> 3) ^ r8) & 7) << 4) + ((cc & 7) << 1);
+        auto at = [&](int row) { return static_cast<uint32_t>(row * 128) + cx[row & 7]; };
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
-            const uint32_t lp = law.v[t >> 1];
-            sum = fmaf((t & 1) ? bf16_hi(lp) : bf16_lo(lp), kLog2e, sum);
+            sum = fmaf(law.get(t), kLog2e, sum);
             const float ga = ex2(sum), iv = ex2(-sum);
-            const float q = ld_shared_bf16(qt + sw128_off(t, cc));
-            const float cg = ld_shared_bf16(qt + sw128_off(32 + t, cc));
-            const float k = ld_shared_bf16(kt + sw128_off(32 + t, cc));
-            const float b = ld_shared_bf16(et + sw128_off(32 + t, cc));
+            const float q = ld_shared_bf16(qt + at(t));
+            const float cg = ld_shared_bf16(qt + at(32 + t));
+            const float k = ld_shared_bf16(kt + at(32 + t));
+            const float b = ld_shared_bf16(et + at(32 + t));
             const float2 sc = scal[t];
             const float u = (q - sc.x * k) * sc.y;
-            st_shared_u16(qt + sw128_off(t, cc), bf16_bits(q * ga));
-            st_shared_u16(qt + sw128_off(32 + t, cc), 0);
-            st_shared_u16(et + sw128_off(2 * t, cc), bf16_bits(b * k * ga));
-            st_shared_u16(et + sw128_off(2 * t + 1, cc), bf16_bits(cg * u * ga));
-            st_shared_u16(kt + sw128_off(2 * t, cc), bf16_bits(k * iv));
-            st_shared_u16(kt + sw128_off(2 * t + 1, cc), bf16_bits(u * iv));
+            st_shared_u16(qt + at(t), bf16_bits(q * ga));
+            st_shared_u16(qt + at(32 + t), 0);
+            st_shared_u16(et + at(2 * t), bf16_bits(b * k * ga));
+            st_shared_u16(et + at(2 * t + 1), bf16_bits(cg * u * ga));
+            st_shared_u16(kt + at(2 * t), bf16_bits(k * iv));
+            st_shared_u16(kt + at(2 * t + 1), bf16_bits(u * iv));
         }
         // sum ends at G_31 - ref = -span / 2 (span: the decay of tokens 1..31)
         gc[c] = ex2(sum);
