@@ -506,7 +506,7 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
 // 64 pseudo-rows: row 2t is token t's key (erase b_t.k_t, value w_t.v_t), row
 // 2t + 1 its query direction u_t (erase c_t.u_t, value 0).  Both rows of a token
 // read the state before the token, so A is strictly lower by token, and only
-// the 32 token rows carry a query (P and O rows 0-31, rows 32-63 zero).  The
+// the 32 token rows carry a query (P and O rows 0-31; rows 32-63 unused).  The
 // tiles keep their 64-row shapes; the TMA brings the 32 token rows in as
 //     Q~ rows 0-31: q      Q~ rows 32-63: c      E rows 32-63: b
 //     K~ rows 32-63: k     v rows 32-63: v       w rows 0-31: w
@@ -544,7 +544,9 @@ __device__ __forceinline__ unsigned short bf16_bits(float x) {
 //  2. thread g = key channel c: the running log2-decay G_t over the 32 tokens,
 //     ref = (G_0 + G_31) / 2, and, in place, u_t = (q_t - coef_t k_t) nu_t and
 //     Q~_t = q.2^(G-ref), E_2t = b.k.2^(G-ref), E_2t+1 = c.u.2^(G-ref),
-//     K~_2t = k.2^(ref-G), K~_2t+1 = u.2^(ref-G), Q~ rows 32-63 cleared.
+//     K~_2t = k.2^(ref-G), K~_2t+1 = u.2^(ref-G).
+// Q~ rows 32-63 keep the raw c: the P read-out masks those rows to zero and the
+// rows of X they reach (32-63) are never stored, so they need no clearing.
 // Every read and write of channel c in step 2 is thread c's, in token order, so
 // the pseudo-row writes of token t only ever overwrite raw rows of tokens
 // <= t that the thread has already read.  gc and the stop flag as prep_chunk.
@@ -639,8 +641,7 @@ __device__ __forceinline__ void prep_chunk_qed(uint8_t *smem, uint32_t oqe, uint
             const float b = ld_shared_bf16(et + at(32 + t));
             const float2 sc = scal[t];
             const float u = (q - sc.x * k) * sc.y;
-            st_shared_u16(qt + at(t), bf16_bits(q * ga));
-            st_shared_u16(qt + at(32 + t), 0);
+            st_shared_u16(qt + at(t), bf16_bits(q * ga));   // rows 32-63 keep c (see below)
             st_shared_u16(et + at(2 * t), bf16_bits(b * k * ga));
             st_shared_u16(et + at(2 * t + 1), bf16_bits(cg * u * ga));
             st_shared_u16(kt + at(2 * t), bf16_bits(k * iv));
