@@ -334,10 +334,13 @@ gdn2_status_t gdn2_decode_step_ex(const void *q, const void *k, const void *v,
  *             to rounding)
  *   qed_eps : >= 0
  * Other arguments, layouts, shapes and errors as gdn2_chunk_fwd (value heads
- * equal key heads, no packing, no fusion) and gdn2_decode_step.  Both run on
- * CUDA cores with fp32 products; the chunk form takes 32 tokens per chunk
- * (64 rows of the chunked solve: each token adds its key and its query
- * direction), so its `chunk` is fixed.
+ * equal key heads, no packing, no fusion) and gdn2_decode_step.  The chunk
+ * form takes 32 tokens per chunk (64 rows of the chunked solve: each token
+ * adds its key and its query direction), so its `chunk` is fixed; with bf16
+ * I/O it runs on the tensor-core kernel (bf16 operands, fp32 accumulation and
+ * state), with fp32 I/O on CUDA cores with fp32 products.  The decode step
+ * runs on CUDA cores.  Any log_alpha in [-inf, 0] is exact, as for
+ * gdn2_chunk_fwd.
  */
 gdn2_status_t gdn2_chunk_fwd_qed(const void *q, const void *k, const void *v,
                                  const void *log_alpha, const void *b, const void *c, const void *w,
