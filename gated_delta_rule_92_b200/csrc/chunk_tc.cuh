@@ -450,24 +450,29 @@ __device__ __forceinline__ void prep_chunk(uint8_t *smem, uint32_t oqe, uint32_t
                     ok[h] = mul_bf16x2(kv[h], ivp);
                 }
             } else {
+                // fp32 products, two channels per paired instruction (same roundings)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const float ga0 = ex2(sum[2 * h]), ga1 = ex2(sum[2 * h + 1]);
-                    const float iv0 = ex2(-sum[2 * h]), iv1 = ex2(-sum[2 * h + 1]);
-                    float k0 = bf16_lo(kv[h]), k1 = bf16_hi(kv[h]);
-                    float b0 = bf16_lo(bv[h]), b1 = bf16_hi(bv[h]);
-                    float q0 = bf16_lo(qv[h]), q1 = bf16_hi(qv[h]);
+                    const float2 ga = make_float2(ex2(sum[2 * h]), ex2(sum[2 * h + 1]));
+                    const float2 iv = make_float2(ex2(-sum[2 * h]), ex2(-sum[2 * h + 1]));
+                    float2 k2 = make_float2(bf16_lo(kv[h]), bf16_hi(kv[h]));
+                    float2 b2 = make_float2(bf16_lo(bv[h]), bf16_hi(bv[h]));
+                    float2 q2 = make_float2(bf16_lo(qv[h]), bf16_hi(qv[h]));
                     if constexpr (PREP) {
-                        k0 *= rk;
-                        k1 *= rk;
-                        q0 *= rq;
-                        q1 *= rq;
-                        b0 = bs * sigmoid_tanh(b0);
-                        b1 = bs * sigmoid_tanh(b1);
+                        k2 = mul_f32x2(k2, make_float2(rk, rk));
+                        q2 = mul_f32x2(q2, make_float2(rq, rq));
+                        // sigmoid(x) = 0.5 + 0.5 tanh(x / 2), times bs
+                        const float2 hx = mul_f32x2(b2, make_float2(0.5f, 0.5f));
+                        float2 th;
+                        asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(hx.x));
+                        asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(hx.y));
+                        const float hb = 0.5f * bs;
+                        b2 = fma_f32x2(th, make_float2(hb, hb), make_float2(hb, hb));
                     }
-                    oq[h] = pack_bf16x2(q0 * ga0, q1 * ga1);
-                    oe[h] = pack_bf16x2(b0 * k0 * ga0, b1 * k1 * ga1);
-                    ok[h] = pack_bf16x2(k0 * iv0, k1 * iv1);
+                    const float2 xq = mul_f32x2(q2, ga), xe = mul_f32x2(mul_f32x2(b2, k2), ga), xk = mul_f32x2(k2, iv);
+                    oq[h] = pack_bf16x2(xq.x, xq.y);
+                    oe[h] = pack_bf16x2(xe.x, xe.y);
+                    ok[h] = pack_bf16x2(xk.x, xk.y);
                 }
             }
             *reinterpret_cast<uint2 *>(q_t + o[j]) = make_uint2(oq[0], oq[1]);
@@ -1376,9 +1381,15 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const uint32_t vv[4] = {a0, a1, a2, a3}, ww[4] = {b0, b1, b2, b3};
                         uint32_t rr[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            rr[e] = pack_bf16x2(sigmoid_tanh(bf16_lo(ww[e])) * bf16_lo(vv[e]),
-                                                sigmoid_tanh(bf16_hi(ww[e])) * bf16_hi(vv[e]));
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 hx = mul_f32x2(make_float2(bf16_lo(ww[e]), bf16_hi(ww[e])), make_float2(0.5f, 0.5f));
+                            float2 th;
+                            asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(hx.x));
+                            asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(hx.y));
+                            const float2 sg = fma_f32x2(th, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
+                            const float2 x = mul_f32x2(sg, make_float2(bf16_lo(vv[e]), bf16_hi(vv[e])));
+                            rr[e] = pack_bf16x2(x.x, x.y);
+                        }
                         r4 = make_uint4(rr[0], rr[1], rr[2], rr[3]);
                     } else {
                         r4 = mul_bf16x8(make_uint4(a0, a1, a2, a3), make_uint4(b0, b1, b2, b3));

@@ -308,6 +308,16 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
     return *reinterpret_cast<float2 *>(&r);
 }
 
+// a * b + c on two fp32 lanes in one paired instruction (each a single fma).
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
