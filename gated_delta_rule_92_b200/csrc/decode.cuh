@@ -103,6 +103,18 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         s[i] = __ldcs(reinterpret_cast<const float4 *>(Sh + (long)row * d_v));
     }
 
+    // fused epilogue: its gate and weight values are read now, under the state loads
+    float gate4[4] = {0.f, 0.f, 0.f, 0.f};
+    float4 wt4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (FUSED) {
+        if (fz.gate != nullptr && rg == 0) {
+            const IO *gp = static_cast<const IO *>(fz.gate) + bh * (long)d_v + j0 + cg * 4;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) gate4[e] = ld_io(gp + e);
+            wt4 = __ldg(reinterpret_cast<const float4 *>(fz.norm_weight + j0 + cg * 4));
+        }
+    }
+
     // per-row and per-column coefficients
     const IO *qh = q + bk * DK, *kh = k + bk * DK, *lah = la + bk * DK, *bh_ = bg + bk * DK;
     float qk = 0.f;
@@ -186,6 +198,19 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         for (int wi = 0; wi < (DK + 31) / 32; ++wi) qkt += s_qk[wi];
         ov = make_float4(pt.x + qkt * u.x, pt.y + qkt * u.y, pt.z + qkt * u.z, pt.w + qkt * u.w);
     }
+    // the state update goes out before the epilogue's synchronisation
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int row = i * RG + rg;
+        const float a = s_alpha[row], kv = s_k[row];
+        float4 n;
+        n.x = a * s[i].x + kv * u.x;
+        n.y = a * s[i].y + kv * u.y;
+        n.z = a * s[i].z + kv * u.z;
+        n.w = a * s[i].w + kv * u.w;
+        __stcs(reinterpret_cast<float4 *>(Sh + (long)row * d_v), n);
+    }
+
     bool plain_store = true;
     if constexpr (FUSED) {
         if (fz.gate != nullptr) {   // gated RMS norm over the whole d_v row
@@ -211,9 +236,8 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
                 for (int r = 0; r < nblk; ++r) tot += s_ss[r];
                 const float inv = rsqrtf(tot / (float)d_v + fz.norm_eps);
                 const long go = bh * (long)d_v + j0 + cg * 4;
-                const IO *gp = static_cast<const IO *>(fz.gate) + go;
-                const float4 wt = __ldg(reinterpret_cast<const float4 *>(fz.norm_weight + j0 + cg * 4));
-                const float g0 = ld_io(gp), g1 = ld_io(gp + 1), g2 = ld_io(gp + 2), g3 = ld_io(gp + 3);
+                const float4 wt = wt4;
+                const float g0 = gate4[0], g1 = gate4[1], g2 = gate4[2], g3 = gate4[3];
                 st_io4<IO>(o + go, ov.x * inv * wt.x * g0 * sigmoid_io<IO>(g0),
                            ov.y * inv * wt.y * g1 * sigmoid_io<IO>(g1), ov.z * inv * wt.z * g2 * sigmoid_io<IO>(g2),
                            ov.w * inv * wt.w * g3 * sigmoid_io<IO>(g3));
@@ -221,18 +245,6 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         }
     }
     if (plain_store && rg == 0) st_io4<IO>(o + bh * (long)d_v + j0 + cg * 4, ov.x, ov.y, ov.z, ov.w);
-
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int row = i * RG + rg;
-        const float a = s_alpha[row], kv = s_k[row];
-        float4 n;
-        n.x = a * s[i].x + kv * u.x;
-        n.y = a * s[i].y + kv * u.y;
-        n.z = a * s[i].z + kv * u.z;
-        n.w = a * s[i].w + kv * u.w;
-        __stcs(reinterpret_cast<float4 *>(Sh + (long)row * d_v), n);
-    }
 }
 
 }  // namespace gdn2
