@@ -20,6 +20,7 @@ log_alpha, b carry the H key heads, v, w, o, gate the HV value heads
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -27,21 +28,30 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn2.so")
+# the same sources with device-side range checks (-DGDN2_DEBUG_BOUNDS); used in
+# place of LIB_PATH when GDN2_DEBUG_BOUNDS=1 is set, or inside debug_bounds()
+DEBUG_LIB_PATH = os.path.join(_HERE, "libgdn2_debug.so")
 
 IO_F32 = 0
 IO_BF16 = 1
 STATUS_NAMES = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED",
-                3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT"}
+                3: "GDN2_ERR_MISALIGNED", 4: "GDN2_ERR_CUDA", 5: "GDN2_ERR_DEVICE_TIMEOUT",
+                6: "GDN2_ERR_OUT_OF_BOUNDS"}
+OUT_OF_BOUNDS = 6
+# argument buffers as gdn2_debug_bounds_site numbers them
+BOUNDS_BUFFERS = ("q", "k", "v", "log_alpha", "b", "w", "c", "S0", "S_T", "o", "gate", "norm_weight",
+                  "cu_seqlens")
 EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_chunk_fwd_host",
             "gdn2_chunk_fwd_host_workspace", "gdn2_chunk_fwd_host_noalloc", "gdn2_decode_step",
             "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex", "gdn2_chunk_fwd_qed", "gdn2_decode_step_qed",
-            "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_status_string",
-            "gdn2_version")
+            "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_debug_bounds_site",
+            "gdn2_selftest_bounds", "gdn2_status_string", "gdn2_version")
 FUSE_INPUT_PREP = 1    # q, k, b, w are raw: L2-normalise q, k over d_k; b, w = sigmoid
 FUSE_NEG_EIGVAL = 2    # with FUSE_INPUT_PREP: b = 2 sigmoid(b)
 NOALLOC_WORKSPACE_BYTES = 64 << 20   # GDN2_NOALLOC_WORKSPACE_BYTES: the no-alloc entry's fixed workspace
 
 _lib = None
+_opened = {}
 
 
 class Gdn2Error(RuntimeError):
@@ -51,13 +61,36 @@ class Gdn2Error(RuntimeError):
 
 
 def lib() -> ctypes.CDLL:
-    """Open libgdn2.so and declare the C signatures (raises if missing)."""
+    """The library the calls go through: libgdn2.so, or its debug build when
+    GDN2_DEBUG_BOUNDS=1 is set (raises if the file is missing)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with "
+        _lib = _open(DEBUG_LIB_PATH if os.environ.get("GDN2_DEBUG_BOUNDS") == "1" else LIB_PATH)
+    return _lib
+
+
+@contextlib.contextmanager
+def debug_bounds():
+    """Route the calls made inside the block through the debug build
+    (libgdn2_debug.so: every per-thread global access range-checked against its
+    argument buffer; a failed check records GDN2_ERR_OUT_OF_BOUNDS instead of
+    touching memory).  Yields the debug library."""
+    global _lib
+    prev = _lib
+    _lib = _open(DEBUG_LIB_PATH)
+    try:
+        yield _lib
+    finally:
+        _lib = prev
+
+
+def _open(path: str) -> ctypes.CDLL:
+    """Open one build of the library (once) and declare the C signatures."""
+    if path not in _opened:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with "
                               "`python -m gated_delta_rule_92_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+        L = ctypes.CDLL(path)
         P, I = ctypes.c_void_p, ctypes.c_int
         chunk_args = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
         for name in ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core"):
@@ -92,10 +125,14 @@ def lib() -> ctypes.CDLL:
         L.gdn2_selftest_wait_timeout.restype = I
         L.gdn2_status_string.argtypes = [I]
         L.gdn2_status_string.restype = ctypes.c_char_p
+        L.gdn2_debug_bounds_site.argtypes = [ctypes.POINTER(I), ctypes.POINTER(I), P]
+        L.gdn2_debug_bounds_site.restype = I
+        L.gdn2_selftest_bounds.argtypes = [P]
+        L.gdn2_selftest_bounds.restype = I
         L.gdn2_version.argtypes = []
         L.gdn2_version.restype = I
-        _lib = L
-    return _lib
+        _opened[path] = L
+    return _opened[path]
 
 
 def status_string(code: int) -> str:
@@ -439,3 +476,19 @@ def device_status(stream=None) -> int:
 
 def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
     return int(lib().gdn2_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def debug_bounds_site(stream=None):
+    """Debug build: (buffer name, source line) of the first failed range check
+    since the last read, or None; clears it.  Raises Gdn2Error in the release
+    build (GDN2_ERR_UNSUPPORTED)."""
+    buf, line = ctypes.c_int(-1), ctypes.c_int(0)
+    st = lib().gdn2_debug_bounds_site(ctypes.byref(buf), ctypes.byref(line), _stream(stream))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_debug_bounds_site")
+    return None if buf.value < 0 else (BOUNDS_BUFFERS[buf.value], line.value)
+
+
+def selftest_bounds(stream=None) -> int:
+    """Debug build: GDN2_ERR_OUT_OF_BOUNDS when the range check works."""
+    return int(lib().gdn2_selftest_bounds(_stream(stream)))

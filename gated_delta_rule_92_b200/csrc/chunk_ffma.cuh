@@ -87,8 +87,8 @@ __device__ __forceinline__ void chunk_token_steps(const float *sQ, const float *
             for (int x = 0; x < P; ++x) nv = fmaf(sKap[(P * t + x) * LK + c], u[x], nv);
             Sr[i] = nv;
         }
-        if (part == 0) {
-            IO *dst = o + o_row0 + (long)t * o_stride + j;
+        IO *dst = o + o_row0 + (long)t * o_stride + j;
+        if (part == 0 && GDN2_IN_BOUNDS(kBufO, dst, sizeof(IO))) {
             if constexpr (sizeof(IO) == 4) *dst = ov;
             else *dst = __float2bfloat16_rn(ov);
         }
@@ -148,7 +148,8 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     long tok_base = (long)bb * T;
     int len = T;
     if (cu_seqlens != nullptr) {
-        const int a = cu_seqlens[bb], e = cu_seqlens[bb + 1];
+        const int a = GDN2_IN_BOUNDS(kBufCU, cu_seqlens + bb, sizeof(int)) ? cu_seqlens[bb] : -1;
+        const int e = GDN2_IN_BOUNDS(kBufCU, cu_seqlens + bb + 1, sizeof(int)) ? cu_seqlens[bb + 1] : -1;
         if (a < 0 || e < a || e > T) {   // malformed packing: this sequence is skipped
             if (threadIdx.x == 0) record_status(kStatusBadArgs);
             return;
@@ -162,7 +163,8 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     // initial state slice
     for (int idx = tid; idx < DK * NV; idx += 256) {
         const int c = idx / NV, j = idx % NV;
-        sS[c * LV + j] = S0 ? S0[(head * DK + c) * d_v + j0 + j] : 0.f;
+        const float *sp = S0 ? S0 + (head * DK + c) * d_v + j0 + j : nullptr;
+        sS[c * LV + j] = (sp && GDN2_IN_BOUNDS(kBufS0, sp, 4)) ? *sp : 0.f;
     }
 
     for (int n = 0; n < NC; ++n) {
@@ -175,16 +177,19 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
             const int r = idx / DK, c = idx % DK;
             const long g = ((tok0 + r) * H + h) * DK + c;
             const bool in = r < rows;
-            sQ[r * LK + c] = in ? ld_io(q + g) : 0.f;
-            sK[r * LK + c] = in ? ld_io(k + g) : 0.f;
-            sE[r * LK + c] = in ? (prep ? bscale * sigmoid_f32(ld_io(bg + g)) : ld_io(bg + g)) : 0.f;
-            sG[r * LK + c] = in ? ld_io(la + g) : 0.f;
+            sQ[r * LK + c] = (in && GDN2_IN_BOUNDS(kBufQ, q + g, sizeof(IO))) ? ld_io(q + g) : 0.f;
+            sK[r * LK + c] = (in && GDN2_IN_BOUNDS(kBufK, k + g, sizeof(IO))) ? ld_io(k + g) : 0.f;
+            const float bx = (in && GDN2_IN_BOUNDS(kBufB, bg + g, sizeof(IO))) ? ld_io(bg + g) : 0.f;
+            sE[r * LK + c] = in ? (prep ? bscale * sigmoid_f32(bx) : bx) : 0.f;
+            sG[r * LK + c] = (in && GDN2_IN_BOUNDS(kBufLA, la + g, sizeof(IO))) ? ld_io(la + g) : 0.f;
         }
         for (int idx = tid; idx < C * NV; idx += 256) {
             const int r = idx / NV, j = idx % NV;
             const long g = ((tok0 + r) * HV + hv) * d_v + j0 + j;
-            const float wv = (r < rows) ? ld_io(wg + g) : 0.f;
-            sWV[r * LV + j] = (r < rows) ? (prep ? sigmoid_f32(wv) : wv) * ld_io(v + g) : 0.f;
+            const bool in = r < rows;
+            const float wv = (in && GDN2_IN_BOUNDS(kBufW, wg + g, sizeof(IO))) ? ld_io(wg + g) : 0.f;
+            const float vv = (in && GDN2_IN_BOUNDS(kBufV, v + g, sizeof(IO))) ? ld_io(v + g) : 0.f;
+            sWV[r * LV + j] = in ? (prep ? sigmoid_f32(wv) : wv) * vv : 0.f;
         }
         __syncthreads();
         if (prep) {   // L2-normalise each row of q and k: warp w takes rows w, w + 8, ...
@@ -390,6 +395,7 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
                     const long g = ((tok0 + r) * HV + hv) * d_v + j0 + 4 * ct;
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
+                        if (!GDN2_IN_BOUNDS(kBufO, o + g + y, sizeof(IO))) continue;
                         if constexpr (sizeof(IO) == 4) o[g + y] = ov[x][y];
                         else o[g + y] = __float2bfloat16_rn(ov[x][y]);
                     }
@@ -428,7 +434,8 @@ chunk_fwd_ffma_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const 
     if (S_T) {
         for (int idx = tid; idx < DK * NV; idx += 256) {
             const int c = idx / NV, j = idx % NV;
-            S_T[(head * DK + c) * d_v + j0 + j] = sS[c * LV + j];
+            float *sp = S_T + (head * DK + c) * d_v + j0 + j;
+            if (GDN2_IN_BOUNDS(kBufST, sp, 4)) *sp = sS[c * LV + j];
         }
     }
 }

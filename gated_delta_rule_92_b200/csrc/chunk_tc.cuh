@@ -288,8 +288,8 @@ struct PrepLA {
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int r = n * 64 + hb * R + i;
-            v[i] = r < len ? __ldg(reinterpret_cast<const uint2 *>(la + ((tok0 + r) * H + h) * DK + 4 * p))
-                           : make_uint2(0u, 0u);
+            const uint2 *src = reinterpret_cast<const uint2 *>(la + ((tok0 + r) * H + h) * DK + 4 * p);
+            v[i] = (r < len && GDN2_IN_BOUNDS(kBufLA, src, 8)) ? __ldg(src) : make_uint2(0u, 0u);
         }
     }
 };
@@ -529,7 +529,8 @@ struct PrepLAQ {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int r = n * 32 + i;
-            v[i] = (c < DK && r < len) ? static_cast<uint32_t>(__ldg(p + ((tok0 + r) * H + h) * DK + c)) : 0u;
+            const unsigned short *src = p + ((tok0 + r) * H + h) * DK + c;
+            v[i] = (c < DK && r < len && GDN2_IN_BOUNDS(kBufLA, src, 2)) ? static_cast<uint32_t>(__ldg(src)) : 0u;
         }
     }
     __device__ __forceinline__ float get(int i) const { return __uint_as_float(v[i] << 16); }
@@ -672,7 +673,8 @@ __device__ __forceinline__ int longest_first_sequence(const int *__restrict__ cu
     if (nseq <= 1 || nseq > kMaxRankedSeqs) return slot;
     int *lens = scratch, *pick = scratch + kMaxRankedSeqs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    for (int i = tid; i < nseq; i += blockDim.x) lens[i] = cu[i + 1] - cu[i];
+    for (int i = tid; i < nseq; i += blockDim.x)
+        lens[i] = (GDN2_IN_BOUNDS(kBufCU, cu + i, 8)) ? cu[i + 1] - cu[i] : 0;
     if (tid == 0) *pick = slot;   // a total order always has one sequence of rank `slot`
     __syncthreads();
     for (int i = warp; i < nseq; i += nwarps) {
@@ -696,7 +698,12 @@ template <int N>
 struct BfVec {
     static_assert(N == 2 || N == 4, "bf16 vector");
     uint32_t w[N / 2];
-    __device__ __forceinline__ void load(const __nv_bfloat16 *p) {
+    __device__ __forceinline__ void load(const __nv_bfloat16 *p, int buf) {
+        if (!GDN2_IN_BOUNDS(buf, p, 2 * N)) {
+#pragma unroll
+            for (int e = 0; e < N / 2; ++e) w[e] = 0u;
+            return;
+        }
         if constexpr (N == 4) {
             const uint2 x = __ldg(reinterpret_cast<const uint2 *>(p));
             w[0] = x.x;
@@ -800,9 +807,11 @@ __device__ __noinline__ void tc_token_tail(uint8_t *smem, const TailArgs ta, con
                         for (int x = 0; x < CJ; ++x) obuf[tt * NV + jb + x] = ov[x];
                     } else {
                         __nv_bfloat16 *dst = o + ((tok0 + tb + tt) * HV + hv) * (long)d_v + j0 + jb;
+                        if (GDN2_IN_BOUNDS(kBufO, dst, 2 * CJ)) {
 #pragma unroll
-                        for (int x = 0; x < CJ; x += 2)
-                            *reinterpret_cast<uint32_t *>(dst + x) = pack_bf16x2(ov[x], ov[x + 1]);
+                            for (int x = 0; x < CJ; x += 2)
+                                *reinterpret_cast<uint32_t *>(dst + x) = pack_bf16x2(ov[x], ov[x + 1]);
+                        }
                     }
                 }
             }
@@ -823,6 +832,8 @@ __device__ __noinline__ void tc_token_tail(uint8_t *smem, const TailArgs ta, con
                     for (int e = 0; e < JPL; ++e) {
                         const int jj = lane + 32 * e;
                         const float gt = cold[(buf * TB + tt) * NV + jj].y;
+                        if (!GDN2_IN_BOUNDS(kBufO, o + vro + jj, 2) || !GDN2_IN_BOUNDS(kBufNW, fz.norm_weight + j0 + jj, 4))
+                            continue;
                         o[vro + jj] = __float2bfloat16_rn(obuf[tt * NV + jj] * inv * fz.norm_weight[j0 + jj] * gt *
                                                           sigmoid_f32(gt));
                     }
@@ -835,6 +846,7 @@ __device__ __noinline__ void tc_token_tail(uint8_t *smem, const TailArgs ta, con
 #pragma unroll
             for (int i = 0; i < RR; ++i) {
                 float *dst = S_T + (head * DK + 8 * i + rb) * d_v + j0 + jb;
+                if (!GDN2_IN_BOUNDS(kBufST, dst, 4 * CJ)) continue;
 #pragma unroll
                 for (int x = 0; x < CJ; ++x) dst[x] = Sr[i][x];
             }
@@ -858,13 +870,13 @@ __device__ __noinline__ void tc_token_tail(uint8_t *smem, const TailArgs ta, con
                     const long tok = tok0 + tb + tt;
                     const long kro = (tok * H + h) * DK + CPL * lane;
                     const long vro = (tok * HV + hv) * (long)d_v + j0 + JPL * lane;
-                    rq[m].load(ta.q + kro);
-                    rk[m].load(ta.k + kro);
-                    rbv[m].load(ta.b + kro);
-                    rl[m].load(la + kro);
-                    rv[m].load(ta.v + vro);
-                    rw[m].load(ta.w + vro);
-                    if constexpr (EPI) rg[m].load(static_cast<const __nv_bfloat16 *>(fz.gate) + vro);
+                    rq[m].load(ta.q + kro, kBufQ);
+                    rk[m].load(ta.k + kro, kBufK);
+                    rbv[m].load(ta.b + kro, kBufB);
+                    rl[m].load(la + kro, kBufLA);
+                    rv[m].load(ta.v + vro, kBufV);
+                    rw[m].load(ta.w + vro, kBufW);
+                    if constexpr (EPI) rg[m].load(static_cast<const __nv_bfloat16 *>(fz.gate) + vro, kBufGate);
                 }
             }
 #pragma unroll
@@ -996,9 +1008,11 @@ __device__ __noinline__ void tc_token_tail_qed(uint8_t *smem, const TailArgs ta,
                 }
                 if (rb == 0) {
                     __nv_bfloat16 *dst = o + ((tok0 + tb + tt) * H + h) * (long)d_v + j0 + jb;
+                    if (GDN2_IN_BOUNDS(kBufO, dst, 2 * CJ)) {
 #pragma unroll
-                    for (int x = 0; x < CJ; x += 2)
-                        *reinterpret_cast<uint32_t *>(dst + x) = pack_bf16x2(ov[x], ov[x + 1]);
+                        for (int x = 0; x < CJ; x += 2)
+                            *reinterpret_cast<uint32_t *>(dst + x) = pack_bf16x2(ov[x], ov[x + 1]);
+                    }
                 }
             }
             if (k + 2 < nb) named_bar_arrive(BAR_EMPTY + buf, kAll);
@@ -1007,6 +1021,7 @@ __device__ __noinline__ void tc_token_tail_qed(uint8_t *smem, const TailArgs ta,
 #pragma unroll
             for (int i = 0; i < RR; ++i) {
                 float *dst = S_T + (head * DK + 8 * i + rb) * d_v + j0 + jb;
+                if (!GDN2_IN_BOUNDS(kBufST, dst, 4 * CJ)) continue;
 #pragma unroll
                 for (int x = 0; x < CJ; ++x) dst[x] = Sr[i][x];
             }
@@ -1026,13 +1041,13 @@ __device__ __noinline__ void tc_token_tail_qed(uint8_t *smem, const TailArgs ta,
                     const long tok = tok0 + tb + tt;
                     const long kro = (tok * H + h) * DK + CPL * lane;
                     const long vro = (tok * H + h) * (long)d_v + j0 + JPL * lane;
-                    rq[m].load(ta.q + kro);
-                    rk[m].load(ta.k + kro);
-                    rbv[m].load(ta.b + kro);
-                    rc[m].load(ta.c + kro);
-                    rl[m].load(la + kro);
-                    rv[m].load(ta.v + vro);
-                    rw[m].load(ta.w + vro);
+                    rq[m].load(ta.q + kro, kBufQ);
+                    rk[m].load(ta.k + kro, kBufK);
+                    rbv[m].load(ta.b + kro, kBufB);
+                    rc[m].load(ta.c + kro, kBufC);
+                    rl[m].load(la + kro, kBufLA);
+                    rv[m].load(ta.v + vro, kBufV);
+                    rw[m].load(ta.w + vro, kBufW);
                 }
             }
 #pragma unroll
@@ -1126,7 +1141,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     long tok0 = (long)bb * T;
     int len = T, tma_t0 = 0, tma_b = bb;
     if constexpr (VARLEN) {
-        const int a = cu_seqlens[bb], e = cu_seqlens[bb + 1];
+        const bool cu_ok = GDN2_IN_BOUNDS(kBufCU, cu_seqlens + bb, 8);
+        const int a = cu_ok ? cu_seqlens[bb] : -1, e = cu_ok ? cu_seqlens[bb + 1] : -1;
         if (a < 0 || e < a || e > T) {   // malformed packing: this sequence is skipped
             if (threadIdx.x == 0) record_status(kStatusBadArgs);
             return;
@@ -1175,7 +1191,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     if constexpr (EPI) {
         float *nw = reinterpret_cast<float *>(smem + Cfg::OFF_NW);
-        for (int i = tid; i < NV; i += kTcThreads) nw[i] = fz.norm_weight[j0 + i];
+        for (int i = tid; i < NV; i += kTcThreads)
+            nw[i] = GDN2_IN_BOUNDS(kBufNW, fz.norm_weight + j0 + i, 4) ? fz.norm_weight[j0 + i] : 0.f;
     }
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
@@ -1508,7 +1525,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 float sv[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) sv[e] = 0.f;
-                if (S0 != nullptr && c < DK) {
+                if (S0 != nullptr && c < DK &&
+                    GDN2_IN_BOUNDS(kBufS0, S0 + (head * DK + c) * d_v + j0 + jc * 32, 128)) {
                     const float4 *src = reinterpret_cast<const float4 *>(S0 + (head * DK + c) * d_v + j0 + jc * 32);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
@@ -1517,7 +1535,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
                 tmem_st32(t_S + lane_q + jc * 32, sv);
-                if (NC == 0 && S_T != nullptr && c < DK) {   // empty sequence: S_T = S0
+                if (NC == 0 && S_T != nullptr && c < DK &&   // empty sequence: S_T = S0
+                    GDN2_IN_BOUNDS(kBufST, S_T + (head * DK + c) * d_v + j0 + jc * 32, 128)) {
                     float4 *dst = reinterpret_cast<float4 *>(S_T + (head * DK + c) * d_v + j0 + jc * 32);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
@@ -1706,7 +1725,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int jc = 0; jc < NV / 32; ++jc) {
                     float sv[32];
                     tmem_ld32(t_S + lane_q + jc * 32, sv);
-                    if (last && S_T != nullptr && c < DK) {
+                    if (last && S_T != nullptr && c < DK &&
+                        GDN2_IN_BOUNDS(kBufST, S_T + (head * DK + c) * d_v + j0 + jc * 32, 128)) {
                         float4 *dst = reinterpret_cast<float4 *>(S_T + (head * DK + c) * d_v + j0 + jc * 32);
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
@@ -1797,7 +1817,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int jc = 0; jc < NV / 32 && plain; ++jc) {
                     float x[32];
                     tmem_ld32(t_X + lane_q + jc * 32, x);
-                    if (valid) {
+                    if (valid && GDN2_IN_BOUNDS(kBufO, orow + jc * 32, 64)) {
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + jc * 32);
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
@@ -1822,10 +1842,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int i = 0; i < 64 / RPP; ++i) {
                     const int r = i * RPP + rr;
-                    gall[i] = (n * 64 + r < len)
-                                  ? __ldg(reinterpret_cast<const uint4 *>(
-                                        gbase + ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * c16))
-                                  : make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 *gp = reinterpret_cast<const uint4 *>(
+                        gbase + ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * c16);
+                    gall[i] = (n * 64 + r < len && GDN2_IN_BOUNDS(kBufGate, gp, 16)) ? __ldg(gp)
+                                                                                     : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
                 for (int i = 0; i < 64 / RPP; ++i) {
@@ -1843,7 +1863,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         pk[e] = pack_bf16x2(bf16_lo(ov[e]) * wt[2 * e] * g0 * sigmoid_tanh(g0),
                                             bf16_hi(ov[e]) * wt[2 * e + 1] * g1 * sigmoid_tanh(g1));
                     }
-                    *reinterpret_cast<uint4 *>(o + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    if (GDN2_IN_BOUNDS(kBufO, o + off, 16))
+                        *reinterpret_cast<uint4 *>(o + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
             tmem_st_wait();

@@ -100,7 +100,8 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int row = i * RG + rg;
-        s[i] = __ldcs(reinterpret_cast<const float4 *>(Sh + (long)row * d_v));
+        const float4 *sp = reinterpret_cast<const float4 *>(Sh + (long)row * d_v);
+        s[i] = GDN2_IN_BOUNDS(kBufS0, sp, 16) ? __ldcs(sp) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
     // fused epilogue: its gate and weight values are read now, under the state loads
@@ -110,8 +111,9 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         if (fz.gate != nullptr && rg == 0) {
             const IO *gp = static_cast<const IO *>(fz.gate) + bh * (long)d_v + j0 + cg * 4;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) gate4[e] = ld_io(gp + e);
-            wt4 = __ldg(reinterpret_cast<const float4 *>(fz.norm_weight + j0 + cg * 4));
+            for (int e = 0; e < 4; ++e) gate4[e] = GDN2_IN_BOUNDS(kBufGate, gp + e, sizeof(IO)) ? ld_io(gp + e) : 0.f;
+            const float4 *wp = reinterpret_cast<const float4 *>(fz.norm_weight + j0 + cg * 4);
+            if (GDN2_IN_BOUNDS(kBufNW, wp, 16)) wt4 = __ldg(wp);
         }
     }
 
@@ -120,9 +122,9 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     float qk = 0.f;
     float kv = 0.f, qv = 0.f, bv = 0.f;
     if (tid < DK) {
-        kv = ld_io(kh + tid);
-        qv = ld_io(qh + tid);
-        bv = ld_io(bh_ + tid);
+        kv = GDN2_IN_BOUNDS(kBufK, kh + tid, sizeof(IO)) ? ld_io(kh + tid) : 0.f;
+        qv = GDN2_IN_BOUNDS(kBufQ, qh + tid, sizeof(IO)) ? ld_io(qh + tid) : 0.f;
+        bv = GDN2_IN_BOUNDS(kBufB, bh_ + tid, sizeof(IO)) ? ld_io(bh_ + tid) : 0.f;
     }
     if constexpr (FUSED) {
         if (fz.prep) {   // q / |q|, k / |k| over d_k (block reduction), sigmoid gates
@@ -144,7 +146,7 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         }
     }
     if (tid < DK) {
-        const float a = __expf(ld_io(lah + tid));
+        const float a = __expf(GDN2_IN_BOUNDS(kBufLA, lah + tid, sizeof(IO)) ? ld_io(lah + tid) : 0.f);
         s_alpha[tid] = a;
         s_erase[tid] = bv * kv * a;
         s_qa[tid] = qv * a;
@@ -153,11 +155,11 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
     }
     if (tid < NVD) {
         const long vo = bh * (long)d_v + j0 + tid;
-        float wv = ld_io(wg + vo);
+        float wv = GDN2_IN_BOUNDS(kBufW, wg + vo, sizeof(IO)) ? ld_io(wg + vo) : 0.f;
         if constexpr (FUSED) {
             if (fz.prep) wv = sigmoid_io<IO>(wv);
         }
-        s_wv[tid] = wv * ld_io(v + vo);
+        s_wv[tid] = wv * (GDN2_IN_BOUNDS(kBufV, v + vo, sizeof(IO)) ? ld_io(v + vo) : 0.f);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, off);
@@ -208,7 +210,8 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
         n.y = a * s[i].y + kv * u.y;
         n.z = a * s[i].z + kv * u.z;
         n.w = a * s[i].w + kv * u.w;
-        __stcs(reinterpret_cast<float4 *>(Sh + (long)row * d_v), n);
+        float4 *sp = reinterpret_cast<float4 *>(Sh + (long)row * d_v);
+        if (GDN2_IN_BOUNDS(kBufST, sp, 16)) __stcs(sp, n);
     }
 
     bool plain_store = true;
@@ -238,13 +241,16 @@ decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO 
                 const long go = bh * (long)d_v + j0 + cg * 4;
                 const float4 wt = wt4;
                 const float g0 = gate4[0], g1 = gate4[1], g2 = gate4[2], g3 = gate4[3];
-                st_io4<IO>(o + go, ov.x * inv * wt.x * g0 * sigmoid_io<IO>(g0),
-                           ov.y * inv * wt.y * g1 * sigmoid_io<IO>(g1), ov.z * inv * wt.z * g2 * sigmoid_io<IO>(g2),
-                           ov.w * inv * wt.w * g3 * sigmoid_io<IO>(g3));
+                if (GDN2_IN_BOUNDS(kBufO, o + go, 4 * sizeof(IO)))
+                    st_io4<IO>(o + go, ov.x * inv * wt.x * g0 * sigmoid_io<IO>(g0),
+                               ov.y * inv * wt.y * g1 * sigmoid_io<IO>(g1),
+                               ov.z * inv * wt.z * g2 * sigmoid_io<IO>(g2),
+                               ov.w * inv * wt.w * g3 * sigmoid_io<IO>(g3));
             }
         }
     }
-    if (plain_store && rg == 0) st_io4<IO>(o + bh * (long)d_v + j0 + cg * 4, ov.x, ov.y, ov.z, ov.w);
+    if (plain_store && rg == 0 && GDN2_IN_BOUNDS(kBufO, o + bh * (long)d_v + j0 + cg * 4, 4 * sizeof(IO)))
+        st_io4<IO>(o + bh * (long)d_v + j0 + cg * 4, ov.x, ov.y, ov.z, ov.w);
 }
 
 }  // namespace gdn2

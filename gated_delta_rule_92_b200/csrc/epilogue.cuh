@@ -23,13 +23,16 @@ gated_rmsnorm_kernel(IO *__restrict__ o, const IO *__restrict__ g, const float *
     const IO *grow = g + row * d_v;
     float ss = 0.f;
     for (int j = l; j < d_v; j += 32) {
-        const float x = ld_io(orow + j);
+        const float x = GDN2_IN_BOUNDS(kBufO, orow + j, sizeof(IO)) ? ld_io(orow + j) : 0.f;
         ss = fmaf(x, x, ss);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     const float inv = rsqrtf(ss / (float)d_v + eps);
     for (int j = l; j < d_v; j += 32) {
+        if (!GDN2_IN_BOUNDS(kBufO, orow + j, sizeof(IO)) || !GDN2_IN_BOUNDS(kBufGate, grow + j, sizeof(IO)) ||
+            !GDN2_IN_BOUNDS(kBufNW, weight + j, sizeof(float)))
+            continue;
         const float x = ld_io(orow + j), gv = ld_io(grow + j);
         const float y = x * inv * __ldg(weight + j) * gv * sigmoid_io<IO>(gv);
         if constexpr (sizeof(IO) == 4) orow[j] = y;

@@ -21,6 +21,12 @@ __device__ int g_device_status = 0;
 constexpr int kStatusTimeout = 5;   // == GDN2_ERR_DEVICE_TIMEOUT
 constexpr int kStatusBadArgs = 1;   // == GDN2_ERR_INVALID_ARG (e.g. malformed cu_seqlens)
 
+}  // namespace gdn2
+
+#include "bounds.cuh"
+
+namespace gdn2 {
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

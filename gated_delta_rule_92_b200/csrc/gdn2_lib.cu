@@ -35,11 +35,85 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
     }
 }
 
+#ifdef GDN2_DEBUG_BOUNDS
+// Debug build: publishes one call's buffer extents, in stream order (a kernel
+// parameter, so the write can also be captured into a CUDA graph).
+__global__ void set_bounds_kernel(BoundsTable t) { g_bounds = t; }
+
+// Exercises the range check on addresses only (nothing is dereferenced): an
+// 8-byte range inside a 64-byte extent passes, one that runs past its end
+// fails and records GDN2_ERR_OUT_OF_BOUNDS with this buffer and line.  A check
+// that answers wrongly leaves GDN2_ERR_INVALID_ARG instead.
+__global__ void selftest_bounds_kernel(unsigned long long fake_base) {
+    g_bounds.lo[kBufQ] = fake_base;
+    g_bounds.hi[kBufQ] = fake_base + 64;
+    const char *base = reinterpret_cast<const char *>(fake_base);
+    const bool inside = GDN2_IN_BOUNDS(kBufQ, base + 56, 8);
+    const bool past_end = GDN2_IN_BOUNDS(kBufQ, base + 60, 8);
+    if (!inside || past_end) record_status(kStatusBadArgs);
+}
+#endif
+
 namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 gdn2_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA; }
+
+// The extents of one call's buffers for the debug build's device-side range
+// checks (bounds.cuh), from the call's pointers and the layouts of gdn2.h;
+// the release build does nothing here.  `e` is the bytes of one token element.
+struct CallBounds {
+    BoundsTable t{};
+    void add(int buf, const void *p, size_t bytes) {
+        if (p == nullptr) return;
+        t.lo[buf] = reinterpret_cast<uintptr_t>(p);
+        t.hi[buf] = t.lo[buf] + bytes;
+    }
+    gdn2_status_t publish(cudaStream_t st) const {
+#ifdef GDN2_DEBUG_BOUNDS
+        set_bounds_kernel<<<1, 1, 0, st>>>(t);
+        return from_cuda(cudaGetLastError());
+#else
+        (void)st;
+        return GDN2_OK;
+#endif
+    }
+};
+
+#ifdef GDN2_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+
+// token tensors [B', T, H | HV, d] (B' = 1 with cu_seqlens), states [B, HV, d_k, d_v]
+gdn2_status_t bounds_chunk(const void *q, const void *k, const void *v, const void *la, const void *b,
+                           const void *c, const void *w, const float *S0, const void *o, const float *S_T, int B,
+                           int Bt, int T, int H, int HV, int d_k, int d_v, const int *cu, size_t e,
+                           const FuseArgs *fz, cudaStream_t st) {
+    if (!kDebugBounds) return GDN2_OK;
+    CallBounds cb;
+    const size_t ntok = (size_t)Bt * T;
+    const size_t kb = ntok * H * d_k * e, vb = ntok * HV * d_v * e;
+    const size_t sb = (size_t)B * HV * d_k * d_v * sizeof(float);
+    cb.add(kBufQ, q, kb);
+    cb.add(kBufK, k, kb);
+    cb.add(kBufLA, la, kb);
+    cb.add(kBufB, b, kb);
+    cb.add(kBufC, c, kb);
+    cb.add(kBufV, v, vb);
+    cb.add(kBufW, w, vb);
+    cb.add(kBufO, o, vb);
+    cb.add(kBufS0, S0, sb);
+    cb.add(kBufST, S_T, sb);
+    if (fz != nullptr && fz->gate != nullptr) {
+        cb.add(kBufGate, fz->gate, vb);
+        cb.add(kBufNW, fz->norm_weight, (size_t)d_v * sizeof(float));
+    }
+    cb.add(kBufCU, cu, (size_t)(B + 1) * sizeof(int));
+    return cb.publish(st);
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
@@ -207,6 +281,10 @@ template <typename IO, int DK, int NVD>
 gdn2_status_t launch_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
                             const void *w, float *S, void *o, int B, int H, int HV, int d_v, cudaStream_t st,
                             const FuseArgs *fz) {
+    // the state is read and written in place: both extents are S
+    gdn2_status_t s = bounds_chunk(q, k, v, la, b, nullptr, w, S, o, S, B, B, 1, H, HV, DK, d_v, nullptr, sizeof(IO),
+                                   fz, st);
+    if (s != GDN2_OK) return s;
     dim3 grid((unsigned)((long)B * HV), d_v / NVD);
     if (fz == nullptr) {
         decode_step_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
@@ -300,6 +378,9 @@ gdn2_status_t dispatch_ffma_io(const void *q, const void *k, const void *v, cons
 gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
                             const void *w, const float *S0, void *o, float *S_T, const Shape &sh, int chunk,
                             gdn2_io_t io, cudaStream_t st, const FuseArgs *fz = nullptr) {
+    gdn2_status_t s = bounds_chunk(q, k, v, la, b, nullptr, w, S0, o, S_T, sh.B, sh.tensor_b(), sh.T, sh.H, sh.HV,
+                                   sh.d_k, sh.d_v, sh.cu, io == GDN2_IO_F32 ? 4 : 2, fz, st);
+    if (s != GDN2_OK) return s;
     if (io == GDN2_IO_F32) return dispatch_ffma_io<float>(q, k, v, la, b, w, S0, o, S_T, sh, chunk, st, fz);
     return dispatch_ffma_io<__nv_bfloat16>(q, k, v, la, b, w, S0, o, S_T, sh, chunk, st, fz);
 }
@@ -307,6 +388,9 @@ gdn2_status_t dispatch_ffma(const void *q, const void *k, const void *v, const v
 gdn2_status_t dispatch_tc(const void *q, const void *k, const void *v, const void *la, const void *b,
                           const void *w, const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
                           const FuseArgs *fz = nullptr) {
+    gdn2_status_t s = bounds_chunk(q, k, v, la, b, nullptr, w, S0, o, S_T, sh.B, sh.tensor_b(), sh.T, sh.H, sh.HV,
+                                   sh.d_k, sh.d_v, sh.cu, 2, fz, st);
+    if (s != GDN2_OK) return s;
     const bool wide = (sh.d_v % 128 == 0);
     if (sh.d_k == 64)
         return wide ? launch_tc<64, 128>(q, k, v, la, b, w, S0, o, S_T, sh, st, fz)
@@ -600,6 +684,9 @@ template <typename IO, int DK, int NVD>
 gdn2_status_t launch_qed_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
                                 const void *c, const void *w, float *S, void *o, int B, int H, int d_v, float eps,
                                 cudaStream_t st) {
+    gdn2_status_t s = bounds_chunk(q, k, v, la, b, c, w, S, o, S, B, B, 1, H, H, DK, d_v, nullptr, sizeof(IO),
+                                   nullptr, st);
+    if (s != GDN2_OK) return s;
     dim3 grid((unsigned)((long)B * H), d_v / NVD);
     decode_step_qed_kernel<IO, DK, NVD><<<grid, 256, 0, st>>>(
         static_cast<const IO *>(q), static_cast<const IO *>(k), static_cast<const IO *>(v),
@@ -622,6 +709,9 @@ extern "C" gdn2_status_t gdn2_chunk_fwd_qed(const void *q, const void *k, const 
     if (c && !aligned16(c)) return GDN2_ERR_MISALIGNED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (T == 0) return empty_sequence(S0, S_T, sh, st);
+    s = bounds_chunk(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, B, T, H, H, d_k, d_v, nullptr,
+                     io == GDN2_IO_F32 ? 4 : 2, nullptr, st);
+    if (s != GDN2_OK) return s;
     if (io == GDN2_IO_F32) {
         if (d_k == 64) return launch_qed_chunk<float, 64>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
         return launch_qed_chunk<float, 128>(q, k, v, log_alpha, b, c, w, S0, o, S_T, B, T, H, d_v, qed_eps, st);
@@ -683,6 +773,39 @@ extern "C" gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream) 
     return gdn2_device_status(stream);
 }
 
+extern "C" gdn2_status_t gdn2_debug_bounds_site(int *buffer, int *line, void *stream) {
+    if (!buffer || !line) return GDN2_ERR_INVALID_ARG;
+    *buffer = -1;
+    *line = 0;
+#ifdef GDN2_DEBUG_BOUNDS
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN2_ERR_CUDA;
+    unsigned int v = 0u;
+    if (cudaMemcpyFromSymbol(&v, g_bounds_site, sizeof(v)) != cudaSuccess) return GDN2_ERR_CUDA;
+    if (v != 0u) {
+        const unsigned int zero = 0u;
+        if (cudaMemcpyToSymbol(g_bounds_site, &zero, sizeof(zero)) != cudaSuccess) return GDN2_ERR_CUDA;
+        *buffer = (int)(v >> 16) - 1;
+        *line = (int)(v & 0xffffu);
+    }
+    return GDN2_OK;
+#else
+    (void)stream;
+    return GDN2_ERR_UNSUPPORTED;
+#endif
+}
+
+extern "C" gdn2_status_t gdn2_selftest_bounds(void *stream) {
+#ifdef GDN2_DEBUG_BOUNDS
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    selftest_bounds_kernel<<<1, 1, 0, st>>>(1ull << 40);
+    if (cudaGetLastError() != cudaSuccess) return GDN2_ERR_CUDA;
+    return gdn2_device_status(stream);
+#else
+    (void)stream;
+    return GDN2_ERR_UNSUPPORTED;
+#endif
+}
+
 extern "C" const char *gdn2_status_string(gdn2_status_t status) {
     switch (status) {
         case GDN2_OK: return "GDN2_OK";
@@ -691,6 +814,7 @@ extern "C" const char *gdn2_status_string(gdn2_status_t status) {
         case GDN2_ERR_MISALIGNED: return "GDN2_ERR_MISALIGNED";
         case GDN2_ERR_CUDA: return "GDN2_ERR_CUDA";
         case GDN2_ERR_DEVICE_TIMEOUT: return "GDN2_ERR_DEVICE_TIMEOUT";
+        case GDN2_ERR_OUT_OF_BOUNDS: return "GDN2_ERR_OUT_OF_BOUNDS";
         default: return "GDN2_ERR_UNKNOWN";
     }
 }

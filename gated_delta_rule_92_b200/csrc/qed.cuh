@@ -64,16 +64,19 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
     float *Sh = S + bh * (long)DK * d_v + j0 + cgr * 4;
     float4 s[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(reinterpret_cast<const float4 *>(Sh + (long)(i * RG + rg) * d_v));
+    for (int i = 0; i < RPT; ++i) {
+        const float4 *sp = reinterpret_cast<const float4 *>(Sh + (long)(i * RG + rg) * d_v);
+        s[i] = GDN2_IN_BOUNDS(kBufS0, sp, 16) ? __ldcs(sp) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 
     float qv = 0.f, kv = 0.f, bv = 0.f, cv = 0.f, lv = 0.f;
     if (tid < DK) {
         const long off = bh * DK + tid;
-        qv = ld_io(q + off);
-        kv = ld_io(k + off);
-        bv = ld_io(bg + off);
-        cv = ld_io(cg_ + off);
-        lv = ld_io(la + off);
+        qv = GDN2_IN_BOUNDS(kBufQ, q + off, sizeof(IO)) ? ld_io(q + off) : 0.f;
+        kv = GDN2_IN_BOUNDS(kBufK, k + off, sizeof(IO)) ? ld_io(k + off) : 0.f;
+        bv = GDN2_IN_BOUNDS(kBufB, bg + off, sizeof(IO)) ? ld_io(bg + off) : 0.f;
+        cv = GDN2_IN_BOUNDS(kBufC, cg_ + off, sizeof(IO)) ? ld_io(cg_ + off) : 0.f;
+        lv = GDN2_IN_BOUNDS(kBufLA, la + off, sizeof(IO)) ? ld_io(la + off) : 0.f;
     }
     // the query's part orthogonal to the key, normalised
     const float qk = block_sum_dk<DK>(qv * kv, s_scr);
@@ -95,7 +98,8 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
     }
     if (tid < NVD) {
         const long vo = bh * (long)d_v + j0 + tid;
-        s_wv[tid] = ld_io(wg + vo) * ld_io(v + vo);
+        s_wv[tid] = (GDN2_IN_BOUNDS(kBufW, wg + vo, sizeof(IO)) ? ld_io(wg + vo) : 0.f) *
+                    (GDN2_IN_BOUNDS(kBufV, v + vo, sizeof(IO)) ? ld_io(v + vo) : 0.f);
     }
     __syncthreads();
 
@@ -130,7 +134,8 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
             const float4 y = *reinterpret_cast<const float4 *>(&s_red[2][g][cgr * 4]);
             p.x += y.x; p.y += y.y; p.z += y.z; p.w += y.w;
         }
-        st_io4<IO>(o + bh * (long)d_v + j0 + cgr * 4, p.x + qk * x.x - qu * r2.x, p.y + qk * x.y - qu * r2.y,
+        if (GDN2_IN_BOUNDS(kBufO, o + bh * (long)d_v + j0 + cgr * 4, 4 * sizeof(IO)))
+            st_io4<IO>(o + bh * (long)d_v + j0 + cgr * 4, p.x + qk * x.x - qu * r2.x, p.y + qk * x.y - qu * r2.y,
                    p.z + qk * x.z - qu * r2.z, p.w + qk * x.w - qu * r2.w);
     }
 #pragma unroll
@@ -142,7 +147,8 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
         n.y = a * s[i].y + kr * x.y - ur * r2.y;
         n.z = a * s[i].z + kr * x.z - ur * r2.z;
         n.w = a * s[i].w + kr * x.w - ur * r2.w;
-        __stcs(reinterpret_cast<float4 *>(Sh + (long)row * d_v), n);
+        float4 *sp = reinterpret_cast<float4 *>(Sh + (long)row * d_v);
+        if (GDN2_IN_BOUNDS(kBufST, sp, 16)) __stcs(sp, n);
     }
 }
 
@@ -201,7 +207,8 @@ chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
 
     for (int idx = tid; idx < DK * NV; idx += 256) {
         const int c = idx / NV, j = idx % NV;
-        sS[c * LV + j] = S0 ? S0[(head * DK + c) * d_v + j0 + j] : 0.f;
+        const float *sp = S0 ? S0 + (head * DK + c) * d_v + j0 + j : nullptr;
+        sS[c * LV + j] = (sp && GDN2_IN_BOUNDS(kBufS0, sp, 4)) ? *sp : 0.f;
     }
     for (int n = 0; n < NC; ++n) {
         const long tok0 = (long)bb * T + (long)n * C;
@@ -212,17 +219,19 @@ chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
             const int t = idx / DK, c = idx % DK;
             const long g = ((tok0 + t) * H + h) * DK + c;
             const bool in = t < rows;
-            const float kv = in ? ld_io(k + g) : 0.f;
-            sQ[t * LK + c] = in ? ld_io(q + g) : 0.f;
+            const float kv = (in && GDN2_IN_BOUNDS(kBufK, k + g, sizeof(IO))) ? ld_io(k + g) : 0.f;
+            sQ[t * LK + c] = (in && GDN2_IN_BOUNDS(kBufQ, q + g, sizeof(IO))) ? ld_io(q + g) : 0.f;
             sK[(2 * t) * LK + c] = kv;
-            sE[(2 * t) * LK + c] = in ? ld_io(bg + g) * kv : 0.f;
-            sE[(2 * t + 1) * LK + c] = in ? ld_io(cg_ + g) : 0.f;
-            sG[t * LK + c] = in ? ld_io(la + g) : 0.f;
+            sE[(2 * t) * LK + c] = (in && GDN2_IN_BOUNDS(kBufB, bg + g, sizeof(IO))) ? ld_io(bg + g) * kv : 0.f;
+            sE[(2 * t + 1) * LK + c] = (in && GDN2_IN_BOUNDS(kBufC, cg_ + g, sizeof(IO))) ? ld_io(cg_ + g) : 0.f;
+            sG[t * LK + c] = (in && GDN2_IN_BOUNDS(kBufLA, la + g, sizeof(IO))) ? ld_io(la + g) : 0.f;
         }
         for (int idx = tid; idx < C * NV; idx += 256) {
             const int t = idx / NV, j = idx % NV;
             const long g = ((tok0 + t) * H + h) * (long)d_v + j0 + j;
-            sWV[(2 * t) * LV + j] = (t < rows) ? ld_io(wg + g) * ld_io(v + g) : 0.f;
+            const bool in = t < rows;
+            const float wv = (in && GDN2_IN_BOUNDS(kBufW, wg + g, sizeof(IO))) ? ld_io(wg + g) : 0.f;
+            sWV[(2 * t) * LV + j] = (in && GDN2_IN_BOUNDS(kBufV, v + g, sizeof(IO))) ? wv * ld_io(v + g) : 0.f;
             sWV[(2 * t + 1) * LV + j] = 0.f;
         }
         __syncthreads();
@@ -467,6 +476,7 @@ chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
                     const long g = ((tok0 + t) * H + h) * (long)d_v + j0 + 4 * ct;
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
+                        if (!GDN2_IN_BOUNDS(kBufO, o + g + y, sizeof(IO))) continue;
                         if constexpr (sizeof(IO) == 4) o[g + y] = ov[x][y];
                         else o[g + y] = __float2bfloat16_rn(ov[x][y]);
                     }
@@ -505,7 +515,8 @@ chunk_fwd_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const I
     if (S_T) {
         for (int idx = tid; idx < DK * NV; idx += 256) {
             const int c = idx / NV, j = idx % NV;
-            S_T[(head * DK + c) * d_v + j0 + j] = sS[c * LV + j];
+            float *sp = S_T + (head * DK + c) * d_v + j0 + j;
+            if (GDN2_IN_BOUNDS(kBufST, sp, 4)) *sp = sS[c * LV + j];
         }
     }
 }

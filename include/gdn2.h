@@ -69,7 +69,9 @@ typedef enum {
     GDN2_ERR_UNSUPPORTED = 2,     /* valid but outside the built shapes      */
     GDN2_ERR_MISALIGNED = 3,      /* a pointer is not 16-byte aligned        */
     GDN2_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed       */
-    GDN2_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait ran out      */
+    GDN2_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out      */
+    GDN2_ERR_OUT_OF_BOUNDS = 6    /* debug build: a device-side range check  */
+                                  /* failed (the access was skipped)         */
 } gdn2_status_t;
 
 /*
@@ -358,7 +360,8 @@ gdn2_status_t gdn2_decode_step_qed(const void *q, const void *k, const void *v,
  * current device's status word.  Returns GDN2_OK, GDN2_ERR_DEVICE_TIMEOUT if
  * a kernel gave up on a bounded wait since the last call,
  * GDN2_ERR_INVALID_ARG if a kernel skipped a sequence with malformed
- * cu_seqlens offsets, or GDN2_ERR_CUDA.
+ * cu_seqlens offsets, GDN2_ERR_OUT_OF_BOUNDS (debug build only) if a range
+ * check failed, or GDN2_ERR_CUDA.
  */
 gdn2_status_t gdn2_device_status(void *stream);
 
@@ -371,6 +374,39 @@ gdn2_status_t gdn2_device_status(void *stream);
  * mechanism works.
  */
 gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream);
+
+/*
+ * Debug build (libgdn2_debug.so: the same sources compiled with
+ * -DGDN2_DEBUG_BOUNDS).  Not an operation of the method; a build of the
+ * library for finding indexing mistakes.  Every per-thread global load and
+ * store of the kernels is checked against the extent of the argument buffer
+ * it belongs to; the host entry points publish those extents -- computed from
+ * the call's pointers and sizes and the layouts documented above -- in stream
+ * order before each launch.  A failed check does not trap or fault: it skips
+ * the access (a load yields 0), records GDN2_ERR_OUT_OF_BOUNDS in the status
+ * word that gdn2_device_status() returns, and records the site of the first
+ * failure.  TMA copies are bounded by their tensor maps.  The extents are one
+ * table per device, so the debug build expects one call in flight per device
+ * (calls on several streams of one device at once may check against each
+ * other's extents).  In the release library the checks are compiled out.
+ *
+ * gdn2_debug_bounds_site -- synchronise `stream`, then read and clear the
+ * site of the first failed check since the last read: *buffer is the
+ * argument (0 q, 1 k, 2 v, 3 log_alpha, 4 b, 5 w, 6 c, 7 S0 (decode: S),
+ * 8 S_T (decode: S), 9 o, 10 gate, 11 norm_weight, 12 cu_seqlens) and *line
+ * the source line of the check; -1 and 0 when none failed.  Returns GDN2_OK,
+ * GDN2_ERR_INVALID_ARG for a null output pointer, GDN2_ERR_CUDA, or
+ * GDN2_ERR_UNSUPPORTED in the release library.
+ *
+ * gdn2_selftest_bounds -- exercise the check on addresses alone (nothing is
+ * dereferenced): one thread sets a 64-byte extent for buffer 0, checks a
+ * range inside it (must pass) and one that runs past its end (must fail).
+ * Returns gdn2_device_status(stream): GDN2_ERR_OUT_OF_BOUNDS when the check
+ * answered both correctly, GDN2_ERR_INVALID_ARG when it did not; the site then
+ * reads buffer 0.  GDN2_ERR_UNSUPPORTED in the release library.
+ */
+gdn2_status_t gdn2_debug_bounds_site(int *buffer, int *line, void *stream);
+gdn2_status_t gdn2_selftest_bounds(void *stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn2_status_string(gdn2_status_t status);

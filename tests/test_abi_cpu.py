@@ -203,3 +203,41 @@ def test_host_binding_rejects_bad_tensors_before_any_copy():
         g.chunk_fwd_host(q, q, v, q, q, v, torch.zeros(B, H, dk, dv + 1))
     with pytest.raises(ValueError):   # mixed dtypes
         g.chunk_fwd_host(q, q.float(), v, q, q, v)
+
+
+@pytest.fixture(scope="module")
+def LD():
+    gbuild.build()
+    return g._open(g.DEBUG_LIB_PATH)
+
+
+def test_debug_build_exports_every_declared_symbol(LD):
+    for name in declared_functions():
+        assert hasattr(LD, name), name
+    out = os.popen(f"nm -D --defined-only {g.DEBUG_LIB_PATH}").read()
+    exported = set(re.findall(r" T (gdn2_[a-z0-9_]+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_debug_bounds_entry_points_on_host(L, LD):
+    P, I = ctypes.c_void_p, ctypes.c_int
+    a, b = I(7), I(7)
+    # the release library has no range checks: both calls say so before any CUDA call
+    assert L.gdn2_debug_bounds_site(ctypes.byref(a), ctypes.byref(b), None) == 2
+    assert (a.value, b.value) == (-1, 0)
+    assert L.gdn2_selftest_bounds(None) == 2
+    # null outputs are argument errors in either build
+    assert L.gdn2_debug_bounds_site(None, ctypes.byref(b), None) == 1
+    assert LD.gdn2_debug_bounds_site(ctypes.byref(a), None, None) == 1
+    assert LD.gdn2_status_string(6) == b"GDN2_ERR_OUT_OF_BOUNDS"
+    # the debug build validates arguments on the host exactly as the release one
+    for kw in ({"ptr": None}, {"B": 0}, {"ptr": 24}, {"chunk": 48}, {"dk": 96}):
+        assert _chunk_call(LD, **kw) == _chunk_call(L, **kw)
+
+
+def test_debug_bounds_context_switches_library():
+    release = g.lib()
+    with g.debug_bounds() as LD:
+        assert g.lib() is LD and LD is not release
+        assert LD._name.endswith("libgdn2_debug.so")
+    assert g.lib() is release
