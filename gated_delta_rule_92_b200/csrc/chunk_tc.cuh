@@ -78,7 +78,8 @@ struct TcCfg {
     static constexpr uint32_t OFF_GC = OFF_CARRY + 2560;         // state factors [3][2][128]
     static constexpr uint32_t OFF_NRM = OFF_GC + 3072;           // fused prep: 1/|q_r|, 1/|k_r| [64][2]
     static constexpr uint32_t OFF_NW = OFF_NRM + 512;            // fused epilogue: norm weight [NV]
-    static constexpr uint32_t OFF_BAR = OFF_NW + 512;
+    static constexpr uint32_t OFF_RMS = OFF_NW + 512;            // fused epilogue: 1 / rms(o_r) [64]
+    static constexpr uint32_t OFF_BAR = OFF_RMS + 256;
     static constexpr uint32_t OFF_TMEMP = OFF_BAR + 256;   // up to 32 mbarriers
     static constexpr uint32_t OFF_STOP = OFF_TMEMP + 4;    // first chunk handed to the token tail
     static constexpr uint32_t OFF_SEQ = OFF_TMEMP + 8;     // this CTA's sequence: tok0 (8 B), len, bb
@@ -1754,6 +1755,23 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             }
+            // fused epilogue: thread t takes the 16-byte column chunk t % (NV / 8) of rows
+            // t / (NV / 8) + i * (128 / (NV / 8)); its gate loads are issued here, so that
+            // they land while MMA_o runs and o is read out of TMEM
+            constexpr int E_CPR = NV / 8, E_RPP = kChainThreads / E_CPR;
+            const int e_c16 = t % E_CPR, e_rr = t / E_CPR;
+            uint4 gall[EPI ? 64 / E_RPP : 1];
+            if constexpr (EPI) {
+                const __nv_bfloat16 *gbase = static_cast<const __nv_bfloat16 *>(fz.gate);
+#pragma unroll
+                for (int i = 0; i < 64 / E_RPP; ++i) {
+                    const int r = i * E_RPP + e_rr;
+                    const uint4 *gp = reinterpret_cast<const uint4 *>(
+                        gbase + ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * e_c16);
+                    gall[i] = (n * 64 + r < len && GDN2_IN_BOUNDS(kBufGate, gp, 16)) ? __ldg(gp)
+                                                                                     : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
             {
                 const bool ok = mbar_wait(bc3, ph3, wait_ns);
                 ph3 ^= 1u;
@@ -1786,7 +1804,7 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const long orow_off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0;
                 __nv_bfloat16 *orow = o + orow_off;
                 bool plain = true;
-                if constexpr (EPI) {   // first half of the epilogue: o / rms(o) -> bf16 in the U tile
+                if constexpr (EPI) {   // first half of the epilogue: o -> bf16 in the U tile, 1/rms(o) per row
                     plain = false;
                     float ss = 0.f;
 #pragma unroll 1
@@ -1795,23 +1813,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tmem_ld32(t_X + lane_q + jc * 32, x);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) ss = fmaf(x[e], x[e], ss);
-                    }
-                    const float inv = rsqrtf(ss / (float)NV + fz.norm_eps);
-#pragma unroll 1
-                    for (int jc = 0; jc < NV / 32; ++jc) {
-                        float x[32];
-                        tmem_ld32(t_X + lane_q + jc * 32, x);
                         const uint32_t tile = sb + Cfg::OFF_U + ((jc * 32) >> 6) * 8192u;
                         const uint32_t ch0 = ((jc * 32) & 63) >> 3;
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const int e = 8 * q4;
-                            st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(x[e] * inv, x[e + 1] * inv),
-                                         pack_bf16x2(x[e + 2] * inv, x[e + 3] * inv),
-                                         pack_bf16x2(x[e + 4] * inv, x[e + 5] * inv),
-                                         pack_bf16x2(x[e + 6] * inv, x[e + 7] * inv));
+                            st_shared_v4(tile + sw128_chunk(r, ch0 + q4), pack_bf16x2(x[e], x[e + 1]),
+                                         pack_bf16x2(x[e + 2], x[e + 3]), pack_bf16x2(x[e + 4], x[e + 5]),
+                                         pack_bf16x2(x[e + 6], x[e + 7]));
                         }
                     }
+                    reinterpret_cast<float *>(smem + Cfg::OFF_RMS)[r] = rsqrtf(ss / (float)NV + fz.norm_eps);
                 }
 #pragma unroll 1
                 for (int jc = 0; jc < NV / 32 && plain; ++jc) {
@@ -1828,40 +1840,35 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             }
-            if constexpr (EPI) {   // second half: . weight . silu(g), coalesced, by all four warps
+            if constexpr (EPI) {   // second half: / rms . weight . silu(g), coalesced, by all four warps
                 named_bar(2, kChainThreads);
                 const float *nw = reinterpret_cast<const float *>(smem + Cfg::OFF_NW);
-                constexpr int CPR = NV / 8;                 // 16-byte chunks per row
-                constexpr int RPP = kChainThreads / CPR;    // rows per pass
-                const int c16 = t % CPR, rr = t / CPR;
-                const float4 w0 = *reinterpret_cast<const float4 *>(nw + 8 * c16);
-                const float4 w1 = *reinterpret_cast<const float4 *>(nw + 8 * c16 + 4);
+                const float *rinv = reinterpret_cast<const float *>(smem + Cfg::OFF_RMS);
+                const float4 w0 = *reinterpret_cast<const float4 *>(nw + 8 * e_c16);
+                const float4 w1 = *reinterpret_cast<const float4 *>(nw + 8 * e_c16 + 4);
                 const float wt[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                const __nv_bfloat16 *gbase = static_cast<const __nv_bfloat16 *>(fz.gate);
-                uint4 gall[64 / RPP];   // every gate load of this thread issued up front
 #pragma unroll
-                for (int i = 0; i < 64 / RPP; ++i) {
-                    const int r = i * RPP + rr;
-                    const uint4 *gp = reinterpret_cast<const uint4 *>(
-                        gbase + ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * c16);
-                    gall[i] = (n * 64 + r < len && GDN2_IN_BOUNDS(kBufGate, gp, 16)) ? __ldg(gp)
-                                                                                     : make_uint4(0u, 0u, 0u, 0u);
-                }
-#pragma unroll
-                for (int i = 0; i < 64 / RPP; ++i) {
-                    const int r = i * RPP + rr;
+                for (int i = 0; i < 64 / E_RPP; ++i) {
+                    const int r = i * E_RPP + e_rr;
                     if (n * 64 + r >= len) continue;   // padding rows
-                    const long off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * c16;
+                    const long off = ((tok0 + (long)n * 64 + r) * HV + hv) * (long)d_v + j0 + 8 * e_c16;
                     const uint4 gv = gall[i];
+                    const float inv = rinv[r];
                     uint32_t a0, a1, a2, a3;
-                    ld_shared_v4(sb + Cfg::OFF_U + (c16 >> 3) * 8192u + sw128_chunk(r, c16 & 7), a0, a1, a2, a3);
+                    ld_shared_v4(sb + Cfg::OFF_U + (e_c16 >> 3) * 8192u + sw128_chunk(r, e_c16 & 7), a0, a1, a2, a3);
                     const uint32_t ov[4] = {a0, a1, a2, a3}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
                     uint32_t pk[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float g0 = bf16_lo(gw[e]), g1 = bf16_hi(gw[e]);
-                        pk[e] = pack_bf16x2(bf16_lo(ov[e]) * wt[2 * e] * g0 * sigmoid_tanh(g0),
-                                            bf16_hi(ov[e]) * wt[2 * e + 1] * g1 * sigmoid_tanh(g1));
+                    for (int e = 0; e < 4; ++e) {   // two channels per paired instruction
+                        const float2 g2 = make_float2(bf16_lo(gw[e]), bf16_hi(gw[e]));
+                        const float2 hx = mul_f32x2(g2, make_float2(0.5f, 0.5f));
+                        float2 th;
+                        asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(hx.x));
+                        asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(hx.y));
+                        const float2 sg = fma_f32x2(th, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
+                        const float2 iw = mul_f32x2(make_float2(inv, inv), make_float2(wt[2 * e], wt[2 * e + 1]));
+                        const float2 y = mul_f32x2(mul_f32x2(mul_f32x2(make_float2(bf16_lo(ov[e]), bf16_hi(ov[e])), iw), g2), sg);
+                        pk[e] = pack_bf16x2(y.x, y.y);
                     }
                     if (GDN2_IN_BOUNDS(kBufO, o + off, 16))
                         *reinterpret_cast<uint4 *>(o + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
