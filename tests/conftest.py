@@ -24,3 +24,17 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _debug_bounds_sweep(request):
+    """With GDN2_DEBUG_BOUNDS=1 every library call goes through the debug build
+    (libgdn2_debug.so, device-side range checks); after each GPU test no check
+    may have failed.  `GDN2_DEBUG_BOUNDS=1 pytest -m gpu` sweeps the whole suite."""
+    yield
+    if os.environ.get("GDN2_DEBUG_BOUNDS") != "1" or request.node.get_closest_marker("gpu") is None:
+        return
+    import gated_delta_rule_92_b200 as g
+    assert os.path.basename(g.lib()._name) == "libgdn2_debug.so"
+    site = g.debug_bounds_site()
+    assert site is None, f"a device-side range check failed: buffer {site[0]}, line {site[1]}"
