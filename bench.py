@@ -208,6 +208,12 @@ def aggregate_throughput(ms_local: float, steps: int, tokens_per_rank_step: int,
 
 
 # ------------------------------------------------------- our measurements
+def nvtx(name: str):
+    """An NVTX range around one phase of the harness (visible to nsys / ncu
+    range filters; a no-op without a profiler attached)."""
+    return torch.cuda.nvtx.range(name)
+
+
 def steady_rounds(step, stream, min_s: float = 0.5, per_round: int = 50, max_rounds: int = 400):
     """Rounds of `per_round` back-to-back calls, each timed with CUDA events on
     `stream`, until `min_s` of device time has been covered; returns the
@@ -230,7 +236,7 @@ def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None, steady_
         g.chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], d["S0"], o=o, S_T=S_T,
                     stream=stream)
 
-    with torch.cuda.stream(stream):
+    with nvtx("warm-up " + wl.name), torch.cuda.stream(stream):
         for _ in range(warmup):
             step()
     torch.cuda.synchronize()
@@ -240,13 +246,16 @@ def bench_chunk(g, wl, steps, warmup, rank, world, stream, sampler=None, steady_
     if sampler is not None:
         # the sampler covers the timed steps and the steady rounds after them
         with sampler:
-            ms = device_time_ms(step, steps, stream)
+            with nvtx("timed " + wl.name):
+                ms = device_time_ms(step, steps, stream)
             torch.cuda.synchronize()
             barrier(world)
             if steady_s > 0:
-                steady = steady_rounds(step, stream, steady_s)
+                with nvtx("steady rounds " + wl.name):
+                    steady = steady_rounds(step, stream, steady_s)
     else:
-        ms = device_time_ms(step, steps, stream)
+        with nvtx("timed " + wl.name):
+            ms = device_time_ms(step, steps, stream)
         torch.cuda.synchronize()
         barrier(world)
     if g.device_status() != 0:
@@ -630,12 +639,14 @@ def main():
     achieved = abytes / (launch_ms / 1e3) / 1e9
     flops = chunk_flops(wl)
 
-    e2e_ms, h2d, d2h, e2e_same = bench_chunk_e2e(g, wl, d, args.e2e_steps, stream, o, S_T)
+    with nvtx("e2e host buffers"):
+        e2e_ms, h2d, d2h, e2e_same = bench_chunk_e2e(g, wl, d, args.e2e_steps, stream, o, S_T)
     e2e_val, e2e_ms = aggregate_throughput(e2e_ms, args.e2e_steps, wl.B * wl.T, world)
     del d, o, S_T
     torch.cuda.empty_cache()
 
     extras = {}
+    torch.cuda.nvtx.range_push("other workloads")
     if not args.no_extras:
         wl3 = W.BY_NAME["chunk_bf16_negeig"]
         ms3, d3, _, _ = bench_chunk(g, wl3, max(5, args.steps // 4), 3, rank, world, stream)
@@ -739,9 +750,11 @@ def main():
                          "unit": "GB/s", "frac": bdq / (pq / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes_per_step": bdq}}
         torch.cuda.empty_cache()
 
+    torch.cuda.nvtx.range_pop()
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
-        tok_s, cores, desc = oracle_sample(wl, head_sample_fn(wl))
+        with nvtx("oracle on the host cores"):
+            tok_s, cores, desc = oracle_sample(wl, head_sample_fn(wl))
         cpu = {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc}
 
     if rank == 0:

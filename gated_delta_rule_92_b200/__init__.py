@@ -45,7 +45,7 @@ EXPORTED = ("gdn2_chunk_fwd", "gdn2_chunk_fwd_cuda_core", "gdn2_chunk_fwd_host",
             "gdn2_chunk_fwd_host_workspace", "gdn2_chunk_fwd_host_noalloc", "gdn2_decode_step",
             "gdn2_chunk_fwd_ex", "gdn2_decode_step_ex", "gdn2_chunk_fwd_qed", "gdn2_decode_step_qed",
             "gdn2_device_status", "gdn2_selftest_wait_timeout", "gdn2_debug_bounds_site",
-            "gdn2_selftest_bounds", "gdn2_status_string", "gdn2_version")
+            "gdn2_selftest_bounds", "gdn2_testing_fail_launches", "gdn2_status_string", "gdn2_version")
 FUSE_INPUT_PREP = 1    # q, k, b, w are raw: L2-normalise q, k over d_k; b, w = sigmoid
 FUSE_NEG_EIGVAL = 2    # with FUSE_INPUT_PREP: b = 2 sigmoid(b)
 NOALLOC_WORKSPACE_BYTES = 64 << 20   # GDN2_NOALLOC_WORKSPACE_BYTES: the no-alloc entry's fixed workspace
@@ -129,6 +129,8 @@ def _open(path: str) -> ctypes.CDLL:
         L.gdn2_debug_bounds_site.restype = I
         L.gdn2_selftest_bounds.argtypes = [P]
         L.gdn2_selftest_bounds.restype = I
+        L.gdn2_testing_fail_launches.argtypes = [I, I]
+        L.gdn2_testing_fail_launches.restype = I
         L.gdn2_version.argtypes = []
         L.gdn2_version.restype = I
         _opened[path] = L
@@ -487,6 +489,14 @@ def debug_bounds_site(stream=None):
     if st != 0:
         raise Gdn2Error(st, "gdn2_debug_bounds_site")
     return None if buf.value < 0 else (BOUNDS_BUFFERS[buf.value], line.value)
+
+
+def testing_fail_launches(pass_: int, fail: int) -> None:
+    """Fault injection for tests: after `pass_` more kernel launch sites, the
+    next `fail` ones return GDN2_ERR_CUDA without launching; fail = 0 disarms."""
+    st = lib().gdn2_testing_fail_launches(int(pass_), int(fail))
+    if st != 0:
+        raise Gdn2Error(st, "gdn2_testing_fail_launches")
 
 
 def selftest_bounds(stream=None) -> int:

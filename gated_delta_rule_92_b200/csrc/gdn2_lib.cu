@@ -9,6 +9,7 @@
 
 #include <climits>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/gdn2.h"
@@ -59,6 +60,26 @@ namespace {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 gdn2_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN2_OK : GDN2_ERR_CUDA; }
+
+// Injected launch failures (gdn2_testing_fail_launches): after `pass` more
+// launches, the next `fail` launch sites return GDN2_ERR_CUDA without
+// launching, as a failed launch would.  Disarmed (the default) it costs one
+// relaxed atomic load per launch.
+std::atomic<bool> g_inject_armed{false};
+std::mutex g_inject_lock;
+long g_inject_pass = 0, g_inject_fail = 0;
+
+gdn2_status_t launch_gate() {
+    if (!g_inject_armed.load(std::memory_order_relaxed)) return GDN2_OK;
+    std::lock_guard<std::mutex> guard(g_inject_lock);
+    if (g_inject_fail <= 0) return GDN2_OK;
+    if (g_inject_pass > 0) {
+        --g_inject_pass;
+        return GDN2_OK;
+    }
+    if (--g_inject_fail == 0) g_inject_armed.store(false, std::memory_order_relaxed);
+    return GDN2_ERR_CUDA;
+}
 
 // The extents of one call's buffers for the debug build's device-side range
 // checks (bounds.cuh), from the call's pointers and the layouts of gdn2.h;
@@ -162,6 +183,7 @@ template <typename IO>
 gdn2_status_t launch_rmsnorm(void *o, const void *g, const float *weight, long rows, int d_v, float eps,
                              cudaStream_t st) {
     if (rows == 0) return GDN2_OK;
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     gated_rmsnorm_kernel<IO><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
         static_cast<IO *>(o), static_cast<const IO *>(g), weight, rows, d_v, eps);
     return from_cuda(cudaGetLastError());
@@ -173,6 +195,7 @@ gdn2_status_t launch_tc_kernel(const CUtensorMap &tq, const CUtensorMap &tk, con
                                const float *S0,
                                void *o, float *S_T, const Shape &sh, cudaStream_t st, const FuseArgs &fz,
                                const TailArgs &ta) {
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     using Cfg = TcCfg<DK, NV>;
     auto kern = chunk_fwd_tc_kernel<DK, NV, PREP, EPI, VARLEN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_ALLOC);
@@ -229,6 +252,7 @@ template <int DK, int NV>
 gdn2_status_t launch_tc_qed(const void *q, const void *k, const void *v, const void *la, const void *b,
                             const void *c, const void *w, const float *S0, void *o, float *S_T, int B, int T, int H,
                             int d_v, float eps, cudaStream_t st) {
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     using Cfg = TcCfg<DK, NV>;
     CUtensorMap tq, tk, tb, tc, tv, tw, to;
     if (!make_token_map(&tq, q, B, T, H, DK, 32) || !make_token_map(&tk, k, B, T, H, DK, 32) ||
@@ -255,6 +279,7 @@ template <typename IO, int DK, int CH>
 gdn2_status_t launch_ffma(const void *q, const void *k, const void *v, const void *la, const void *b,
                           const void *w, const float *S0, void *o, float *S_T, const Shape &sh, cudaStream_t st,
                           const FuseArgs *fz = nullptr) {
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     using Cfg = FfmaCfg<DK, CH>;
     dim3 grid(sh.d_v / Cfg::NV, sh.HV, sh.B);
     const IO *qp = static_cast<const IO *>(q), *kp = static_cast<const IO *>(k), *vp = static_cast<const IO *>(v);
@@ -281,6 +306,7 @@ template <typename IO, int DK, int NVD>
 gdn2_status_t launch_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
                             const void *w, float *S, void *o, int B, int H, int HV, int d_v, cudaStream_t st,
                             const FuseArgs *fz) {
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     // the state is read and written in place: both extents are S
     gdn2_status_t s = bounds_chunk(q, k, v, la, b, nullptr, w, S, o, S, B, B, 1, H, HV, DK, d_v, nullptr, sizeof(IO),
                                    fz, st);
@@ -668,6 +694,7 @@ template <typename IO, int DK>
 gdn2_status_t launch_qed_chunk(const void *q, const void *k, const void *v, const void *la, const void *b,
                                const void *c, const void *w, const float *S0, void *o, float *S_T, int B,
                                int T, int H, int d_v, float eps, cudaStream_t st) {
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     using Cfg = QedCfg<DK>;
     auto kern = chunk_fwd_qed_kernel<IO, DK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::BYTES) != cudaSuccess)
@@ -684,6 +711,7 @@ template <typename IO, int DK, int NVD>
 gdn2_status_t launch_qed_decode(const void *q, const void *k, const void *v, const void *la, const void *b,
                                 const void *c, const void *w, float *S, void *o, int B, int H, int d_v, float eps,
                                 cudaStream_t st) {
+    if (launch_gate() != GDN2_OK) return GDN2_ERR_CUDA;
     gdn2_status_t s = bounds_chunk(q, k, v, la, b, c, w, S, o, S, B, B, 1, H, H, DK, d_v, nullptr, sizeof(IO),
                                    nullptr, st);
     if (s != GDN2_OK) return s;
@@ -771,6 +799,15 @@ extern "C" gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream) 
     selftest_wait_kernel<<<1, 32, 0, st>>>(1000ull * (unsigned long long)limit_us);
     if (cudaGetLastError() != cudaSuccess) return GDN2_ERR_CUDA;
     return gdn2_device_status(stream);
+}
+
+extern "C" gdn2_status_t gdn2_testing_fail_launches(int pass, int fail) {
+    if (pass < 0 || fail < 0) return GDN2_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> guard(g_inject_lock);
+    g_inject_pass = pass;
+    g_inject_fail = fail;
+    g_inject_armed.store(fail > 0, std::memory_order_relaxed);
+    return GDN2_OK;
 }
 
 extern "C" gdn2_status_t gdn2_debug_bounds_site(int *buffer, int *line, void *stream) {

@@ -408,6 +408,17 @@ gdn2_status_t gdn2_selftest_wait_timeout(int limit_us, void *stream);
 gdn2_status_t gdn2_debug_bounds_site(int *buffer, int *line, void *stream);
 gdn2_status_t gdn2_selftest_bounds(void *stream);
 
+/*
+ * gdn2_testing_fail_launches -- fault injection on the host, for tests of the
+ * error paths (not an operation of the method).  After `pass` more kernel
+ * launch sites have run normally, the next `fail` launch sites return
+ * GDN2_ERR_CUDA without launching, as a launch that the driver refused would;
+ * the calls that reach them return that status.  Nothing faults on the
+ * device and the context stays usable.  `fail` = 0 disarms (the default).
+ * Process-wide; returns GDN2_ERR_INVALID_ARG for a negative argument.
+ */
+gdn2_status_t gdn2_testing_fail_launches(int pass, int fail);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdn2_status_string(gdn2_status_t status);
 

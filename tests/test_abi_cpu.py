@@ -242,3 +242,10 @@ def test_debug_bounds_context_switches_library():
         assert g.lib() is LD and LD is not release
         assert LD._name.endswith("libgdn2_debug.so")
     assert g.lib() is release
+
+
+def test_testing_fail_launches_arguments(L):
+    assert L.gdn2_testing_fail_launches(-1, 1) == 1
+    assert L.gdn2_testing_fail_launches(0, -1) == 1
+    assert L.gdn2_testing_fail_launches(3, 2) == 0
+    assert L.gdn2_testing_fail_launches(0, 0) == 0   # disarmed again
