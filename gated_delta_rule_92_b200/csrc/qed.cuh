@@ -32,6 +32,26 @@ __device__ __forceinline__ float block_sum_dk(float x, float *scratch) {
     return t;
 }
 
+// The same for two values at once (one exchange through `scratch`, DK / 32 float2).
+template <int DK>
+__device__ __forceinline__ float2 block_sum2_dk(float2 x, float2 *scratch) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        x.x += __shfl_xor_sync(0xffffffffu, x.x, off);
+        x.y += __shfl_xor_sync(0xffffffffu, x.y, off);
+    }
+    if ((threadIdx.x & 31) == 0 && threadIdx.x < DK) scratch[threadIdx.x >> 5] = x;
+    __syncthreads();
+    float2 t = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < DK / 32; ++w) {
+        t.x += scratch[w].x;
+        t.y += scratch[w].y;
+    }
+    __syncthreads();
+    return t;
+}
+
 // One decode step per (b, h, NVD-column slice of d_v), 256 threads.  Per
 // value column j, with S = S_{t-1} and the decay alpha:
 //     r1_j = sum_i (b_i k_i alpha_i) S_ij,  r2_j = sum_i (c_i u_i alpha_i) S_ij,
@@ -54,6 +74,7 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
     __shared__ float s_wv[NVD];
     __shared__ __align__(16) float s_red[3][RG][NVD];
     __shared__ float s_scr[DK / 32];
+    __shared__ float2 s_scr2[DK / 32];
 
     const int tid = threadIdx.x;
     const int cgr = tid % TPR;   // float4 column group
@@ -79,8 +100,8 @@ decode_step_qed_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const
         lv = GDN2_IN_BOUNDS(kBufLA, la + off, sizeof(IO)) ? ld_io(la + off) : 0.f;
     }
     // the query's part orthogonal to the key, normalised
-    const float qk = block_sum_dk<DK>(qv * kv, s_scr);
-    const float kk = block_sum_dk<DK>(kv * kv, s_scr);
+    const float2 qkk = block_sum2_dk<DK>(make_float2(qv * kv, kv * kv), s_scr2);
+    const float qk = qkk.x, kk = qkk.y;
     const float coef = kk > 0.f ? qk / kk : 0.f;
     const float rv = qv - coef * kv;
     const float rr = block_sum_dk<DK>(rv * rv, s_scr);
