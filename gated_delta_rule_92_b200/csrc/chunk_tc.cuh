@@ -1171,10 +1171,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *bk1 = bars + 19;        // MMA1 complete
     uint64_t *bct = bars + 20;        // MMA_T complete (chain)
     uint64_t *bc1 = bars + 21, *bc2 = bars + 22, *bc3 = bars + 23;
-    uint64_t *drain = bars + 24;      // [2] teardown: key and chain MMA issuers
+    uint64_t *drain = bars + 24;      // [2] teardown: key and chain MMA issuers (the MMA3 issuer: drain3)
     uint64_t *ut_ready = bars + 26;   // MMA3 of a chunk complete: T(W.V) in TMEM
     uint64_t *t_free = bars + 27;     // MMA_T complete: the T tile is free for the next solve
-    constexpr int kNumBars = 28;
+    uint64_t *drain3 = bars + 28;     // teardown: the MMA3 issuer (key thread 128)
+    constexpr int kNumBars = 29;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_TMEMP);
     float *gC = reinterpret_cast<float *>(smem + Cfg::OFF_GC);
     float *sA = reinterpret_cast<float *>(smem + Cfg::OFF_SCR);
@@ -1313,7 +1314,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int t = tid, l = tid & 31, kq = warp & 3, kh = warp >> 2;   // lane quarter, column half
         const bool grp_b = t >= 128;
         uint32_t ph1 = 0;
-        bool mma3_failed = false;   // thread 0 only
+        // MMA1 is issued by key thread 0 and MMA3 by key thread 128 (warp 4), so that
+        // the two issues, each held while the tensor pipe works through its queue,
+        // overlap at the turn of an iteration instead of following each other
+        constexpr int kMma3Issuer = 128;
+        bool mma3_failed = false;   // thread kMma3Issuer only
         float *carry = reinterpret_cast<float *>(smem + Cfg::OFF_CARRY);
         float2 *nrm = reinterpret_cast<float2 *>(smem + Cfg::OFF_NRM);
         // group B: log_alpha of the next chunk to prepare
@@ -1497,6 +1502,8 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (t == 0) {
                 mbar_arrive(w_free);   // w tile (solve scratch) is free
                 mbar_arrive(&full[s]);
+            }
+            if (t == kMma3Issuer) {
                 const bool ok_ut = (m == 0) || mbar_wait(utfree, static_cast<uint32_t>((m - 1) & 1), wait_ns);
                 if (ok_ut) {
                     tc_fence_after();
@@ -1513,9 +1520,10 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         if (mma3_failed) failed = true;
-        if (t == 0) {   // wait (bounded) for this issuer's MMAs before teardown
-            umma_commit(&drain[0]);
-            mbar_wait(&drain[0], 0u, wait_ns);
+        if (t == 0 || t == kMma3Issuer) {   // wait (bounded) for each issuer's MMAs before teardown
+            uint64_t *db = (t == 0) ? &drain[0] : drain3;
+            umma_commit(db);
+            mbar_wait(db, 0u, wait_ns);
         }
     } else {
         // ========================================================== chain side
