@@ -1608,12 +1608,16 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             const uint32_t OQE = s ? Cfg::OFF_QE1 : Cfg::OFF_QE0, OK = Cfg::OFF_K + (n % 3) * 16384u;
             const uint32_t OP = s ? Cfg::OFF_P1 : Cfg::OFF_P0;
-            {
+            // MMA_s needs only chunk n's prepared Q~ and E (done before the hand-off of
+            // chunk n - 1, or, for chunk 0, before full[0]) and the chain's own state,
+            // so it is issued before the wait for the rest of chunk n's key products
+            // (T, P and the next chunk's prep); for the same reason chunk n's own stop
+            // decision is final here
+            if (n == 0) {
                 const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((n >> 1) & 1), wait_ns);
                 if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
             }
-            const int stop_now = *stop_at;   // includes chunk n + 1's decision (its prep is done)
-            if (stop_now <= n) break;        // handed to the token tail from chunk n on
+            if (*stop_at <= n) break;   // handed to the token tail from chunk n on
             // ------------------------------------------------------ MMA_s
             if (t == 0) {
                 tc_fence_after();
@@ -1625,6 +1629,11 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 umma_commit(bc1);
                 if (!EPI) bulk_wait_read_all();   // the previous O store has read the U tile
             }
+            if (n > 0) {
+                const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((n >> 1) & 1), wait_ns);
+                if (group_any(2, kChainThreads, !ok)) { failed = true; break; }
+            }
+            const int stop_now = *stop_at;   // includes chunk n + 1's decision (its prep is done)
             {
                 const bool ok = mbar_wait(bc1, ph1, wait_ns);
                 ph1 ^= 1u;
