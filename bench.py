@@ -540,6 +540,11 @@ def profile_case(g, args, stream):
         print(json.dumps({"profile_case": "decode", "workload": wl.describe(),
                           "us_per_step": 1e3 * ms / wl.decode_steps}))
         return
+    if args.profile_case == "chunk_fused":   # the headline shape at B = 2, fused prep + epilogue
+        wl = dataclasses.replace(W.BY_NAME[HEADLINE], B=2)
+        ms = bench_chunk_fused(g, wl, args.steps, args.warmup, 0, stream)
+        print(json.dumps({"profile_case": "chunk_fused", "workload": wl.describe(), "ms_per_call": ms}))
+        return
     base = W.BY_NAME[HEADLINE if args.profile_case == "chunk" else "chunk_bf16_negeig"]
     wl = dataclasses.replace(base, B=2 if base.d_v == 128 else 1)
     ms, d, _, _ = bench_chunk(g, wl, args.steps, args.warmup, 0, 1, stream)
@@ -606,7 +611,7 @@ def main():
     ap.add_argument("--steady-s", type=float, default=0.5,
                     help="after the timed steps, time rounds of 50 calls for at least this long (median reported)")
     ap.add_argument("--no-extras", action="store_true", help="skip decode/expanded-value/CPU legs")
-    ap.add_argument("--profile-case", choices=["chunk", "chunk_v256", "decode"], default=None,
+    ap.add_argument("--profile-case", choices=["chunk", "chunk_v256", "chunk_fused", "decode"], default=None,
                     help="only launch one kernel on a reduced batch (inputs still larger than L2), "
                          "for ncu captures; prints a short line")
     args = ap.parse_args()
