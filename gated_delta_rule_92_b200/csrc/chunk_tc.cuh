@@ -1293,16 +1293,17 @@ chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (progress) t0 = now;
                 else if (now - t0 > wait_ns) { failed = true; break; }
             }
-            if (!failed && lim < NC) {
-                // handed off: let every issued load land before the shared memory is reused
+            if (failed || lim < NC) {
+                // handed off, or stopped by a failed wait: let every issued load land
+                // (each wait bounded) before the shared memory is reused or released
                 // (the last load of each barrier slot completes that slot's last phase)
                 bool ok = true;
                 for (int j = max(0, nq - 2); j < nq; ++j)
-                    ok = ok && mbar_wait(&qb_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), wait_ns);
+                    ok &= mbar_wait(&qb_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), wait_ns);
                 for (int j = max(0, nk - 3); j < nk; ++j)
-                    ok = ok && mbar_wait(&k_full[j % 3], static_cast<uint32_t>((j / 3) & 1), wait_ns);
-                if (nv > 0) ok = ok && mbar_wait(v_full, static_cast<uint32_t>((nv - 1) & 1), wait_ns);
-                if (nw > 0) ok = ok && mbar_wait(w_full, static_cast<uint32_t>((nw - 1) & 1), wait_ns);
+                    ok &= mbar_wait(&k_full[j % 3], static_cast<uint32_t>((j / 3) & 1), wait_ns);
+                if (nv > 0) ok &= mbar_wait(v_full, static_cast<uint32_t>((nv - 1) & 1), wait_ns);
+                if (nw > 0) ok &= mbar_wait(w_full, static_cast<uint32_t>((nw - 1) & 1), wait_ns);
                 if (!ok) failed = true;
             }
         }
